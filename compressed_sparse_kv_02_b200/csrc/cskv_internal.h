@@ -1,0 +1,114 @@
+// cskv_internal.h -- parameter blocks and launchers shared by the C-ABI layer
+// (cskv_abi.cu) and the kernel files. Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "cskv.h"
+
+namespace cskv {
+
+// One stream of raw tokens folded into compressed entries (the latent-KV
+// stream, or the indexer-key stream of a CSA layer).
+struct FoldStream {
+  const uint16_t* x;      // new raw rows (bf16 bits)
+  const uint16_t* z;      // new gate-logit rows
+  const uint16_t* ring_x; // ring rows of the state cache (append path)
+  const uint16_t* ring_z;
+  uint16_t* ring_x_w;     // ring written by the append path
+  uint16_t* ring_z_w;
+  const float* bias;      // [m, d] or null
+  int d;                  // channels
+  int gc;                 // gate columns: 1 or d
+  int out_dtype;          // CSKV_BF16 / CSKV_FP8_E4M3 / CSKV_FP4_E2M1
+  void* pool;             // entry rows
+  float* scale_f32;       // FP8 per-entry scale
+  uint8_t* scale_e4m3;    // FP4 per-16 scale bytes
+};
+
+struct FoldParams {
+  FoldStream s[2];
+  int n_streams;
+  int m, n_win, page_size, max_pages_per_seq;
+  int64_t n_pages;
+  const int32_t* page_table;
+  int n_seq;
+  const int32_t* seq_ids;
+  int n_seqs_layer;
+  // bulk: rows [n_seq, n_tok, ...] starting at position tok0
+  int64_t tok0, n_tok;
+  // append: rows [n_seq, n_new, ...] starting at pos[b]
+  const int64_t* pos;
+  int n_new;
+  int ring_only;
+  int32_t* status;
+};
+
+cudaError_t launch_fold_bulk(const FoldParams& p, cudaStream_t st);
+cudaError_t launch_append(const FoldParams& p, cudaStream_t st);
+
+// Lightning indexer scan (scores of every visible entry) + top-k.
+struct IndexParams {
+  int n_q, n_heads_idx, d_idx, idx_dtype;
+  int m, n_win, page_size, max_pages_per_seq, n_seqs_layer;
+  int64_t n_pages;
+  const int32_t* page_table;
+  const void* idx_pool;
+  const uint8_t* idx_scale;
+  const int32_t* q_seq;
+  const int64_t* q_pos;
+  int64_t max_pos;
+  const void* q_idx;
+  const uint8_t* q_idx_scale;
+  const float* w;
+  int k;
+  int32_t* out_idx;
+  int32_t* out_cnt;
+  float* out_scores;
+  int32_t* status;
+  // workspace
+  float* scores;        // [n_q, vis_stride]
+  int64_t vis_stride;
+  int cluster;          // CTAs per query in the selection kernel
+  int slice;            // entries per CTA of the selection kernel
+};
+
+size_t index_ws_bytes(int n_q, int64_t max_pos, int m, int n_win);
+cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st);
+
+// Split-KV attention over window + compressed keys, then the LSE merge.
+struct AttendParams {
+  int is_csa;
+  int n_q, n_heads, d_qk, d_v, kv_dtype;
+  int m, n_win, page_size, max_pages_per_seq, n_seqs_layer;
+  int64_t n_pages;
+  const int32_t* page_table;
+  const void* kv_pool;
+  const float* kv_scale;
+  const uint16_t* ring_x;
+  const int32_t* q_seq;
+  const int64_t* q_pos;
+  int64_t max_pos;
+  const uint16_t* q;
+  const int32_t* sel_idx;
+  const int32_t* sel_cnt;
+  int k;
+  float sm_scale;
+  uint16_t* out;
+  float* lse;
+  const uint16_t* x_chunk;
+  int64_t chunk_pos0, chunk_len;
+  int32_t* status;
+  // workspace / plan
+  float* part_o;   // [n_q * max_splits * n_heads, d_v]
+  float* part_lse; // [n_q * max_splits * n_heads]
+  int max_splits;
+  int keys_per_split;
+};
+
+size_t attend_ws_bytes(const AttendParams& p, int n_sm);
+cudaError_t launch_attend(AttendParams& p, void* ws, int n_sm, cudaStream_t st);
+bool attend_supported(int d_qk, int d_v, int n_heads, int kv_dtype);
+
+}  // namespace cskv

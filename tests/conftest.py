@@ -23,3 +23,10 @@ def orc():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def cskv_built():
+    """Build libcskv.so in-tree if it is missing or stale (nvcc cross-compiles without a GPU)."""
+    from compressed_sparse_kv_02_b200 import build
+    return build.build()

@@ -1,0 +1,171 @@
+"""GPU parity: CSA / HCA core attention against the oracle (DeepSeek-V4
+report digest, section 3: one softmax over the n_win raw window tokens and
+the selected (CSA) or all visible (HCA) compressed entries; every head reads
+the same latent KV, V being its first d_v channels)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import (ATOL_BF16, ATOL_LP, REL_BF16, REL_LP, assert_close, layer_entries, make_layer,
+                         ring_window, stored_bf16)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ck(cskv_built):
+    import compressed_sparse_kv_02_b200 as ck
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return ck
+
+
+def _fill(ck, L, B, n_e, g, sharp, fp8=False):
+    std = 1.0 if sharp else 1.0 / math.sqrt(L.d_qk)
+    for b in range(B):
+        e = torch.randn(n_e, L.d_qk, generator=g) * std
+        if fp8:
+            amax = e.abs().amax(dim=1).clamp_min(1e-30)
+            scale = amax / 448.0
+            codes = (e / scale[:, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+            L.write_entries(b, 0, kv=codes.cuda(), kv_scale=scale.cuda())
+        else:
+            L.write_entries(b, 0, kv=e.to(torch.bfloat16).cuda())
+    L.ring_x.copy_((torch.randn(L.ring_x.shape, generator=g) * std).to(torch.bfloat16))
+
+
+def _run(ck, orc, kind, d_qk, d_v, H, positions, sharp=False, fp8=False, k=64, seed=0, with_lse=True,
+         sel_mode="random"):
+    B = len(positions)
+    m = 4 if kind == "csa" else 128
+    n_e = max(positions) // m + 2
+    L = make_layer(ck.LAYER_CSA if kind == "csa" else ck.LAYER_HCA, m, d_qk, d_v, B, n_e,
+                   d_idx=64 if kind == "csa" else 0, kv_dtype=ck.FP8_E4M3 if fp8 else ck.BF16, seed=seed)
+    g = torch.Generator().manual_seed(1000 + seed)
+    _fill(ck, L, B, n_e, g, sharp, fp8)
+    q = (torch.randn(B, H, d_qk, generator=g) * (math.sqrt(d_qk) if sharp else 1.0)).to(torch.bfloat16).cuda()
+    seq = torch.arange(B, dtype=torch.int32, device="cuda")
+    pos = torch.tensor(positions, dtype=torch.int64, device="cuda")
+    out = torch.zeros(B, H, d_v, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(B, H, device="cuda") if with_lse else None
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sel = None
+    if kind == "csa":
+        sel = torch.full((B, k), -1, dtype=torch.int32)
+        cnt = torch.zeros(B, dtype=torch.int32)
+        for b, t in enumerate(positions):
+            nv = orc.visible_entries(t, m, 128)
+            c = min(k, nv) if sel_mode == "random" else min(k, nv, 7)
+            ids = np.sort(np.random.default_rng(b + seed).choice(nv, c, replace=False)) if c else np.zeros(0, int)
+            sel[b, :c] = torch.from_numpy(ids.astype(np.int32))
+            cnt[b] = c
+        sel, cnt = sel.cuda(), cnt.cuda()
+        ck.csa_attend(L, seq, pos, max(positions), q, sel, cnt, out, lse, status=status)
+    else:
+        ck.hca_attend(L, seq, pos, max(positions), q, out, lse, status=status)
+    assert ck.cskv_get_status(status) == ck.OK
+    scale = 1.0 / math.sqrt(d_qk)
+    atol, rel = (ATOL_LP, REL_LP) if fp8 else (ATOL_BF16, REL_BF16)
+    got_o = out.float().cpu().numpy()
+    for b, t in enumerate(positions):
+        nv = orc.visible_entries(t, m, 128)
+        win = ring_window(L, b, t)
+        ent = layer_entries(L, b, max(nv, 1))["kv"]
+        qb = stored_bf16(q[b])
+        if kind == "csa":
+            c = int(cnt[b])
+            ids = sel[b, :c].cpu().numpy()
+            keys = np.vstack([orc.decode(win), orc.decode(ent)[ids]]) if c else orc.decode(win)
+            o, l = orc.attend(qb, orc.f64(keys), d_v, scale)
+        else:
+            o, l = orc.hca_query(t, m, 128, qb, win, ent if nv else ent.rows_subset(0, 0), d_v, scale)
+        assert_close(got_o[b], o, atol, rel, "%s o b=%d t=%d" % (kind, b, t))
+        if with_lse:
+            assert np.allclose(lse[b].cpu().numpy(), l, rtol=0, atol=2e-3), "lse b=%d" % b
+    return L
+
+
+@pytest.mark.parametrize("H", [16, 32, 64])
+def test_hca_d128(ck, orc, H):
+    _run(ck, orc, "hca", 128, 128, H, [3, 127, 128, 300, 128 * 40 + 77, 128 * 300 + 5], seed=H)
+
+
+@pytest.mark.parametrize("H", [16, 64, 128])
+def test_hca_latent_576(ck, orc, H):
+    _run(ck, orc, "hca", 576, 512, H, [127, 128 * 9 + 1, 128 * 700 + 127], seed=H + 1)
+
+
+@pytest.mark.parametrize("H", [16, 32])
+def test_csa_d128(ck, orc, H):
+    _run(ck, orc, "csa", 128, 128, H, [10, 130, 127 + 4 * 30, 127 + 4 * 5000 + 2], k=512, seed=H + 2)
+
+
+@pytest.mark.parametrize("H", [32, 128])
+def test_csa_latent_576(ck, orc, H):
+    _run(ck, orc, "csa", 576, 512, H, [200, 127 + 4 * 3000 + 1], k=1024, seed=H + 3)
+
+
+def test_sharp_inputs(ck, orc):
+    # q scaled by sqrt(d) and V ~ N(0,1): peaked softmax, outputs of order 1
+    _run(ck, orc, "hca", 128, 128, 32, [128 * 50 + 3, 700], sharp=True, seed=11)
+    _run(ck, orc, "csa", 576, 512, 64, [127 + 4 * 800], sharp=True, k=256, seed=12)
+
+
+def test_short_selection_and_no_lse(ck, orc):
+    _run(ck, orc, "csa", 128, 128, 16, [127 + 4 * 40, 127 + 4 * 9], k=64, seed=13, with_lse=False, sel_mode="short")
+
+
+@pytest.mark.parametrize("kind", ["csa", "hca"])
+def test_fp8_kv(ck, orc, kind):
+    _run(ck, orc, kind, 576, 512, 64, [127 + 128 * 30 + 3, 129], fp8=True, k=256, seed=14)
+
+
+def test_prefill_chunk_window(ck, orc):
+    # window rows of positions in the chunk come from x_chunk, older ones from the ring
+    B, d, H, m = 1, 128, 16, 128
+    t0, T = 1024, 64  # chunk positions 1024 .. 1087; the ring holds 896 .. 1023
+    L = make_layer(ck.LAYER_HCA, m, d, d, B, 16, seed=15)
+    g = torch.Generator().manual_seed(15)
+    _fill(ck, L, B, 16, g, sharp=True)
+    ring_pos = list(range(t0 - 128, t0))
+    x_chunk = (torch.randn(T, d, generator=g)).to(torch.bfloat16).cuda()
+    q = torch.randn(T, H, d, generator=g).to(torch.bfloat16).cuda()
+    pos = torch.arange(t0, t0 + T, dtype=torch.int64, device="cuda")
+    seq = torch.zeros(T, dtype=torch.int32, device="cuda")
+    out = torch.zeros(T, H, d, dtype=torch.bfloat16, device="cuda")
+    ck.hca_attend(L, seq, pos, t0 + T - 1, q, out, x_chunk=x_chunk, chunk_pos0=t0)
+    torch.cuda.synchronize()
+    ring = L.ring_x[0].cpu()
+    for i in range(0, T, 9):
+        t = t0 + i
+        rows = [ring[p % 128] if p < t0 else x_chunk[p - t0].cpu() for p in range(t - 127, t + 1)]
+        win = stored_bf16(torch.stack(rows))
+        nv = orc.visible_entries(t, m, 128)
+        ent = layer_entries(L, 0, nv)["kv"]
+        o, _ = orc.hca_query(t, m, 128, stored_bf16(q[i]), win, ent, d, 1.0 / math.sqrt(d))
+        assert_close(out[i].float().cpu().numpy(), o, ATOL_BF16, REL_BF16, "chunk row %d" % i)
+
+
+def test_invalid_selection_is_reported(ck, orc):
+    B, d, H, m, k = 1, 128, 16, 4, 8
+    t = 127 + 4 * 20
+    L = make_layer(ck.LAYER_CSA, m, d, d, B, 40, d_idx=64, seed=16)
+    g = torch.Generator().manual_seed(16)
+    _fill(ck, L, B, 40, g, sharp=False)
+    sel = torch.tensor([[0, 3, 25, -1, -1, -1, -1, -1]], dtype=torch.int32, device="cuda")  # 25 is not visible
+    cnt = torch.tensor([3], dtype=torch.int32, device="cuda")
+    q = torch.randn(B, H, d, generator=g).to(torch.bfloat16).cuda()
+    out = torch.zeros(B, H, d, dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ck.csa_attend(L, torch.zeros(1, dtype=torch.int32, device="cuda"), torch.tensor([t], device="cuda"), t, q, sel,
+                  cnt, out, status=status)
+    assert ck.cskv_get_status(status) == ck.ERR_OUT_OF_RANGE
+    # the bad key is masked: the output is attention over the window and entries 0 and 3
+    win = ring_window(L, 0, t)
+    ent = layer_entries(L, 0, 20)["kv"]
+    keys = np.vstack([orc.decode(win), orc.decode(ent)[[0, 3]]])
+    o, _ = orc.attend(stored_bf16(q[0]), orc.f64(keys), d, 1.0 / math.sqrt(d))
+    assert_close(out[0].float().cpu().numpy(), o, ATOL_BF16, REL_BF16, "masked")
