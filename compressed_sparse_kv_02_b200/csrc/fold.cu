@@ -5,12 +5,15 @@
 // step (report digest, section 7, Figure 6: window + not-yet-compressed
 // tokens).
 //
-// One warp folds one entry; lane l owns the 16-byte channel groups l, l+32,
-// l+64, ... (8 channels each), so every load is a coalesced 128-bit access
-// across the warp. The gate softmax runs online in fp32 (running max,
-// denominator and weighted sum per channel); the entry is rounded to its
-// storage type: bf16 (RNE), FP8 e4m3 with an fp32 scale per entry
-// (amax / 448), or FP4 e2m1 with an e4m3 scale per 16 channels (amax / 6).
+// Small blocks (CSA, m = 4) fold one entry per warp: lane l owns the 16-byte
+// channel groups l, l+32, l+64, ... (8 channels each), so every load is a
+// coalesced 128-bit access across the warp. Large blocks (HCA, m' = 128) and
+// the decode append fold one entry per CTA: threads split the entry over
+// (channel group, token slice) and merge their partial states in shared
+// memory. The gate softmax runs online in fp32 (running max, denominator and
+// weighted sum per channel); the entry is rounded to its storage type: bf16
+// (RNE), FP8 e4m3 with an fp32 scale per entry (amax / 448), or FP4 e2m1 with
+// an e4m3 scale per 16 channels (amax / 6).
 #include "cskv_device.cuh"
 #include "cskv_internal.h"
 
@@ -34,12 +37,12 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
   f[7] = __uint_as_float(v.w & 0xffff0000u);
 }
 
-// Fold channels [c0, c0+8) of one block. rows(i, xr, zr) yields token i's
-// raw row and gate row.
+// Online-softmax partial state of channels [c0, c0+8) over tokens i0 .. i1-1
+// of one block: running max, denominator and weighted sum (fp32). rows(i, xr,
+// zr) yields token i's raw row and gate row.
 template <class Rows>
-__device__ __forceinline__ void fold_group(const FoldStream& S, int m, int c0, Rows rows,
-                                           float (&out)[8]) {
-  float mx[8], den[8], acc[8];
+__device__ __forceinline__ void fold_partial(const FoldStream& S, int i0, int i1, int c0, Rows rows,
+                                             float (&mx)[8], float (&den)[8], float (&acc)[8]) {
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     mx[e] = -INFINITY;
@@ -47,7 +50,7 @@ __device__ __forceinline__ void fold_group(const FoldStream& S, int m, int c0, R
     acc[e] = 0.f;
   }
 #pragma unroll 4
-  for (int i = 0; i < m; ++i) {
+  for (int i = i0; i < i1; ++i) {
     const uint16_t* xr;
     const uint16_t* zr;
     rows(i, xr, zr);
@@ -77,32 +80,32 @@ __device__ __forceinline__ void fold_group(const FoldStream& S, int m, int c0, R
       acc[e] += p * xf[e];
     }
   }
+}
+
+// Fold channels [c0, c0+8) over tokens i0 .. i1-1 (a whole block) into out.
+template <class Rows>
+__device__ __forceinline__ void fold_group(const FoldStream& S, int m, int i0, int i1, int c0, Rows rows,
+                                           float (&out)[8]) {
+  float mx[8], den[8], acc[8];
+  fold_partial(S, i0, i1, c0, rows, mx, den, acc);
 #pragma unroll
   for (int e = 0; e < 8; ++e) out[e] = acc[e] / den[e];
 }
 
-// Fold one entry (whole warp) and store it at pool row `row` (-1: skip).
-template <class Rows>
-__device__ void fold_entry(const FoldStream& S, int m, int64_t row, Rows rows) {
-  const int lane = threadIdx.x & 31;
+// Round one entry to its storage type and store it at pool row `row`. The
+// calling threads hold 8 consecutive channels each: thread i of `n` holds
+// groups i, i + n, i + 2n, ... (up to kGroupsPerLane of them); `amax` is the
+// entry-wide max |value| (needed for FP8), already reduced by the caller.
+// Adjacent threads hold adjacent groups, so an FP4 16-channel block is the
+// pair (2q, 2q+1) of threads with the same parity pattern.
+__device__ __forceinline__ void store_groups(const FoldStream& S, int64_t row, int first, int stride,
+                                             const float (&v)[kGroupsPerLane][8], float amax) {
   const int G = S.d / 8;
-  float v[kGroupsPerLane][8];
-  float amax = 0.f;
-#pragma unroll
-  for (int gi = 0; gi < kGroupsPerLane; ++gi) {
-    const int grp = lane + 32 * gi;
-    if (grp < G) {
-      fold_group(S, m, grp * 8, rows, v[gi]);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[gi][e]));
-    }
-  }
-  if (row < 0) return;
   if (S.out_dtype == CSKV_BF16) {
     uint16_t* dst = static_cast<uint16_t*>(S.pool) + row * S.d;
 #pragma unroll
     for (int gi = 0; gi < kGroupsPerLane; ++gi) {
-      const int grp = lane + 32 * gi;
+      const int grp = first + stride * gi;
       if (grp < G) {
         uint4 o;
         o.x = pack_bf16(v[gi][0], v[gi][1]);
@@ -113,13 +116,11 @@ __device__ void fold_entry(const FoldStream& S, int m, int64_t row, Rows rows) {
       }
     }
   } else if (S.out_dtype == CSKV_FP8_E4M3) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
     const float s = amax > 0.f ? amax / 448.0f : 1.0f;
     uint8_t* dst = static_cast<uint8_t*>(S.pool) + row * S.d;
 #pragma unroll
     for (int gi = 0; gi < kGroupsPerLane; ++gi) {
-      const int grp = lane + 32 * gi;
+      const int grp = first + stride * gi;
       if (grp < G) {
         uint32_t w[2] = {0u, 0u};
 #pragma unroll
@@ -128,14 +129,14 @@ __device__ void fold_entry(const FoldStream& S, int m, int64_t row, Rows rows) {
           w[e >> 2] |= c << (8 * (e & 3));
         }
         *reinterpret_cast<uint2*>(dst + grp * 8) = make_uint2(w[0], w[1]);
+        if (grp == 0) S.scale_f32[row] = s;
       }
     }
-    if (lane == 0) S.scale_f32[row] = s;
-  } else {  // CSKV_FP4_E2M1: one e4m3 scale per 16 channels = lanes (2q, 2q+1)
+  } else {  // CSKV_FP4_E2M1: one e4m3 scale per 16 channels = groups (2q, 2q+1)
     uint8_t* dst = static_cast<uint8_t*>(S.pool) + row * (S.d / 2);
 #pragma unroll
     for (int gi = 0; gi < kGroupsPerLane; ++gi) {
-      const int grp = lane + 32 * gi;
+      const int grp = first + stride * gi;
       float a = 0.f;
       if (grp < G) {
 #pragma unroll
@@ -159,6 +160,91 @@ __device__ void fold_entry(const FoldStream& S, int m, int64_t row, Rows rows) {
   }
 }
 
+// Fold one entry with one warp (small m: every lane runs the m tokens of its
+// channel groups) and store it at pool row `row`.
+template <class Rows>
+__device__ void fold_entry_warp(const FoldStream& S, int m, int64_t row, Rows rows) {
+  const int lane = threadIdx.x & 31;
+  const int G = S.d / 8;
+  float v[kGroupsPerLane][8];
+  float amax = 0.f;
+#pragma unroll
+  for (int gi = 0; gi < kGroupsPerLane; ++gi) {
+    const int grp = lane + 32 * gi;
+    if (grp < G) {
+      fold_group(S, m, 0, m, grp * 8, rows, v[gi]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[gi][e]));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+  store_groups(S, row, lane, 32, v, amax);
+}
+
+// Fold one entry with the whole block (large m, or one entry per block):
+// thread t takes channel group t % G and token slice t / G; the partial
+// online-softmax states (max, denominator, weighted sum) of the slices are
+// merged through shared memory. `sm` holds 3 * blockDim.x * 8 floats.
+template <class Rows>
+__device__ void fold_entry_block(const FoldStream& S, int m, int64_t row, Rows rows, float* sm) {
+  const int G = S.d / 8;
+  const int t = threadIdx.x;
+  int ns = blockDim.x / G;  // token slices
+  if (ns > m) ns = m;
+  const int per = (m + ns - 1) / ns;
+  const int g = t % G, sl = t / G;
+  float* smx = sm;
+  float* sden = sm + blockDim.x * 8;
+  float* sacc = sm + 2 * blockDim.x * 8;
+  if (sl < ns) {
+    float mx[8], den[8], acc[8];
+    const int i0 = sl * per, i1 = min(m, i0 + per);
+    fold_partial(S, i0, i1, g * 8, rows, mx, den, acc);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      smx[(sl * G + g) * 8 + e] = mx[e];
+      sden[(sl * G + g) * 8 + e] = den[e];
+      sacc[(sl * G + g) * 8 + e] = acc[e];
+    }
+  }
+  __syncthreads();
+  // threads 0..G-1 merge the slices of their group (warps that hold no group still join the reductions)
+  float v[kGroupsPerLane][8];
+  float amax = 0.f;
+  if (t < G) {
+    float M[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) M[e] = -INFINITY;
+    for (int q = 0; q < ns; ++q)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) M[e] = fmaxf(M[e], smx[(q * G + t) * 8 + e]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float den = 0.f, acc = 0.f;
+      for (int q = 0; q < ns; ++q) {
+        const float mq = smx[(q * G + t) * 8 + e];
+        if (mq == -INFINITY) continue;
+        const float f = expf(mq - M[e]);
+        den += sden[(q * G + t) * 8 + e] * f;
+        acc += sacc[(q * G + t) * 8 + e] * f;
+      }
+      v[0][e] = acc / den;
+      amax = fmaxf(amax, fabsf(v[0][e]));
+    }
+  }
+  // entry-wide amax (FP8 scale): block reduction
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+  __syncthreads();
+  if ((t & 31) == 0) smx[t >> 5] = amax;
+  __syncthreads();
+  amax = 0.f;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) amax = fmaxf(amax, smx[w]);
+  if (t < ((G + 31) & ~31)) store_groups(S, row, t, G, v, amax);  // one group per thread (gi = 0)
+  __syncthreads();  // shared memory is reused by the next entry
+}
+
 // pool row of entry j of sequence seq, or -1 (and a status code) when the
 // page table points outside the pool
 __device__ __forceinline__ int64_t entry_row(const FoldParams& p, int seq, int64_t j) {
@@ -179,32 +265,63 @@ __device__ __forceinline__ int64_t entry_row(const FoldParams& p, int seq, int64
   return (int64_t)page * p.page_size + (j % p.page_size);
 }
 
-__global__ void __launch_bounds__(256) fold_bulk_kernel(FoldParams p) {
-  const int warps = blockDim.x / 32;
+constexpr int kWarpFoldMaxM = 16;  // up to this many tokens per entry one warp folds an entry
+constexpr int kBlockFoldThreads = 512;
+
+// rows of the bulk input: token i of entry jj of row block b
+struct BulkRows {
+  const FoldStream* S;
+  int64_t t0;
+  __device__ void operator()(int i, const uint16_t*& xr, const uint16_t*& zr) const {
+    xr = S->x + (t0 + i) * S->d;
+    zr = S->z + (t0 + i) * S->gc;
+  }
+};
+
+__device__ __forceinline__ void bulk_item(const FoldParams& p, int64_t it, int& si, int64_t& row, BulkRows& r) {
   const int64_t per_seq = p.n_tok / p.m;
-  const int64_t total = (int64_t)p.n_streams * p.n_seq * per_seq;
+  si = static_cast<int>(it / (p.n_seq * per_seq));
+  const int64_t rem = it % (p.n_seq * per_seq);
+  const int b = static_cast<int>(rem / per_seq);
+  const int64_t jj = rem % per_seq;
+  row = entry_row(p, p.seq_ids[b], p.tok0 / p.m + jj);
+  r.S = &p.s[si];
+  r.t0 = (int64_t)b * p.n_tok + jj * p.m;
+}
+
+// small m (CSA): one warp per entry
+__global__ void __launch_bounds__(256) fold_bulk_warp_kernel(FoldParams p) {
+  const int warps = blockDim.x / 32;
+  const int64_t total = (int64_t)p.n_streams * p.n_seq * (p.n_tok / p.m);
   for (int64_t it = (int64_t)blockIdx.x * warps + (threadIdx.x >> 5); it < total;
        it += (int64_t)gridDim.x * warps) {
-    const int si = static_cast<int>(it / (p.n_seq * per_seq));
-    const int64_t rem = it % (p.n_seq * per_seq);
-    const int b = static_cast<int>(rem / per_seq);
-    const int64_t jj = rem % per_seq;
-    const FoldStream& S = p.s[si];
-    const int64_t row = entry_row(p, p.seq_ids[b], p.tok0 / p.m + jj);
-    const int64_t t0 = (int64_t)b * p.n_tok + jj * p.m;
-    auto rows = [&](int i, const uint16_t*& xr, const uint16_t*& zr) {
-      xr = S.x + (t0 + i) * S.d;
-      zr = S.z + (t0 + i) * S.gc;
-    };
-    if (row >= 0) fold_entry(S, p.m, row, rows);
+    int si;
+    int64_t row;
+    BulkRows r;
+    bulk_item(p, it, si, row, r);
+    if (row >= 0) fold_entry_warp(p.s[si], p.m, row, r);
+  }
+}
+
+// large m (HCA): one block per entry, tokens split over thread slices
+__global__ void __launch_bounds__(kBlockFoldThreads) fold_bulk_block_kernel(FoldParams p) {
+  __shared__ float sm[3 * kBlockFoldThreads * 8];
+  const int64_t total = (int64_t)p.n_streams * p.n_seq * (p.n_tok / p.m);
+  for (int64_t it = blockIdx.x; it < total; it += gridDim.x) {
+    int si;
+    int64_t row;
+    BulkRows r;
+    bulk_item(p, it, si, row, r);
+    if (row >= 0) fold_entry_block(p.s[si], p.m, row, r, sm);  // row is uniform across the block
   }
 }
 
 // One CTA per sequence: copy the new rows into the ring, then fold every
-// block the new tokens complete (old rows from the ring, new rows from the
-// input; the slots written and the slots read never coincide because
-// n_new + m - 1 <= n_win).
-__global__ void __launch_bounds__(256) append_kernel(FoldParams p) {
+// block the new tokens complete, one entry at a time with the whole CTA (old
+// rows from the ring, new rows from the input; the slots written and the
+// slots read never coincide because n_new + m - 1 <= n_win).
+__global__ void __launch_bounds__(kBlockFoldThreads) append_kernel(FoldParams p) {
+  __shared__ float sm[3 * kBlockFoldThreads * 8];
   const int b = blockIdx.x;
   const int seq = p.seq_ids[b];
   if (seq < 0 || seq >= p.n_seqs_layer) {
@@ -232,8 +349,7 @@ __global__ void __launch_bounds__(256) append_kernel(FoldParams p) {
   const int64_t j_first = pos / p.m;                 // first block ending at or after pos
   const int64_t j_last = (pos + p.n_new) / p.m - 1;  // last block ending before pos+n_new
   const int64_t nb = j_last >= j_first ? j_last - j_first + 1 : 0;
-  const int warps = blockDim.x / 32;
-  for (int64_t it = threadIdx.x >> 5; it < nb * p.n_streams; it += warps) {
+  for (int64_t it = 0; it < nb * p.n_streams; ++it) {
     const int si = static_cast<int>(it / nb);
     const int64_t j = j_first + it % nb;
     const FoldStream& S = p.s[si];
@@ -249,7 +365,7 @@ __global__ void __launch_bounds__(256) append_kernel(FoldParams p) {
         zr = S.ring_z + ((int64_t)seq * p.n_win + slot) * S.gc;
       }
     };
-    if (row >= 0) fold_entry(S, p.m, row, rows);
+    if (row >= 0) fold_entry_block(S, p.m, row, rows, sm);  // row is uniform across the block
   }
 }
 
@@ -261,15 +377,20 @@ cudaError_t launch_fold_bulk(const FoldParams& p, cudaStream_t st) {
   int dev = 0, n_sm = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t want = (total + 7) / 8;
-  const int grid = static_cast<int>(want < (int64_t)n_sm * 8 ? want : (int64_t)n_sm * 8);
-  fold_bulk_kernel<<<grid, 256, 0, st>>>(p);
+  if (p.m <= kWarpFoldMaxM) {
+    const int64_t want = (total + 7) / 8;
+    const int grid = static_cast<int>(want < (int64_t)n_sm * 8 ? want : (int64_t)n_sm * 8);
+    fold_bulk_warp_kernel<<<grid, 256, 0, st>>>(p);
+  } else {
+    const int grid = static_cast<int>(total < (int64_t)n_sm * 4 ? total : (int64_t)n_sm * 4);
+    fold_bulk_block_kernel<<<grid, kBlockFoldThreads, 0, st>>>(p);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_append(const FoldParams& p, cudaStream_t st) {
   if (p.n_seq == 0 || p.n_new == 0) return cudaSuccess;
-  append_kernel<<<p.n_seq, 256, 0, st>>>(p);
+  append_kernel<<<p.n_seq, kBlockFoldThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 
