@@ -145,6 +145,8 @@ def run_ours(args, rank, world):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     cfg = synth.CONFIGS[args.config]
+    if args.batch:
+        cfg = synth.Config(**{**cfg.__dict__, "batch": args.batch})
     if rank:
         cfg = synth.Config(**{**cfg.__dict__, "seed": cfg.seed + 17 * rank})
     model = decode.DecodeModel(cfg, device="cuda")
@@ -444,6 +446,7 @@ def main():
     ap.add_argument("--config", default="pro")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling captures)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     world = int(os.environ.get("WORLD_SIZE", "1"))
