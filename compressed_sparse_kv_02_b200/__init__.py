@@ -10,7 +10,7 @@ from ._binding import (  # noqa: F401
     OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_OUT_OF_RANGE,
     SYMBOLS, CskvError, Layer, lib, status_string,
     csa_compress_kv, hca_compress_kv, cskv_cache_append,
-    csa_index_ws_bytes, csa_index_score_topk,
+    csa_index_ws_bytes, csa_index_score_topk, csa_index_score_topk_static,
     cskv_attend_ws_bytes, csa_attend, hca_attend,
     cskv_get_status, cskv_version,
 )

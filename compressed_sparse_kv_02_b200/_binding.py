@@ -96,6 +96,7 @@ SYMBOLS = {
     "cskv_cache_append": (_I32, [ctypes.POINTER(AppendArgs), _P]),
     "csa_index_ws_bytes": (_I32, [ctypes.POINTER(IndexArgs), ctypes.POINTER(ctypes.c_size_t)]),
     "csa_index_score_topk": (_I32, [ctypes.POINTER(IndexArgs), _P, ctypes.c_size_t, _P]),
+    "csa_index_score_topk_static": (_I32, [ctypes.POINTER(IndexArgs), _P]),
     "cskv_attend_ws_bytes": (_I32, [ctypes.POINTER(AttendArgs), ctypes.POINTER(ctypes.c_size_t)]),
     "csa_attend": (_I32, [ctypes.POINTER(AttendArgs), _P, ctypes.c_size_t, _P]),
     "hca_attend": (_I32, [ctypes.POINTER(AttendArgs), _P, ctypes.c_size_t, _P]),
@@ -386,6 +387,27 @@ def csa_index_score_topk(layer: Layer, q_seq, q_pos, max_pos: int, q_idx, w, k: 
     a = _index_args(layer, q_seq, q_pos, max_pos, q_idx, w, k, out_idx, out_cnt, out_scores, q_idx_scale, status)
     _check(lib().csa_index_score_topk(ctypes.byref(a), _ptr(workspace), workspace.numel(), _stream(stream)),
            "csa_index_score_topk")
+
+
+def csa_index_score_topk_static(layer: Layer, q_seq, q_pos, max_pos: int, q_idx, w, k: int, out_idx, out_cnt,
+                                out_scores=None, q_idx_scale=None, status=None, stream=None):
+    """csa_index_score_topk without a workspace: the library's fixed device scratch is used instead.
+
+    For callers that cannot allocate device memory where they call the indexer; the scratch
+    holds CSKV_STATIC_INDEX_SCRATCH_FLOATS scores, is shared by every call (overlapping calls
+    race), and is set up by the first call on each device, which should precede any stream capture.
+    """
+    if not layer.is_csa:
+        raise ValueError("csa_index_score_topk_static needs a CSA layer")
+    _need(w, "w", torch.float32)
+    n_q, h_i = w.shape
+    _need(q_seq, "q_seq", torch.int32, (n_q,))
+    _need(q_pos, "q_pos", torch.int64, (n_q,))
+    _need(out_idx, "out_idx", torch.int32, (n_q, k))
+    _need(out_cnt, "out_cnt", torch.int32, (n_q,))
+    _need(out_scores, "out_scores", torch.float32, (n_q, k), optional=True)
+    a = _index_args(layer, q_seq, q_pos, max_pos, q_idx, w, k, out_idx, out_cnt, out_scores, q_idx_scale, status)
+    _check(lib().csa_index_score_topk_static(ctypes.byref(a), _stream(stream)), "csa_index_score_topk_static")
 
 
 def _attend_args(layer, q_seq, q_pos, max_pos, q, sel_idx, sel_cnt, k, sm_scale, out, lse, x_chunk, chunk_pos0,

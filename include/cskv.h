@@ -245,6 +245,34 @@ cskv_status csa_index_score_topk(const cskv_index_args* args, void* workspace, s
                                  void* stream);
 
 /*
+ * csa_index_score_topk_static -- the same scores and selection as
+ * csa_index_score_topk, with no workspace argument and no allocation of any
+ * kind. The paper has no counterpart to this call; it exists for callers
+ * that cannot obtain device memory where they call the indexer: a plugin
+ * running inside a host engine that owns all device memory and offers its
+ * plugins no workspace, or a latency-critical loop that must not call
+ * cudaMalloc (which can synchronise the device and take unbounded time).
+ *   - Scratch: a file-scope device array of CSKV_STATIC_INDEX_SCRATCH_FLOATS
+ *     fp32 values (16 MiB) inside libcskv.so. Every GPU that loads the
+ *     library holds it until the process exits.
+ *   - Limit: a call needs csa_index_ws_bytes() bytes of it; a larger request
+ *     (n_q x the visible entries of max_pos, rounded up to 64) returns
+ *     CSKV_ERR_WORKSPACE and launches nothing.
+ *   - Set-up: the first call on each device looks up the array's device
+ *     address (cudaGetSymbolAddress) with that device current; make that
+ *     first call before any stream capture.
+ *   - Sharing: every call uses the same array and leaves its contents
+ *     behind. Nothing in it needs clearing (each call writes every score it
+ *     reads), but two calls that can run on the GPU at the same time -- on
+ *     unordered streams, or from several host threads -- race on it and
+ *     corrupt each other's results; order them on one stream or with events.
+ *   - Arguments, outputs and errors are otherwise those of
+ *     csa_index_score_topk.
+ */
+#define CSKV_STATIC_INDEX_SCRATCH_FLOATS (4u << 20)
+cskv_status csa_index_score_topk_static(const cskv_index_args* args, void* stream);
+
+/*
  * csa_attend / hca_attend -- core attention of one layer (report digest
  * section 3: one softmax over the window of the last n_win raw tokens and
  * the top-k entries (CSA) or all visible entries (HCA); DeepSeek-V4-book
