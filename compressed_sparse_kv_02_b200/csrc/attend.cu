@@ -394,10 +394,7 @@ cudaError_t run_attend(AttendParams& p, int n_sm, cudaStream_t st) {
   kern<<<static_cast<int>(grid), 32 * MT * VS, smem, st>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int hb = 256 / (p.d_v / 4);
-  dim3 mg(static_cast<unsigned>(p.n_q), static_cast<unsigned>((p.n_heads + hb - 1) / hb));
-  attend_merge_kernel<<<mg, 256, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_attend_merge(p, st);
 }
 
 // heads per CTA for each supported shape
@@ -415,6 +412,13 @@ Plan plan_for(int d_qk, int d_v, int n_heads) {
 }
 
 }  // namespace
+
+cudaError_t launch_attend_merge(AttendParams& p, cudaStream_t st) {
+  const int hb = 256 / (p.d_v / 4);
+  dim3 mg(static_cast<unsigned>(p.n_q), static_cast<unsigned>((p.n_heads + hb - 1) / hb));
+  attend_merge_kernel<<<mg, 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
 
 bool attend_supported(int d_qk, int d_v, int n_heads, int kv_dtype) {
   if (kv_dtype != CSKV_BF16 && kv_dtype != CSKV_FP8_E4M3) return false;
@@ -441,18 +445,26 @@ static void choose_split(AttendParams& p, int n_sm) {
 
 size_t attend_ws_bytes(const AttendParams& p0, int n_sm) {
   AttendParams p = p0;
-  choose_split(p, n_sm);
+  if (attend_tc_supported(p.d_qk, p.d_v, p.n_heads, p.kv_dtype))
+    attend_tc_plan(p, n_sm);
+  else
+    choose_split(p, n_sm);
   const size_t rows = (size_t)p.n_q * p.max_splits * p.n_heads;
   return rows * p.d_v * sizeof(float) + rows * sizeof(float) + 256;
 }
 
 cudaError_t launch_attend(AttendParams& p, void* ws, int n_sm, cudaStream_t st) {
-  choose_split(p, n_sm);
+  const bool tc = attend_tc_supported(p.d_qk, p.d_v, p.n_heads, p.kv_dtype);
+  if (tc)
+    attend_tc_plan(p, n_sm);
+  else
+    choose_split(p, n_sm);
   if (p.n_q > kMaxQ) return cudaErrorNotSupported;
   const size_t rows = (size_t)p.n_q * p.max_splits * p.n_heads;
   p.part_o = static_cast<float*>(ws);
   p.part_lse = p.part_o + rows * p.d_v;
   if (p.n_q == 0) return cudaSuccess;
+  if (tc) return launch_attend_tc(p, n_sm, st);
   const Plan pl = plan_for(p.d_qk, p.d_v, p.n_heads);
   const bool fp8 = p.kv_dtype == CSKV_FP8_E4M3;
   if (p.d_qk == 128 && p.d_v == 128) {

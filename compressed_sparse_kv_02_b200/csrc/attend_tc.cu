@@ -1,0 +1,374 @@
+// attend_tc.cu -- CSA / HCA core attention on the 5th-generation tensor cores
+// (tcgen05) for the wide shared latent: d_qk = 576 (512 latent + 64 RoPE
+// channels), d_v = 512, query heads in groups of 128 (DeepSeek-V4 report
+// digest, section 3: one softmax over the window and the selected / all
+// compressed entries; DeepSeek-V4-book ch.1, section 4: the MLA latent shared
+// by every head).
+//
+// With 128 heads on one 576-wide latent every key carries 2 x 128 x 1088
+// flops: the product is a real dense contraction, with the heads as M = 128.
+// Work item = (query, 128-head group, key split, half of d_v). Per item:
+//   - Q [128 heads x 576] sits in shared memory as nine 128-byte-swizzled
+//     K-major blocks of 64 channels; 32-key tiles of K stream through two
+//     swizzled buffers (cp.async gathers through the page table);
+//   - S = Q K^T (M 128, N 32, K 576: 36 tcgen05.mma) lands in tensor memory;
+//   - four warps take one head row each from S (tcgen05.ld), run the online
+//     softmax in fp32 and write P (bf16) back to tensor memory;
+//   - O[:, half] += P V (M 128, N 256, K 32) with P as the tensor-memory A
+//     operand and V read MN-major from the same K tile (V = the first d_v
+//     channels of each key);
+//   - O is rescaled only when a row's running max rises by more than 2^8 (the
+//     probabilities stay below 256 in bf16), so most tiles skip it.
+// The two d_v halves of a (query, split) run in two CTAs that both compute S
+// (the accumulator for all 512 output channels would fill the whole tensor
+// memory). Each item writes its normalised partial output and log-sum-exp;
+// attend_merge_kernel combines the splits.
+#include "cskv_device.cuh"
+#include "cskv_internal.h"
+
+namespace cskv {
+
+// defined in attend.cu
+cudaError_t launch_attend_merge(AttendParams& p, cudaStream_t st);
+
+namespace {
+
+constexpr int kDqk = 576, kDv = 512, kM = 128, kNk = 32;
+constexpr int kKb = kDqk / 64;                // 64-channel (128-byte) blocks per row
+constexpr int kQBytes = kKb * kM * 128;       // 147456
+constexpr int kKBytes = kKb * kNk * 128;      // 36864 per key tile
+constexpr int kThreads = 256;
+constexpr int kMmaThread = 128;               // warp 4, lane 0 issues the tensor-core work
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 0, kColS = 256, kColP = 288;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;     // log2 units
+
+struct Smem {
+  static constexpr int Q = 0;
+  static constexpr int K = kQBytes;                 // two tile buffers
+  static constexpr int BAR = K + 2 * kKBytes;       // bar_s, bar_o
+  static constexpr int SCALE = BAR + 64;            // [2][kNk] key weight: 1 valid, 0 masked
+  static constexpr int TMEM = SCALE + 2 * kNk * 4;  // allocated tensor-memory address
+  static constexpr int FLAGS = TMEM + 16;
+  static constexpr int PREF = FLAGS + 16;
+  static size_t bytes(int n_q) { return 1024 + PREF + sizeof(int) * (size_t)(n_q + 1); }
+};
+
+struct Keys {
+  int64_t t, ws;
+  int n_w;
+  int64_t n;
+};
+
+__device__ __forceinline__ Keys keys_of(const AttendParams& p, int b) {
+  Keys r;
+  r.t = p.q_pos[b];
+  r.ws = 0;
+  r.n_w = 0;
+  r.n = 0;
+  if (r.t < 0 || r.t > p.max_pos) return r;
+  r.ws = window_start(r.t, p.n_win);
+  r.n_w = static_cast<int>(r.t - r.ws + 1);
+  int64_t n_c;
+  if (p.is_csa) {
+    const int64_t c = p.sel_cnt[b];
+    n_c = c < 0 ? 0 : (c > p.k ? p.k : c);
+  } else {
+    n_c = visible_entries(r.t, p.m, p.n_win);
+  }
+  r.n = r.n_w + n_c;
+  return r;
+}
+
+// source row of key u (window rows first, then compressed entries); null if invalid
+__device__ __forceinline__ const uint16_t* key_src(const AttendParams& p, int b, int seq, const Keys& k,
+                                                   int64_t u) {
+  if (u < k.n_w) {
+    const int64_t pos = k.ws + u;
+    if (p.x_chunk && pos >= p.chunk_pos0 && pos < p.chunk_pos0 + p.chunk_len)
+      return p.x_chunk + (pos - p.chunk_pos0) * kDqk;
+    return p.ring_x + ((int64_t)seq * p.n_win + pos % p.n_win) * kDqk;
+  }
+  const int64_t jj = u - k.n_w;
+  const int64_t j = p.is_csa ? static_cast<int64_t>(p.sel_idx[(int64_t)b * p.k + jj]) : jj;
+  if (j < 0 || j >= visible_entries(k.t, p.m, p.n_win)) return nullptr;
+  const int64_t pi = j / p.page_size;
+  if (pi >= p.max_pages_per_seq) return nullptr;
+  const int32_t page = p.page_table[(int64_t)seq * p.max_pages_per_seq + pi];
+  if (page < 0 || page >= p.n_pages) return nullptr;
+  return static_cast<const uint16_t*>(p.kv_pool) + ((int64_t)page * p.page_size + j % p.page_size) * kDqk;
+}
+
+// byte offset of 16-byte chunk `ch` (0..71) of row `r` in a swizzled block set
+// whose 64-channel blocks are `block_bytes` apart
+__device__ __forceinline__ uint32_t swz(int r, int ch, int block_bytes) {
+  return (ch >> 3) * block_bytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = sm + Smem::Q;
+  uint8_t* sK = sm + Smem::K;
+  uint64_t* bar_s = reinterpret_cast<uint64_t*>(sm + Smem::BAR);
+  uint64_t* bar_o = bar_s + 1;
+  float* sScale = reinterpret_cast<float*>(sm + Smem::SCALE);
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + Smem::TMEM);
+  int* sAbort = reinterpret_cast<int*>(sm + Smem::FLAGS);
+  int* sPref = reinterpret_cast<int*>(sm + Smem::PREF);
+  __shared__ int s_wsum[32];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int groups = p.n_heads / kM;
+  const int kps = p.keys_per_split;
+
+  {  // items per query: splits x head groups x 2 halves of d_v
+    int run = 0;
+    for (int base = 0; base < p.n_q; base += kThreads) {
+      const int b = base + tid;
+      int v = 0;
+      if (b < p.n_q) {
+        const Keys k = keys_of(p, b);
+        v = static_cast<int>((k.n + kps - 1) / kps) * groups * 2;
+      }
+      int tot;
+      const int ex = block_exclusive_scan<kThreads>(v, s_wsum, tot);
+      if (b < p.n_q) sPref[b] = run + ex;
+      run += tot;
+    }
+    if (tid == 0) sPref[p.n_q] = run;
+  }
+  if (tid == 0) {
+    mbar_init(bar_s, 1);
+    mbar_init(bar_o, 1);
+    fence_barrier_init();
+    *sAbort = 0;
+  }
+  if (warp == 4) {
+    tmem_alloc(sTmem, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sTmem;
+  if (blockIdx.x == 0)
+    for (int b = tid; b < p.n_q; b += kThreads)
+      if (p.q_pos[b] < 0 || p.q_pos[b] > p.max_pos) report(p.status, CSKV_ERR_INVALID_ARG);
+  const int total = sPref[p.n_q];
+  const float sl2 = p.sm_scale * kLog2e;
+  const uint32_t idesc_s = umma_idesc_bf16(kM, kNk, false);
+  const uint32_t idesc_pv = umma_idesc_bf16(kM, 256, true);
+  const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK);
+  uint32_t g = 0;  // tiles processed by this CTA so far (mbarrier phases)
+
+  for (int item = blockIdx.x; item < total; item += gridDim.x) {
+    int lo = 0, hi = p.n_q - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sPref[mid] <= item) lo = mid; else hi = mid - 1;
+    }
+    const int b = lo;
+    const int r = item - sPref[b];
+    const int vh = r & 1;
+    const int grp = (r >> 1) % groups;
+    const int split = (r >> 1) / groups;
+    const Keys kk = keys_of(p, b);
+    const int seq = p.q_seq[b];
+    const bool seq_ok = seq >= 0 && seq < p.n_seqs_layer;
+    const int64_t u0 = (int64_t)split * kps;
+    const int nk = static_cast<int>(kk.n - u0 < kps ? kk.n - u0 : kps);
+    const int ntiles = (nk + kNk - 1) / kNk;
+
+    // ---- loads: Q rows (thread: one head row, half of its 72 chunks), key tiles (thread: one key row, 9 chunks)
+    {
+      const int qr = tid >> 1, half = tid & 1;
+      const uint16_t* src = p.q + ((int64_t)b * p.n_heads + grp * kM + qr) * kDqk;
+      for (int c = half * 36; c < half * 36 + 36; ++c) cp_async16(sQ + swz(qr, c, kM * 128), src + c * 8, 16);
+    }
+    auto issue_tile = [&](int it, int buf) {
+      const int kr = tid >> 3, part = tid & 7;
+      const int i = it * kNk + kr;
+      const uint16_t* src = nullptr;
+      if (i < nk && seq_ok) src = key_src(p, b, seq, kk, u0 + i);
+      if (i < nk && !src) report(p.status, CSKV_ERR_OUT_OF_RANGE);
+      if (part == 0) sScale[buf * kNk + kr] = src ? 1.f : 0.f;
+      uint8_t* dst = sK + buf * kKBytes;
+#pragma unroll
+      for (int q = 0; q < 9; ++q) {
+        const int c = part * 9 + q;
+        cp_async16(dst + swz(kr, c, kNk * 128), src ? static_cast<const void*>(src + c * 8) : p.q, src ? 16 : 0);
+      }
+      cp_async_commit();
+    };
+    issue_tile(0, 0);
+
+    float m_used = -INFINITY, l_run = 0.f;  // softmax state of this thread's head row (warps 0-3)
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    bool aborted = false;
+    for (int it = 0; it < ntiles; ++it) {
+      const int buf = it & 1;
+      const uint32_t gt = g + it;
+      if (it + 1 < ntiles) {
+        // buffer buf^1 was last read by the PV of tile it-1
+        if (it >= 1 && !mbar_wait(bar_o, (gt - 1) & 1u, p.status)) *sAbort = 1;
+        issue_tile(it + 1, buf ^ 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      fence_proxy_async_smem();
+      __syncthreads();
+      if (*sAbort) { aborted = true; break; }
+      tc_fence_after();
+      if (tid == kMmaThread) {
+        const uint32_t kb_base = sKa + buf * kKBytes;
+#pragma unroll 1
+        for (int kb = 0; kb < kKb; ++kb) {
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t da = umma_desc_sw128(sQa + kb * (kM * 128) + ks * 32, 16, 1024);
+            const uint64_t db = umma_desc_sw128(kb_base + kb * (kNk * 128) + ks * 32, 16, 1024);
+            umma_ss(tmem + kColS, da, db, idesc_s, (kb | ks) != 0);
+          }
+        }
+        umma_commit(bar_s);
+      }
+      if (warp < 4) {
+        bool ok = mbar_wait(bar_s, gt & 1u, p.status);
+        tc_fence_after();
+        uint32_t sr[32];
+        tmem_ld32(tmem + lane_base + kColS, sr);
+        tmem_ld_wait();
+        float v[32];
+        float mt = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float w = sScale[buf * kNk + j];
+          v[j] = (it * kNk + j < nk && w != 0.f) ? __uint_as_float(sr[j]) * sl2 * w : -INFINITY;
+          mt = fmaxf(mt, v[j]);
+        }
+        float corr = 1.f;
+        bool rescale = false;
+        if (mt > m_used + kRescaleThreshold || (m_used == -INFINITY && mt != -INFINITY)) {
+          corr = exp2f(m_used - mt);  // 0 when m_used is -inf
+          rescale = it > 0;
+          l_run *= corr;
+          m_used = mt;
+        }
+        const float msub = m_used == -INFINITY ? 0.f : m_used;
+        uint32_t pp[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float p0 = exp2f(v[2 * j] - msub), p1 = exp2f(v[2 * j + 1] - msub);
+          l_run += p0 + p1;
+          pp[j] = pack_bf16(p0, p1);
+        }
+        // the previous tile's P V must be done before P and O are rewritten
+        if (it >= 1) ok = mbar_wait(bar_o, (gt - 1) & 1u, p.status) && ok;
+        tc_fence_after();
+        if (__any_sync(kFull, rescale)) {
+#pragma unroll 1
+          for (int c = 0; c < 256; c += 32) {
+            uint32_t orow[32];
+            tmem_ld32(tmem + lane_base + kColO + c, orow);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) orow[j] = __float_as_uint(__uint_as_float(orow[j]) * corr);
+            tmem_st32(tmem + lane_base + kColO + c, orow);
+          }
+        }
+        tmem_st16(tmem + lane_base + kColP, pp);
+        tmem_st_wait();
+        if (!ok) *sAbort = 1;
+      }
+      tc_fence_before();
+      __syncthreads();
+      if (*sAbort) { aborted = true; break; }
+      tc_fence_after();
+      if (tid == kMmaThread) {
+        const uint32_t v_base = sKa + buf * kKBytes + vh * 4 * (kNk * 128);
+#pragma unroll
+        for (int k2 = 0; k2 < 2; ++k2) {
+          const uint64_t db = umma_desc_sw128(v_base + k2 * 16 * 128, kNk * 128, 1024);
+          umma_ts(tmem + kColO, tmem + kColP + k2 * 8, db, idesc_pv, (it > 0 || k2 > 0) ? 1u : 0u);
+        }
+        umma_commit(bar_o);
+      }
+    }
+    if (aborted) break;
+    // ---- epilogue: normalised partial output of this split and half, and its log-sum-exp
+    if (warp < 4) {
+      if (!mbar_wait(bar_o, (g + ntiles - 1) & 1u, p.status)) *sAbort = 1;
+      tc_fence_after();
+      const int head = grp * kM + warp * 32 + lane;
+      const int64_t prow = ((int64_t)b * p.max_splits + split) * p.n_heads + head;
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      float* dst = p.part_o + prow * kDv + vh * 256;
+#pragma unroll 1
+      for (int c = 0; c < 256; c += 32) {
+        uint32_t orow[32];
+        tmem_ld32(tmem + lane_base + kColO + c, orow);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(dst + c + j) =
+              make_float4(__uint_as_float(orow[j]) * inv, __uint_as_float(orow[j + 1]) * inv,
+                          __uint_as_float(orow[j + 2]) * inv, __uint_as_float(orow[j + 3]) * inv);
+      }
+      if (vh == 0) p.part_lse[prow] = l_run > 0.f ? (m_used + log2f(l_run)) * kLn2 : -INFINITY;
+    }
+    g += ntiles;
+    tc_fence_before();
+    __syncthreads();  // shared and tensor memory are reused by the next item
+    if (*sAbort) break;
+  }
+  // on an abort, give outstanding tensor-core work a bounded chance to finish before freeing
+  if (*sAbort && tid == kMmaThread) {
+    mbar_wait(bar_s, (g + 1) & 1u, nullptr);
+    mbar_wait(bar_o, (g + 1) & 1u, nullptr);
+  }
+  cp_async_wait<0>();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 4) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+bool attend_tc_supported(int d_qk, int d_v, int n_heads, int kv_dtype) {
+  return d_qk == kDqk && d_v == kDv && n_heads % kM == 0 && kv_dtype == CSKV_BF16;
+}
+
+// keys per split: queries x head groups x splits x 2 halves ~ one CTA per SM
+void attend_tc_plan(AttendParams& p, int n_sm) {
+  const int64_t groups = p.n_heads / kM;
+  const int64_t n_max = (int64_t)p.n_win + (p.is_csa ? p.k : visible_entries(p.max_pos, p.m, p.n_win));
+  int64_t splits = n_sm / ((int64_t)p.n_q * groups * 2);
+  if (splits < 1) splits = 1;
+  int64_t kps = (n_max + splits - 1) / splits;
+  kps = (kps + kNk - 1) / kNk * kNk;
+  if (kps < kNk) kps = kNk;
+  p.keys_per_split = static_cast<int>(kps);
+  p.max_splits = static_cast<int>((n_max + kps - 1) / kps);
+  if (p.max_splits < 1) p.max_splits = 1;
+}
+
+cudaError_t launch_attend_tc(AttendParams& p, int n_sm, cudaStream_t st) {
+  const size_t smem = Smem::bytes(p.n_q);
+  cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t upper = (int64_t)p.n_q * p.max_splits * (p.n_heads / kM) * 2;
+  int64_t grid = upper < n_sm ? upper : n_sm;
+  if (grid < 1) grid = 1;
+  attend_tc_kernel<<<static_cast<int>(grid), kThreads, smem, st>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_attend_merge(p, st);
+}
+
+}  // namespace cskv

@@ -21,6 +21,7 @@
 // summed through distributed shared memory, and writes the chosen indices in
 // ascending order (equal scores prefer the lower index).
 #include <cooperative_groups.h>
+#include <cudaTypedefs.h>
 
 #include "cskv_device.cuh"
 #include "cskv_internal.h"
@@ -34,6 +35,7 @@ constexpr int kScanThreads = 256;
 constexpr int kMaxQueries = 4096;  // queries per call (prefix table in shared memory)
 constexpr int kSelThreads = 1024;
 constexpr int kSliceCap = 40960;   // scores per CTA of the selection kernel
+constexpr int kMaxCluster = 16;   // CTAs per query in the selection kernel (above 8: non-portable)
 
 __device__ __forceinline__ int64_t query_visible(const IndexParams& p, int b) {
   const int64_t t = p.q_pos[b];
@@ -291,6 +293,228 @@ __global__ void __launch_bounds__(kScanThreads, 2) index_scan_kernel(IndexParams
   }
 }
 
+// ---------------------------------------------------------------- TMA-fed scan
+// bf16 keys on pages of a multiple of 64 entries. One persistent CTA per SM:
+// warp 0 issues 2D TMA loads of 64-key units (rows of d_idx bf16, boxes of 64
+// rows x 128 bytes with the 128-byte swizzle) into an NSTAGE-deep ring of
+// shared-memory stages; consumer warps 1..16, in four groups of four that take
+// every fourth unit, each run one 16-key sub-tile of a unit through mma.sync.
+// Under the swizzle, 16-byte chunk ch of row r sits at chunk ch ^ (r % 8) of
+// its 128-byte row. A quarter-warp reads the same logical chunks of two rows;
+// those rows are chosen 4 apart (fragment row g -> key (g >> 1) + 4 (g & 1))
+// so that the two land on disjoint halves of the 128-byte row and every
+// 128-bit shared load is conflict-free.
+constexpr int kTmaConsumerWarps = 16;  // four groups of four warps
+constexpr int kTmaThreads = 32 * (1 + kTmaConsumerWarps);
+constexpr int kUnitKeys = 64;
+constexpr int kTmaRingBytes = 128 * 1024;
+
+template <int NCH>
+struct TmaScanShape {
+  static constexpr int ROWB = NCH * 64;                     // bytes per key row
+  static constexpr int STAGE_BYTES = kUnitKeys * ROWB;      // one 64-key unit
+  static constexpr int NSTAGE = kTmaRingBytes / STAGE_BYTES;  // even
+  static size_t smem_bytes(int n_q) {
+    return 1024 + (size_t)kTmaRingBytes + 2 * NSTAGE * sizeof(uint64_t) + NSTAGE * sizeof(int) +
+           sizeof(int) * (size_t)(n_q + 1);
+  }
+};
+
+template <int NCH, int NTH>
+__global__ void __launch_bounds__(kTmaThreads, 1)
+    index_scan_tma_kernel(const __grid_constant__ CUtensorMap tmap, IndexParams p) {
+  using Sh = TmaScanShape<NCH>;
+  constexpr int NSTAGE = Sh::NSTAGE;
+  constexpr int NGROUP = kTmaConsumerWarps / 4;
+  static_assert(NSTAGE % NGROUP == 0, "each consumer group owns a fixed set of stages");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(tiles + kTmaRingBytes);
+  uint64_t* empty = full + NSTAGE;
+  int* s_valid = reinterpret_cast<int*>(empty + NSTAGE);
+  int* s_pref = s_valid + NSTAGE;
+  __shared__ int s_wsum[32];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  {  // 64-key units per query, exclusive prefix
+    int run = 0;
+    for (int base = 0; base < p.n_q; base += kTmaThreads) {
+      const int b = base + tid;
+      int u = 0;
+      if (b < p.n_q) {
+        const int64_t nv = query_visible(p, b);
+        u = nv > 0 ? static_cast<int>((nv + kUnitKeys - 1) / kUnitKeys) : 0;
+      }
+      int tot;
+      const int ex = block_exclusive_scan<kTmaThreads>(u, s_wsum, tot);
+      if (b < p.n_q) s_pref[b] = run + ex;
+      run += tot;
+    }
+    if (tid == 0) s_pref[p.n_q] = run;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 4);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (blockIdx.x == 0)
+    for (int b = tid; b < p.n_q; b += kTmaThreads)
+      if (query_visible(p, b) < 0) report(p.status, CSKV_ERR_INVALID_ARG);
+
+  const int64_t total = s_pref[p.n_q];
+  const int64_t u_begin = total * blockIdx.x / gridDim.x;
+  const int64_t n_units = total * (blockIdx.x + 1) / gridDim.x - u_begin;
+  auto locate = [&](int64_t u, int& b, int64_t& j0) {
+    int lo = 0, hi = p.n_q - 1;  // last b with s_pref[b] <= u
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_pref[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    b = lo;
+    j0 = (u - s_pref[lo]) * kUnitKeys;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    // The warp resolves the pool rows of 32 units at a time (one page-table
+    // load per lane, in parallel); lane 0 then issues their loads in order.
+    if (lane == 0) prefetch_tensormap(&tmap);
+    int64_t issued = 0;
+    bool ok = true;
+    for (int64_t i0 = 0; i0 < n_units && ok; i0 += 32) {
+      int row0 = -1;
+      if (i0 + lane < n_units) {
+        int b;
+        int64_t j0;
+        locate(u_begin + i0 + lane, b, j0);
+        const int seq = p.q_seq[b];
+        const int64_t pi = j0 / p.page_size;
+        int32_t page = -1;
+        if (seq >= 0 && seq < p.n_seqs_layer && pi < p.max_pages_per_seq)
+          page = p.page_table[(int64_t)seq * p.max_pages_per_seq + pi];
+        if (page >= 0 && page < p.n_pages) row0 = static_cast<int>((int64_t)page * p.page_size + (j0 % p.page_size));
+      }
+      const int nb = static_cast<int>(n_units - i0 < 32 ? n_units - i0 : 32);
+      for (int k = 0; k < nb; ++k) {
+        const int r0 = __shfl_sync(kFull, row0, k);
+        if (lane == 0) {
+          const int64_t i = i0 + k;
+          const int s = static_cast<int>(i % NSTAGE);
+          const uint32_t round = static_cast<uint32_t>(i / NSTAGE);
+          if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, p.status)) {
+            ok = false;
+          } else {
+            if (r0 >= 0) {
+              s_valid[s] = 1;
+              mbar_arrive_expect_tx(&full[s], Sh::STAGE_BYTES);
+#pragma unroll
+              for (int box = 0; box < Sh::ROWB / 128; ++box)
+                tma_load_2d(tiles + (size_t)s * Sh::STAGE_BYTES + box * (kUnitKeys * 128), &tmap, box * 64, r0,
+                            &full[s]);
+            } else {
+              report(p.status, CSKV_ERR_OUT_OF_RANGE);
+              s_valid[s] = 0;
+              mbar_arrive(&full[s]);
+            }
+            issued = i + 1;
+          }
+        }
+        ok = __shfl_sync(kFull, ok, 0);
+        if (!ok) break;
+      }
+    }
+    // drain: every load issued must land before the CTA may exit
+    if (lane == 0)
+      for (int64_t r = issued > NSTAGE ? issued - NSTAGE : 0; r < issued; ++r)
+        mbar_wait(&full[r % NSTAGE], static_cast<uint32_t>((r / NSTAGE) & 1), p.status);
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int cw = warp - 1, group = cw >> 2, sub = cw & 3;
+  const int g = lane >> 2, c = lane & 3;
+  const int pg = (g >> 1) + 4 * (g & 1);  // physical row of fragment row g within its 8-row half
+  uint4 qf[NTH][NCH];
+  float wv[NTH][2];
+  int cur_b = -1;
+  for (int64_t i = group; i < n_units; i += NGROUP) {
+    const int s = static_cast<int>(i % NSTAGE);
+    const uint32_t round = static_cast<uint32_t>(i / NSTAGE);
+    if (!mbar_wait(&full[s], round & 1u, p.status)) break;
+    int b;
+    int64_t j0;
+    locate(u_begin + i, b, j0);
+    if (b != cur_b) {
+      cur_b = b;
+#pragma unroll
+      for (int nt = 0; nt < NTH; ++nt) {
+        const int n = 8 * nt + g;
+        const uint16_t* qr = static_cast<const uint16_t*>(p.q_idx) + ((int64_t)b * p.n_heads_idx + n) * p.d_idx;
+#pragma unroll
+        for (int jj = 0; jj < NCH; ++jj)
+          qf[nt][jj] = n < p.n_heads_idx ? ldg16(qr + (c + 4 * jj) * 8) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int h = 8 * nt + 2 * c + e;
+          wv[nt][e] = h < p.n_heads_idx ? p.w[(int64_t)b * p.n_heads_idx + h] : 0.f;
+        }
+      }
+    }
+    const int64_t nv = query_visible(p, b);
+    const int64_t j = j0 + 16 * sub;  // this warp's 16 keys
+    if (j < nv) {
+      float s0 = -INFINITY, s1 = -INFINITY;
+      if (s_valid[s]) {
+        const uint8_t* tb = tiles + (size_t)s * Sh::STAGE_BYTES;
+        const int r0 = 16 * sub + pg;  // rows r0 and r0 + 8 (same swizzle phase)
+        // two independent accumulation chains (k-steps h = 0 and h = 1), summed at the end
+        float acc[2][NTH][4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int nt = 0; nt < NTH; ++nt) acc[h][nt][0] = acc[h][nt][1] = acc[h][nt][2] = acc[h][nt][3] = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < NCH; ++jj) {
+          const int q = c + 4 * jj;
+          const int off = (q >> 3) * (kUnitKeys * 128) + (((q & 7) ^ pg) << 4);
+          const uint4 ka = lds16(tb + off + r0 * 128);
+          const uint4 kb = lds16(tb + off + (r0 + 8) * 128);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t a[4] = {u4_at(ka, 2 * h), u4_at(kb, 2 * h), u4_at(ka, 2 * h + 1), u4_at(kb, 2 * h + 1)};
+#pragma unroll
+            for (int nt = 0; nt < NTH; ++nt)
+              mma_bf16(acc[h][nt], a, u4_at(qf[nt][jj], 2 * h), u4_at(qf[nt][jj], 2 * h + 1));
+          }
+        }
+        s0 = 0.f;
+        s1 = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < NTH; ++nt) {
+          const float d0 = acc[0][nt][0] + acc[1][nt][0], d1 = acc[0][nt][1] + acc[1][nt][1];
+          const float d2 = acc[0][nt][2] + acc[1][nt][2], d3 = acc[0][nt][3] + acc[1][nt][3];
+          s0 += wv[nt][0] * fmaxf(d0, 0.f) + wv[nt][1] * fmaxf(d1, 0.f);
+          s1 += wv[nt][0] * fmaxf(d2, 0.f) + wv[nt][1] * fmaxf(d3, 0.f);
+        }
+        s0 += __shfl_xor_sync(kFull, s0, 1);
+        s0 += __shfl_xor_sync(kFull, s0, 2);
+        s1 += __shfl_xor_sync(kFull, s1, 1);
+        s1 += __shfl_xor_sync(kFull, s1, 2);
+      }
+      if (c == 0) {
+        float* out = p.scores + (int64_t)b * p.vis_stride;
+        if (j + pg < nv) out[j + pg] = s0;
+        if (j + pg + 8 < nv) out[j + pg + 8] = s1;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+}
+
 // ---------------------------------------------------------------- top-k
 __device__ __forceinline__ int scan256_inclusive(int v, int* s_w) {
   // threads 0..255 participate; returns the inclusive prefix over them
@@ -364,7 +588,12 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
     if (tid < 256) {
       const int bin = 255 - tid;  // descending digit order
       int cnt = 0;
-      for (int r = 0; r < CL; ++r) cnt += static_cast<int>(*cluster.map_shared_rank(&s_hist[pass][bin], r));
+      uint32_t part[kMaxCluster];
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r)  // all remote loads in flight before the sum
+        part[r] = r < CL ? *cluster.map_shared_rank(&s_hist[pass][bin], r) : 0u;
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r) cnt += static_cast<int>(part[r]);
       const int incl = scan256_inclusive(cnt, s_w);
       const int excl = incl - cnt;
       if (excl < krem && krem <= incl) {
@@ -380,18 +609,38 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
   }
   const uint32_t T = prefix;  // the k-th largest key; take the first krem keys equal to T
 
-  // per-CTA counts, exchanged across the cluster
+  // Ordered output. Warp w owns the contiguous segment [w*seg, (w+1)*seg) of
+  // this CTA's slice. Pass 1 counts, per warp, keys above T and equal to T;
+  // the counts are scanned over the warps of the CTA and then over the CTAs
+  // of the cluster; pass 2 writes the chosen ids in index order.
+  constexpr int NW = kSelThreads / 32;
+  const int wid = tid >> 5;
+  const int seg = ((len + NW - 1) / NW + 31) / 32 * 32;
+  const int s_lo = wid * seg, s_hi = min(len, s_lo + seg);
   int gt = 0, eq = 0;
-  for (int i = tid; i < len; i += kSelThreads) {
-    gt += s_keys[i] > T;
-    eq += s_keys[i] == T;
+  for (int base = s_lo; base < s_hi; base += 32) {
+    const int i = base + lane;
+    const uint32_t key = i < s_hi ? s_keys[i] : 0u;
+    gt += __popc(__ballot_sync(kFull, i < s_hi && key > T));
+    eq += __popc(__ballot_sync(kFull, i < s_hi && key == T));
   }
-  int tot;
-  block_exclusive_scan<kSelThreads>(gt, s_w, tot);
-  if (tid == 0) s_cnt[0] = tot;
-  block_exclusive_scan<kSelThreads>(eq, s_w, tot);
-  if (tid == 0) s_cnt[1] = tot;
+  __shared__ int s_wgt[NW], s_weq[NW];
+  if (lane == 0) {
+    s_wgt[wid] = gt;
+    s_weq[wid] = eq;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int tg = 0, te = 0;
+    for (int w = 0; w < NW; ++w) {
+      tg += s_wgt[w];
+      te += s_weq[w];
+    }
+    s_cnt[0] = tg;
+    s_cnt[1] = te;
+  }
   cluster.sync();
+  // ties are taken in index order: CTA r may take krem minus the ties of CTAs before it
   int eq_before = 0, sel_before = 0, take_eq = 0;
   for (int r = 0; r < CL; ++r) {
     const int g_r = *cluster.map_shared_rank(&s_cnt[0], r);
@@ -406,22 +655,30 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
       break;
     }
   }
-  int run_eq = 0, run_sel = 0;
-  for (int base = 0; base < len; base += kSelThreads) {
-    const int i = base + tid;
-    const uint32_t key = i < len ? s_keys[i] : 0u;
-    const int is_eq = i < len && key == T;
-    int tot_eq;
-    const int eq_rank = run_eq + block_exclusive_scan<kSelThreads>(is_eq, s_w, tot_eq);
-    const int sel = (i < len && key > T) || (is_eq && eq_rank < take_eq);
-    int tot_sel;
-    const int at = run_sel + block_exclusive_scan<kSelThreads>(sel, s_w, tot_sel);
-    if (sel && sel_before + at < k) {
-      oidx[sel_before + at] = static_cast<int32_t>(lo + i);
-      if (osc) osc[sel_before + at] = key2f(key);
+  // the same split inside the CTA, over its warps
+  int w_eq_before = 0, w_sel_before = sel_before;
+  for (int w = 0; w < wid; ++w) {
+    int t_w = take_eq - w_eq_before;
+    t_w = t_w < 0 ? 0 : (t_w > s_weq[w] ? s_weq[w] : t_w);
+    w_sel_before += s_wgt[w] + t_w;
+    w_eq_before += s_weq[w];
+  }
+  int run_eq = w_eq_before, run_sel = w_sel_before;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = s_lo; base < s_hi; base += 32) {
+    const int i = base + lane;
+    const uint32_t key = i < s_hi ? s_keys[i] : 0u;
+    const unsigned m_eq = __ballot_sync(kFull, i < s_hi && key == T);
+    const int eq_rank = run_eq + __popc(m_eq & lt);
+    const bool sel = (i < s_hi && key > T) || ((m_eq >> lane) & 1u && eq_rank < take_eq);
+    const unsigned m_sel = __ballot_sync(kFull, sel);
+    const int at = run_sel + __popc(m_sel & lt);
+    if (sel && at < k) {
+      oidx[at] = static_cast<int32_t>(lo + i);
+      if (osc) osc[at] = key2f(key);
     }
-    run_eq += tot_eq;
-    run_sel += tot_sel;
+    run_eq += __popc(m_eq);
+    run_sel += __popc(m_sel);
   }
   if (rank == 0 && tid == 0) p.out_cnt[b] = k;
   cluster.sync();  // peers may still read this CTA's shared memory
@@ -441,6 +698,44 @@ cudaError_t launch_scan(IndexParams& p, int n_sm, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link)
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+template <int NCH, int NTH>
+cudaError_t launch_scan_tma(IndexParams& p, int n_sm, cudaStream_t st) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.d_idx), static_cast<cuuint64_t>(p.n_pages) * p.page_size};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.d_idx) * 2};
+  const cuuint32_t box[2] = {64, kUnitKeys};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p.idx_pool), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  auto kern = index_scan_tma_kernel<NCH, NTH>;
+  const size_t smem = TmaScanShape<NCH>::smem_bytes(p.n_q);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t units_max = (visible_entries(p.max_pos, p.m, p.n_win) + kUnitKeys - 1) / kUnitKeys;
+  int64_t grid = units_max * p.n_q;
+  if (grid > n_sm) grid = n_sm;
+  if (grid < 1) grid = 1;
+  kern<<<static_cast<int>(grid), kTmaThreads, smem, st>>>(map, p);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t index_ws_bytes(int n_q, int64_t max_pos, int m, int n_win) {
@@ -457,7 +752,16 @@ cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st) {
   cudaError_t e = cudaSuccess;
   const bool fp4 = p.idx_dtype == CSKV_FP4_E2M1;
   const int nth = (p.n_heads_idx + 7) / 8;
-  if (nv_max > 0) {
+  const bool tma_ok = !fp4 && p.page_size % kUnitKeys == 0 && (p.d_idx == 64 || p.d_idx == 128) && nth <= 2 &&
+                      (reinterpret_cast<uintptr_t>(p.idx_pool) & 15u) == 0 &&
+                      (int64_t)p.n_pages * p.page_size < (int64_t(1) << 31);
+  if (nv_max > 0 && tma_ok) {
+    if (p.d_idx == 64 && nth == 1) e = launch_scan_tma<2, 1>(p, n_sm, st);
+    else if (p.d_idx == 64 && nth == 2) e = launch_scan_tma<2, 2>(p, n_sm, st);
+    else if (p.d_idx == 128 && nth == 1) e = launch_scan_tma<4, 1>(p, n_sm, st);
+    else e = launch_scan_tma<4, 2>(p, n_sm, st);
+    if (e != cudaSuccess) return e;
+  } else if (nv_max > 0) {
     if (!fp4 && p.d_idx == 64 && nth == 1) e = launch_scan<2, 1, 2, false>(p, n_sm, st);
     else if (!fp4 && p.d_idx == 64 && nth == 2) e = launch_scan<2, 2, 2, false>(p, n_sm, st);
     else if (!fp4 && p.d_idx == 128 && nth == 1) e = launch_scan<4, 1, 1, false>(p, n_sm, st);
@@ -471,9 +775,9 @@ cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st) {
   // selection: a cluster of CL CTAs per query, each holding a slice of scores
   int cl_min = static_cast<int>((nv_max + kSliceCap - 1) / kSliceCap);
   if (cl_min < 1) cl_min = 1;
-  if (cl_min > 8) return cudaErrorNotSupported;
+  if (cl_min > kMaxCluster) return cudaErrorNotSupported;
   int cl_par = n_sm / (p.n_q > 0 ? p.n_q : 1);
-  if (cl_par > 8) cl_par = 8;
+  if (cl_par > kMaxCluster) cl_par = kMaxCluster;
   int cl = cl_min > cl_par ? cl_min : cl_par;
   if (cl < 1) cl = 1;
   // no point in CTAs that would hold fewer than 4096 scores
@@ -485,6 +789,10 @@ cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st) {
   e = cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
   if (e != cudaSuccess) return e;
+  if (cl > 8) {
+    e = cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
   if (p.n_q == 0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(p.n_q * cl), 1, 1);
@@ -498,6 +806,22 @@ cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (cl > 8) {  // a non-portable cluster must fit in one GPC; else fall back to 8
+    int n_clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&n_clusters, index_select_kernel, &cfg) != cudaSuccess || n_clusters < 1) {
+      (void)cudaGetLastError();
+      if (cl_min > 8) return cudaErrorNotSupported;
+      cl = 8;
+      p.cluster = cl;
+      p.slice = static_cast<int>(((nv_max + cl - 1) / cl + 3) / 4 * 4);
+      cfg.gridDim = dim3(static_cast<unsigned>(p.n_q * cl), 1, 1);
+      cfg.dynamicSmemBytes = sizeof(uint32_t) * static_cast<size_t>(p.slice);
+      attr[0].val.clusterDim.x = static_cast<unsigned>(cl);
+      e = cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(cfg.dynamicSmemBytes));
+      if (e != cudaSuccess) return e;
+    }
+  }
   return cudaLaunchKernelEx(&cfg, index_select_kernel, p);
 }
 
