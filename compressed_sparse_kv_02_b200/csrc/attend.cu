@@ -340,6 +340,8 @@ __global__ void __launch_bounds__(32 * MT * VS) attend_kernel(AttendParams p) {
 }
 
 // out[b,h,:] = sum_s exp(lse_s - L) o_s,  L = log sum_s exp(lse_s)
+// d_v / 4 threads per head, four channels each; the split loop issues eight
+// independent loads at a time.
 __global__ void __launch_bounds__(256) attend_merge_kernel(AttendParams p) {
   const int b = blockIdx.x;
   const QueryKeys qk = query_keys(p, b);
@@ -354,15 +356,27 @@ __global__ void __launch_bounds__(256) attend_merge_kernel(AttendParams p) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     float wsum = 0.f;
     if (L != -INFINITY) {
-      for (int s = 0; s < ns; ++s) {
-        const float ls = p.part_lse[base + (int64_t)s * p.n_heads];
-        const float wgt = expf(ls - L);
-        wsum += wgt;
-        const float4 o = *reinterpret_cast<const float4*>(p.part_o + (base + (int64_t)s * p.n_heads) * p.d_v + c4);
-        acc[0] += wgt * o.x;
-        acc[1] += wgt * o.y;
-        acc[2] += wgt * o.z;
-        acc[3] += wgt * o.w;
+      for (int s0 = 0; s0 < ns; s0 += 8) {
+        float wg[8];
+        float4 o[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int s = s0 + j;
+          wg[j] = 0.f;
+          o[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (s < ns) {
+            wg[j] = expf(p.part_lse[base + (int64_t)s * p.n_heads] - L);
+            o[j] = *reinterpret_cast<const float4*>(p.part_o + (base + (int64_t)s * p.n_heads) * p.d_v + c4);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          wsum += wg[j];
+          acc[0] += wg[j] * o[j].x;
+          acc[1] += wg[j] * o[j].y;
+          acc[2] += wg[j] * o[j].z;
+          acc[3] += wg[j] * o[j].w;
+        }
       }
     }
     const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
@@ -445,7 +459,7 @@ static void choose_split(AttendParams& p, int n_sm) {
 
 size_t attend_ws_bytes(const AttendParams& p0, int n_sm) {
   AttendParams p = p0;
-  if (attend_tc_supported(p.d_qk, p.d_v, p.n_heads, p.kv_dtype))
+  if (attend_tc_supported(p.d_qk, p.d_v, p.n_heads, p.kv_dtype, p.n_q))
     attend_tc_plan(p, n_sm);
   else
     choose_split(p, n_sm);
@@ -454,7 +468,7 @@ size_t attend_ws_bytes(const AttendParams& p0, int n_sm) {
 }
 
 cudaError_t launch_attend(AttendParams& p, void* ws, int n_sm, cudaStream_t st) {
-  const bool tc = attend_tc_supported(p.d_qk, p.d_v, p.n_heads, p.kv_dtype);
+  const bool tc = attend_tc_supported(p.d_qk, p.d_v, p.n_heads, p.kv_dtype, p.n_q);
   if (tc)
     attend_tc_plan(p, n_sm);
   else

@@ -37,20 +37,23 @@ constexpr int kDqk = 576, kDv = 512, kM = 128, kNk = 32;
 constexpr int kKb = kDqk / 64;                // 64-channel (128-byte) blocks per row
 constexpr int kQBytes = kKb * kM * 128;       // 147456
 constexpr int kKBytes = kKb * kNk * 128;      // 36864 per key tile
-constexpr int kThreads = 256;
-constexpr int kMmaThread = 128;               // warp 4, lane 0 issues the tensor-core work
+constexpr int kThreads = 256;                 // warps 0-3 softmax, warp 4 MMA, warps 5-7 loads
+constexpr int kMmaThread = 128;
+constexpr int kLoadThread0 = 160;
+constexpr int kLoaders = kThreads - kLoadThread0;  // 96
+constexpr int kRowCap = 1024;                 // keys per work item (row table in shared memory)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0, kColS = 256, kColP = 288;
+constexpr uint32_t kColO = 0, kColS = 256, kColP = 320;  // O 256 | S 2 x 32 | P 2 x 16 (bf16 pairs)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 
 struct Smem {
   static constexpr int Q = 0;
-  static constexpr int K = kQBytes;                 // two tile buffers
-  static constexpr int BAR = K + 2 * kKBytes;       // bar_s, bar_o
-  static constexpr int SCALE = BAR + 64;            // [2][kNk] key weight: 1 valid, 0 masked
-  static constexpr int TMEM = SCALE + 2 * kNk * 4;  // allocated tensor-memory address
+  static constexpr int K = kQBytes;                  // two tile buffers
+  static constexpr int BAR = K + 2 * kKBytes;        // 9 mbarriers
+  static constexpr int ROWS = BAR + 128;             // source row of every key of the item
+  static constexpr int TMEM = ROWS + kRowCap * 8;    // allocated tensor-memory address
   static constexpr int FLAGS = TMEM + 16;
   static constexpr int PREF = FLAGS + 16;
   static size_t bytes(int n_q) { return 1024 + PREF + sizeof(int) * (size_t)(n_q + 1); }
@@ -107,14 +110,26 @@ __device__ __forceinline__ uint32_t swz(int r, int ch, int block_bytes) {
   return (ch >> 3) * block_bytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
 }
 
+// Pipeline (per CTA, tiles numbered gt across its items; buffer gt & 1):
+//   loaders  : wait kempty[buf] (P V of tile gt-2 done) -> cp.async tile gt ->
+//              wait own copies -> proxy fence -> arrive kfull[buf]
+//   MMA      : wait kfull -> S(gt) = Q K^T into S[buf] -> commit sfull[buf];
+//              then wait pfull of tile gt-1 -> O += P V -> commit kempty, obar
+//   softmax  : wait sfull[buf] -> S row -> P row into P[buf] (+ rare O rescale
+//              after obar of tile gt-1) -> arrive pfull[buf]
+// S(gt) is issued before P V (gt-1), so the tensor core overlaps the softmax.
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = sm + Smem::Q;
   uint8_t* sK = sm + Smem::K;
-  uint64_t* bar_s = reinterpret_cast<uint64_t*>(sm + Smem::BAR);
-  uint64_t* bar_o = bar_s + 1;
-  float* sScale = reinterpret_cast<float*>(sm + Smem::SCALE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Smem::BAR);
+  uint64_t* kfull = bars;       // [2] loaders -> MMA (96 arrivals)
+  uint64_t* kempty = bars + 2;  // [2] MMA -> loaders (commit)
+  uint64_t* sfull = bars + 4;   // [2] MMA -> softmax (commit)
+  uint64_t* pfull = bars + 6;   // [2] softmax -> MMA (128 arrivals)
+  uint64_t* obar = bars + 8;    //     MMA -> softmax (commit after each P V)
+  const uint16_t** sRow = reinterpret_cast<const uint16_t**>(sm + Smem::ROWS);
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + Smem::TMEM);
   int* sAbort = reinterpret_cast<int*>(sm + Smem::FLAGS);
   int* sPref = reinterpret_cast<int*>(sm + Smem::PREF);
@@ -141,8 +156,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendParams p) 
     if (tid == 0) sPref[p.n_q] = run;
   }
   if (tid == 0) {
-    mbar_init(bar_s, 1);
-    mbar_init(bar_o, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kfull[i], kLoaders);
+      mbar_init(&kempty[i], 1);
+      mbar_init(&sfull[i], 1);
+      mbar_init(&pfull[i], kM);
+    }
+    mbar_init(obar, 1);
     fence_barrier_init();
     *sAbort = 0;
   }
@@ -158,11 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendParams p) 
     for (int b = tid; b < p.n_q; b += kThreads)
       if (p.q_pos[b] < 0 || p.q_pos[b] > p.max_pos) report(p.status, CSKV_ERR_INVALID_ARG);
   const int total = sPref[p.n_q];
-  const float sl2 = p.sm_scale * kLog2e;
-  const uint32_t idesc_s = umma_idesc_bf16(kM, kNk, false);
-  const uint32_t idesc_pv = umma_idesc_bf16(kM, 256, true);
-  const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK);
-  uint32_t g = 0;  // tiles processed by this CTA so far (mbarrier phases)
+  uint32_t g = 0;  // tiles processed by this CTA before the current item
 
   for (int item = blockIdx.x; item < total; item += gridDim.x) {
     int lo = 0, hi = p.n_q - 1;
@@ -182,72 +198,111 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendParams p) 
     const int nk = static_cast<int>(kk.n - u0 < kps ? kk.n - u0 : kps);
     const int ntiles = (nk + kNk - 1) / kNk;
 
-    // ---- loads: Q rows (thread: one head row, half of its 72 chunks), key tiles (thread: one key row, 9 chunks)
-    {
-      const int qr = tid >> 1, half = tid & 1;
-      const uint16_t* src = p.q + ((int64_t)b * p.n_heads + grp * kM + qr) * kDqk;
-      for (int c = half * 36; c < half * 36 + 36; ++c) cp_async16(sQ + swz(qr, c, kM * 128), src + c * 8, 16);
-    }
-    auto issue_tile = [&](int it, int buf) {
-      const int kr = tid >> 3, part = tid & 7;
-      const int i = it * kNk + kr;
-      const uint16_t* src = nullptr;
-      if (i < nk && seq_ok) src = key_src(p, b, seq, kk, u0 + i);
-      if (i < nk && !src) report(p.status, CSKV_ERR_OUT_OF_RANGE);
-      if (part == 0) sScale[buf * kNk + kr] = src ? 1.f : 0.f;
-      uint8_t* dst = sK + buf * kKBytes;
+    // source rows of this item's keys, visible to every role after the barrier;
+    // all 256 threads resolve them, four independent lookups at a time
+    for (int i0 = 0; i0 < nk; i0 += 4 * kThreads) {
+      const uint16_t* src[4];
 #pragma unroll
-      for (int q = 0; q < 9; ++q) {
-        const int c = part * 9 + q;
-        cp_async16(dst + swz(kr, c, kNk * 128), src ? static_cast<const void*>(src + c * 8) : p.q, src ? 16 : 0);
+      for (int q = 0; q < 4; ++q) {
+        const int i = i0 + q * kThreads + tid;
+        src[q] = (i < nk && seq_ok) ? key_src(p, b, seq, kk, u0 + i) : nullptr;
       }
-      cp_async_commit();
-    };
-    issue_tile(0, 0);
-
-    float m_used = -INFINITY, l_run = 0.f;  // softmax state of this thread's head row (warps 0-3)
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    bool aborted = false;
-    for (int it = 0; it < ntiles; ++it) {
-      const int buf = it & 1;
-      const uint32_t gt = g + it;
-      if (it + 1 < ntiles) {
-        // buffer buf^1 was last read by the PV of tile it-1
-        if (it >= 1 && !mbar_wait(bar_o, (gt - 1) & 1u, p.status)) *sAbort = 1;
-        issue_tile(it + 1, buf ^ 1);
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
-      }
-      fence_proxy_async_smem();
-      __syncthreads();
-      if (*sAbort) { aborted = true; break; }
-      tc_fence_after();
-      if (tid == kMmaThread) {
-        const uint32_t kb_base = sKa + buf * kKBytes;
-#pragma unroll 1
-        for (int kb = 0; kb < kKb; ++kb) {
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t da = umma_desc_sw128(sQa + kb * (kM * 128) + ks * 32, 16, 1024);
-            const uint64_t db = umma_desc_sw128(kb_base + kb * (kNk * 128) + ks * 32, 16, 1024);
-            umma_ss(tmem + kColS, da, db, idesc_s, (kb | ks) != 0);
-          }
+      for (int q = 0; q < 4; ++q) {
+        const int i = i0 + q * kThreads + tid;
+        if (i < nk) {
+          if (!src[q]) report(p.status, CSKV_ERR_OUT_OF_RANGE);
+          sRow[i] = src[q];
         }
-        umma_commit(bar_s);
       }
-      if (warp < 4) {
-        bool ok = mbar_wait(bar_s, gt & 1u, p.status);
+    }
+    __syncthreads();
+
+    if (tid >= kLoadThread0) {
+      // ------------------------------------------------------------ loaders
+      const int lt = tid - kLoadThread0;
+      for (int i = lt; i < kM * 72; i += kLoaders) {  // Q rows of this head group (same copy group as tile 0)
+        const int qr = i / 72, c = i % 72;
+        cp_async16(sQ + swz(qr, c, kM * 128), p.q + ((int64_t)b * p.n_heads + grp * kM + qr) * kDqk + c * 8, 16);
+      }
+      for (int it = 0; it < ntiles; ++it) {
+        const uint32_t gt = g + it;
+        const int buf = gt & 1;
+        if (gt >= 2 && !mbar_wait(&kempty[buf], ((gt >> 1) - 1) & 1u, p.status)) { *sAbort = 1; break; }
+        uint8_t* dst = sK + buf * kKBytes;
+        // consecutive threads take consecutive 16-byte chunks of a row (coalesced)
+#pragma unroll 4
+        for (int id = lt; id < kNk * 72; id += kLoaders) {
+          const int kr = id / 72, c = id % 72;
+          const int i = it * kNk + kr;
+          const uint16_t* src = i < nk ? sRow[i] : nullptr;
+          cp_async16(dst + swz(kr, c, kNk * 128), src ? static_cast<const void*>(src + c * 8) : p.q, src ? 16 : 0);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        mbar_arrive(&kfull[buf]);
+      }
+    } else if (tid == kMmaThread) {
+      // ------------------------------------------------------------ MMA issue
+      const uint32_t idesc_s = umma_idesc_bf16(kM, kNk, false);
+      const uint32_t idesc_pv = umma_idesc_bf16(kM, 256, true);
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK);
+      for (int it = 0; it <= ntiles; ++it) {
+        if (it < ntiles) {
+          const uint32_t gt = g + it;
+          const int buf = gt & 1;
+          if (!mbar_wait(&kfull[buf], (gt >> 1) & 1u, p.status)) { *sAbort = 1; break; }
+          tc_fence_after();
+          const uint32_t kb_base = sKa + buf * kKBytes;
+          const uint32_t d = tmem + kColS + buf * kNk;
+#pragma unroll 1
+          for (int kb = 0; kb < kKb; ++kb) {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t da = umma_desc_sw128(sQa + kb * (kM * 128) + ks * 32, 16, 1024);
+              const uint64_t db = umma_desc_sw128(kb_base + kb * (kNk * 128) + ks * 32, 16, 1024);
+              umma_ss(d, da, db, idesc_s, (kb | ks) != 0);
+            }
+          }
+          umma_commit(&sfull[buf]);
+        }
+        if (it >= 1) {
+          const uint32_t gp = g + it - 1;
+          const int pb = gp & 1;
+          if (!mbar_wait(&pfull[pb], (gp >> 1) & 1u, p.status)) { *sAbort = 1; break; }
+          tc_fence_after();
+          const uint32_t v_base = sKa + pb * kKBytes + vh * 4 * (kNk * 128);
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2) {
+            const uint64_t db = umma_desc_sw128(v_base + k2 * 16 * 128, kNk * 128, 1024);
+            umma_ts(tmem + kColO, tmem + kColP + pb * 16 + k2 * 8, db, idesc_pv, (it > 1 || k2 > 0) ? 1u : 0u);
+          }
+          umma_commit(&kempty[pb]);
+          umma_commit(obar);
+        }
+      }
+    } else if (warp < 4) {
+      // ------------------------------------------------------------ softmax (one head row per thread)
+      const float sl2 = p.sm_scale * kLog2e;
+      const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+      float m_used = -INFINITY, l_run = 0.f;
+      bool ok = true;
+      for (int it = 0; it < ntiles && ok; ++it) {
+        const uint32_t gt = g + it;
+        const int buf = gt & 1;
+        ok = mbar_wait(&sfull[buf], (gt >> 1) & 1u, p.status);
+        if (!ok) break;
         tc_fence_after();
         uint32_t sr[32];
-        tmem_ld32(tmem + lane_base + kColS, sr);
+        tmem_ld32(tmem + lane_base + kColS + buf * kNk, sr);
         tmem_ld_wait();
         float v[32];
         float mt = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float w = sScale[buf * kNk + j];
-          v[j] = (it * kNk + j < nk && w != 0.f) ? __uint_as_float(sr[j]) * sl2 * w : -INFINITY;
+          const int i = it * kNk + j;
+          v[j] = (i < nk && sRow[i] != nullptr) ? __uint_as_float(sr[j]) * sl2 : -INFINITY;
           mt = fmaxf(mt, v[j]);
         }
         float corr = 1.f;
@@ -266,10 +321,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendParams p) 
           l_run += p0 + p1;
           pp[j] = pack_bf16(p0, p1);
         }
-        // the previous tile's P V must be done before P and O are rewritten
-        if (it >= 1) ok = mbar_wait(bar_o, (gt - 1) & 1u, p.status) && ok;
-        tc_fence_after();
         if (__any_sync(kFull, rescale)) {
+          // O is being accumulated by P V of tile gt-1: rescale after it lands
+          ok = mbar_wait(obar, (gt - 1) & 1u, p.status);
+          tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < 256; c += 32) {
             uint32_t orow[32];
@@ -280,55 +335,45 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendParams p) 
             tmem_st32(tmem + lane_base + kColO + c, orow);
           }
         }
-        tmem_st16(tmem + lane_base + kColP, pp);
+        tmem_st16(tmem + lane_base + kColP + buf * 16, pp);
         tmem_st_wait();
-        if (!ok) *sAbort = 1;
+        tc_fence_before();
+        mbar_arrive(&pfull[buf]);
       }
-      tc_fence_before();
-      __syncthreads();
-      if (*sAbort) { aborted = true; break; }
-      tc_fence_after();
-      if (tid == kMmaThread) {
-        const uint32_t v_base = sKa + buf * kKBytes + vh * 4 * (kNk * 128);
-#pragma unroll
-        for (int k2 = 0; k2 < 2; ++k2) {
-          const uint64_t db = umma_desc_sw128(v_base + k2 * 16 * 128, kNk * 128, 1024);
-          umma_ts(tmem + kColO, tmem + kColP + k2 * 8, db, idesc_pv, (it > 0 || k2 > 0) ? 1u : 0u);
-        }
-        umma_commit(bar_o);
-      }
-    }
-    if (aborted) break;
-    // ---- epilogue: normalised partial output of this split and half, and its log-sum-exp
-    if (warp < 4) {
-      if (!mbar_wait(bar_o, (g + ntiles - 1) & 1u, p.status)) *sAbort = 1;
-      tc_fence_after();
-      const int head = grp * kM + warp * 32 + lane;
-      const int64_t prow = ((int64_t)b * p.max_splits + split) * p.n_heads + head;
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      float* dst = p.part_o + prow * kDv + vh * 256;
+      // epilogue: normalised partial output of this split and half, and its log-sum-exp
+      if (ok && ntiles > 0) ok = mbar_wait(obar, (g + ntiles - 1) & 1u, p.status);
+      if (!ok) {
+        *sAbort = 1;
+      } else {
+        tc_fence_after();
+        const int head = grp * kM + warp * 32 + lane;
+        const int64_t prow = ((int64_t)b * p.max_splits + split) * p.n_heads + head;
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        float* dst = p.part_o + prow * kDv + vh * 256;
 #pragma unroll 1
-      for (int c = 0; c < 256; c += 32) {
-        uint32_t orow[32];
-        tmem_ld32(tmem + lane_base + kColO + c, orow);
-        tmem_ld_wait();
+        for (int c = 0; c < 256; c += 32) {
+          uint32_t orow[32];
+          tmem_ld32(tmem + lane_base + kColO + c, orow);
+          tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<float4*>(dst + c + j) =
-              make_float4(__uint_as_float(orow[j]) * inv, __uint_as_float(orow[j + 1]) * inv,
-                          __uint_as_float(orow[j + 2]) * inv, __uint_as_float(orow[j + 3]) * inv);
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(dst + c + j) =
+                make_float4(__uint_as_float(orow[j]) * inv, __uint_as_float(orow[j + 1]) * inv,
+                            __uint_as_float(orow[j + 2]) * inv, __uint_as_float(orow[j + 3]) * inv);
+        }
+        if (vh == 0) p.part_lse[prow] = l_run > 0.f ? (m_used + log2f(l_run)) * kLn2 : -INFINITY;
       }
-      if (vh == 0) p.part_lse[prow] = l_run > 0.f ? (m_used + log2f(l_run)) * kLn2 : -INFINITY;
     }
     g += ntiles;
     tc_fence_before();
     __syncthreads();  // shared and tensor memory are reused by the next item
+    tc_fence_after();
     if (*sAbort) break;
   }
-  // on an abort, give outstanding tensor-core work a bounded chance to finish before freeing
+  // after an abort, give tensor-core work in flight a bounded chance to land before freeing
   if (*sAbort && tid == kMmaThread) {
-    mbar_wait(bar_s, (g + 1) & 1u, nullptr);
-    mbar_wait(bar_o, (g + 1) & 1u, nullptr);
+    mbar_wait(&kempty[0], 0u, nullptr);
+    mbar_wait(obar, (g + 1) & 1u, nullptr);
   }
   cp_async_wait<0>();
   tc_fence_before();
@@ -339,8 +384,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(AttendParams p) 
 
 }  // namespace
 
-bool attend_tc_supported(int d_qk, int d_v, int n_heads, int kv_dtype) {
-  return d_qk == kDqk && d_v == kDv && n_heads % kM == 0 && kv_dtype == CSKV_BF16;
+bool attend_tc_supported(int d_qk, int d_v, int n_heads, int kv_dtype, int n_q) {
+  return d_qk == kDqk && d_v == kDv && n_heads % kM == 0 && kv_dtype == CSKV_BF16 &&
+         Smem::bytes(n_q) <= 232448;  // the per-query prefix table shares shared memory with the tiles
 }
 
 // keys per split: queries x head groups x splits x 2 halves ~ one CTA per SM
@@ -352,6 +398,7 @@ void attend_tc_plan(AttendParams& p, int n_sm) {
   int64_t kps = (n_max + splits - 1) / splits;
   kps = (kps + kNk - 1) / kNk * kNk;
   if (kps < kNk) kps = kNk;
+  if (kps > kRowCap) kps = kRowCap;
   p.keys_per_split = static_cast<int>(kps);
   p.max_splits = static_cast<int>((n_max + kps - 1) / kps);
   if (p.max_splits < 1) p.max_splits = 1;

@@ -112,7 +112,7 @@ cudaError_t launch_attend(AttendParams& p, void* ws, int n_sm, cudaStream_t st);
 bool attend_supported(int d_qk, int d_v, int n_heads, int kv_dtype);
 cudaError_t launch_attend_merge(AttendParams& p, cudaStream_t st);
 // tensor-core (tcgen05) attention for the 576 / 512 latent with heads in groups of 128
-bool attend_tc_supported(int d_qk, int d_v, int n_heads, int kv_dtype);
+bool attend_tc_supported(int d_qk, int d_v, int n_heads, int kv_dtype, int n_q);
 void attend_tc_plan(AttendParams& p, int n_sm);
 cudaError_t launch_attend_tc(AttendParams& p, int n_sm, cudaStream_t st);
 

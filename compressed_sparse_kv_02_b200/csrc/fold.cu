@@ -21,6 +21,7 @@ namespace cskv {
 namespace {
 
 constexpr int kGroupsPerLane = 4;  // d <= 1024 channels
+constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);
@@ -38,8 +39,8 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
 }
 
 // Online-softmax partial state of channels [c0, c0+8) over tokens i0 .. i1-1
-// of one block: running max, denominator and weighted sum (fp32). rows(i, xr,
-// zr) yields token i's raw row and gate row.
+// of one block: running max (of the logits times log2 e), denominator and
+// weighted sum (fp32). rows(i, xr, zr) yields token i's raw row and gate row.
 template <class Rows>
 __device__ __forceinline__ void fold_partial(const FoldStream& S, int i0, int i1, int c0, Rows rows,
                                              float (&mx)[8], float (&den)[8], float (&acc)[8]) {
@@ -69,13 +70,14 @@ __device__ __forceinline__ void fold_partial(const FoldStream& S, int i0, int i1
     }
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      if (zl[e] > mx[e]) {
-        float corr = expf(mx[e] - zl[e]);  // 0 while mx is -inf
+      const float l2 = zl[e] * kLog2e;  // softmax weights in base 2: 2^(l2 - max) = e^(z - max_z)
+      if (l2 > mx[e]) {
+        const float corr = exp2f(mx[e] - l2);  // 0 while mx is -inf
         den[e] *= corr;
         acc[e] *= corr;
-        mx[e] = zl[e];
+        mx[e] = l2;
       }
-      float p = expf(zl[e] - mx[e]);
+      const float p = exp2f(l2 - mx[e]);
       den[e] += p;
       acc[e] += p * xf[e];
     }
@@ -93,12 +95,12 @@ __device__ __forceinline__ void fold_group(const FoldStream& S, int m, int i0, i
 }
 
 // Round one entry to its storage type and store it at pool row `row`. The
-// calling threads hold 8 consecutive channels each: thread i of `n` holds
-// groups i, i + n, i + 2n, ... (up to kGroupsPerLane of them); `amax` is the
+// calling threads hold 8 consecutive channels each: a thread holds groups
+// first, first + stride, ... (its first `nslots` slots of v); `amax` is the
 // entry-wide max |value| (needed for FP8), already reduced by the caller.
 // Adjacent threads hold adjacent groups, so an FP4 16-channel block is the
 // pair (2q, 2q+1) of threads with the same parity pattern.
-__device__ __forceinline__ void store_groups(const FoldStream& S, int64_t row, int first, int stride,
+__device__ __forceinline__ void store_groups(const FoldStream& S, int64_t row, int first, int stride, int nslots,
                                              const float (&v)[kGroupsPerLane][8], float amax) {
   const int G = S.d / 8;
   if (S.out_dtype == CSKV_BF16) {
@@ -106,7 +108,7 @@ __device__ __forceinline__ void store_groups(const FoldStream& S, int64_t row, i
 #pragma unroll
     for (int gi = 0; gi < kGroupsPerLane; ++gi) {
       const int grp = first + stride * gi;
-      if (grp < G) {
+      if (gi < nslots && grp < G) {
         uint4 o;
         o.x = pack_bf16(v[gi][0], v[gi][1]);
         o.y = pack_bf16(v[gi][2], v[gi][3]);
@@ -121,7 +123,7 @@ __device__ __forceinline__ void store_groups(const FoldStream& S, int64_t row, i
 #pragma unroll
     for (int gi = 0; gi < kGroupsPerLane; ++gi) {
       const int grp = first + stride * gi;
-      if (grp < G) {
+      if (gi < nslots && grp < G) {
         uint32_t w[2] = {0u, 0u};
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -137,13 +139,14 @@ __device__ __forceinline__ void store_groups(const FoldStream& S, int64_t row, i
 #pragma unroll
     for (int gi = 0; gi < kGroupsPerLane; ++gi) {
       const int grp = first + stride * gi;
+      const bool mine = gi < nslots && grp < G;
       float a = 0.f;
-      if (grp < G) {
+      if (mine) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(v[gi][e]));
       }
       a = fmaxf(a, __shfl_xor_sync(kFull, a, 1));
-      if (grp < G) {
+      if (mine) {
         const __nv_fp8_storage_t sb = __nv_cvt_float_to_fp8(a / 6.0f, __NV_SATFINITE, __NV_E4M3);
         const float sd = __half2float(__half(__nv_cvt_fp8_to_halfraw(sb, __NV_E4M3)));
         uint32_t w = 0u;
@@ -179,16 +182,18 @@ __device__ void fold_entry_warp(const FoldStream& S, int m, int64_t row, Rows ro
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
-  store_groups(S, row, lane, 32, v, amax);
+  store_groups(S, row, lane, 32, kGroupsPerLane, v, amax);
 }
 
-// Fold one entry with the whole block (large m, or one entry per block):
-// thread t takes channel group t % G and token slice t / G; the partial
+// Fold channels [c_lo, c_hi) of one entry with the whole block: thread t
+// takes channel group t % G of the range and token slice t / G; the partial
 // online-softmax states (max, denominator, weighted sum) of the slices are
-// merged through shared memory. `sm` holds 3 * blockDim.x * 8 floats.
+// merged through shared memory. `sm` holds 3 * blockDim.x * 8 floats. For an
+// FP8 entry the range must be the whole row (its scale is the row's amax).
 template <class Rows>
-__device__ void fold_entry_block(const FoldStream& S, int m, int64_t row, Rows rows, float* sm) {
-  const int G = S.d / 8;
+__device__ void fold_entry_block(const FoldStream& S, int m, int64_t row, Rows rows, float* sm, int c_lo,
+                                 int c_hi) {
+  const int G = (c_hi - c_lo) / 8;
   const int t = threadIdx.x;
   int ns = blockDim.x / G;  // token slices
   if (ns > m) ns = m;
@@ -200,7 +205,7 @@ __device__ void fold_entry_block(const FoldStream& S, int m, int64_t row, Rows r
   if (sl < ns) {
     float mx[8], den[8], acc[8];
     const int i0 = sl * per, i1 = min(m, i0 + per);
-    fold_partial(S, i0, i1, g * 8, rows, mx, den, acc);
+    fold_partial(S, i0, i1, c_lo + g * 8, rows, mx, den, acc);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       smx[(sl * G + g) * 8 + e] = mx[e];
@@ -209,7 +214,7 @@ __device__ void fold_entry_block(const FoldStream& S, int m, int64_t row, Rows r
     }
   }
   __syncthreads();
-  // threads 0..G-1 merge the slices of their group (warps that hold no group still join the reductions)
+  // threads 0..G-1 merge the slices of their group
   float v[kGroupsPerLane][8];
   float amax = 0.f;
   if (t < G) {
@@ -225,7 +230,7 @@ __device__ void fold_entry_block(const FoldStream& S, int m, int64_t row, Rows r
       for (int q = 0; q < ns; ++q) {
         const float mq = smx[(q * G + t) * 8 + e];
         if (mq == -INFINITY) continue;
-        const float f = expf(mq - M[e]);
+        const float f = exp2f(mq - M[e]);
         den += sden[(q * G + t) * 8 + e] * f;
         acc += sacc[(q * G + t) * 8 + e] * f;
       }
@@ -233,15 +238,16 @@ __device__ void fold_entry_block(const FoldStream& S, int m, int64_t row, Rows r
       amax = fmaxf(amax, fabsf(v[0][e]));
     }
   }
-  // entry-wide amax (FP8 scale): block reduction
+  if (S.out_dtype == CSKV_FP8_E4M3) {  // entry-wide amax: block reduction
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
-  __syncthreads();
-  if ((t & 31) == 0) smx[t >> 5] = amax;
-  __syncthreads();
-  amax = 0.f;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) amax = fmaxf(amax, smx[w]);
-  if (t < ((G + 31) & ~31)) store_groups(S, row, t, G, v, amax);  // one group per thread (gi = 0)
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+    __syncthreads();
+    if ((t & 31) == 0) smx[t >> 5] = amax;
+    __syncthreads();
+    amax = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) amax = fmaxf(amax, smx[w]);
+  }
+  if (t < ((G + 31) & ~31)) store_groups(S, row, c_lo / 8 + t, G, t < G ? 1 : 0, v, amax);
   __syncthreads();  // shared memory is reused by the next entry
 }
 
@@ -312,34 +318,41 @@ __global__ void __launch_bounds__(kBlockFoldThreads) fold_bulk_block_kernel(Fold
     int64_t row;
     BulkRows r;
     bulk_item(p, it, si, row, r);
-    if (row >= 0) fold_entry_block(p.s[si], p.m, row, r, sm);  // row is uniform across the block
+    if (row >= 0) fold_entry_block(p.s[si], p.m, row, r, sm, 0, p.s[si].d);  // row is uniform across the block
   }
 }
 
-// One CTA per sequence: copy the new rows into the ring, then fold every
-// block the new tokens complete, one entry at a time with the whole CTA (old
-// rows from the ring, new rows from the input; the slots written and the
-// slots read never coincide because n_new + m - 1 <= n_win).
-__global__ void __launch_bounds__(kBlockFoldThreads) append_kernel(FoldParams p) {
-  __shared__ float sm[3 * kBlockFoldThreads * 8];
-  const int b = blockIdx.x;
+constexpr int kAppendThreads = 256;
+constexpr int kSliceCh = 64;  // channels per CTA of the append kernel
+
+// Grid (sequence, 64-channel slice). Each CTA copies its slice of the new rows
+// into the rings, then folds its slice of every block the new tokens complete
+// (old rows from the ring, new rows from the input; the slots written and the
+// slots read never coincide because n_new + m - 1 <= n_win). An FP8 stream
+// needs the whole row for its scale, so slice 0 folds all of it.
+__global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
+  __shared__ float sm[3 * kAppendThreads * 8];
+  const int b = blockIdx.x, slice = blockIdx.y;
   const int seq = p.seq_ids[b];
   if (seq < 0 || seq >= p.n_seqs_layer) {
-    if (threadIdx.x == 0) report(p.status, CSKV_ERR_OUT_OF_RANGE);
+    if (threadIdx.x == 0 && slice == 0) report(p.status, CSKV_ERR_OUT_OF_RANGE);
     return;
   }
   const int64_t pos = p.pos[b];
   for (int si = 0; si < p.n_streams; ++si) {
     const FoldStream& S = p.s[si];
-    const int cx = S.d / 8;  // 16-byte chunks per x row
+    const int c_lo = slice * kSliceCh, c_hi = min(S.d, c_lo + kSliceCh);
+    if (c_lo >= S.d) continue;
+    const int cx = (c_hi - c_lo) / 8;  // 16-byte chunks of this slice per row
     for (int t = threadIdx.x; t < p.n_new * cx; t += blockDim.x) {
       const int i = t / cx, ch = t % cx;
       const int64_t slot = (pos + i) % p.n_win;
-      *reinterpret_cast<uint4*>(S.ring_x_w + ((int64_t)seq * p.n_win + slot) * S.d + ch * 8) =
-          ldg16(S.x + ((int64_t)b * p.n_new + i) * S.d + ch * 8);
+      *reinterpret_cast<uint4*>(S.ring_x_w + ((int64_t)seq * p.n_win + slot) * S.d + c_lo + ch * 8) =
+          ldg16(S.x + ((int64_t)b * p.n_new + i) * S.d + c_lo + ch * 8);
     }
-    for (int t = threadIdx.x; t < p.n_new * S.gc; t += blockDim.x) {
-      const int i = t / S.gc, c = t % S.gc;
+    const int z_lo = S.gc == 1 ? (slice == 0 ? 0 : 1) : c_lo, z_hi = S.gc == 1 ? 1 : c_hi;
+    for (int t = threadIdx.x; t < p.n_new * (z_hi - z_lo); t += blockDim.x) {
+      const int i = t / (z_hi - z_lo), c = z_lo + t % (z_hi - z_lo);
       const int64_t slot = (pos + i) % p.n_win;
       S.ring_z_w[((int64_t)seq * p.n_win + slot) * S.gc + c] = S.z[((int64_t)b * p.n_new + i) * S.gc + c];
     }
@@ -353,6 +366,10 @@ __global__ void __launch_bounds__(kBlockFoldThreads) append_kernel(FoldParams p)
     const int si = static_cast<int>(it / nb);
     const int64_t j = j_first + it % nb;
     const FoldStream& S = p.s[si];
+    const bool whole = S.out_dtype == CSKV_FP8_E4M3;
+    const int c_lo = whole ? 0 : slice * kSliceCh;
+    const int c_hi = whole ? S.d : min(S.d, c_lo + kSliceCh);
+    if (c_lo >= S.d || (whole && slice != 0)) continue;  // uniform across the block
     const int64_t row = entry_row(p, seq, j);
     auto rows = [&](int i, const uint16_t*& xr, const uint16_t*& zr) {
       const int64_t q = j * p.m + i;
@@ -365,7 +382,7 @@ __global__ void __launch_bounds__(kBlockFoldThreads) append_kernel(FoldParams p)
         zr = S.ring_z + ((int64_t)seq * p.n_win + slot) * S.gc;
       }
     };
-    if (row >= 0) fold_entry_block(S, p.m, row, rows, sm);  // row is uniform across the block
+    if (row >= 0) fold_entry_block(S, p.m, row, rows, sm, c_lo, c_hi);  // row is uniform across the block
   }
 }
 
@@ -390,7 +407,10 @@ cudaError_t launch_fold_bulk(const FoldParams& p, cudaStream_t st) {
 
 cudaError_t launch_append(const FoldParams& p, cudaStream_t st) {
   if (p.n_seq == 0 || p.n_new == 0) return cudaSuccess;
-  append_kernel<<<p.n_seq, kBlockFoldThreads, 0, st>>>(p);
+  int dmax = 0;
+  for (int si = 0; si < p.n_streams; ++si) dmax = p.s[si].d > dmax ? p.s[si].d : dmax;
+  dim3 grid(static_cast<unsigned>(p.n_seq), static_cast<unsigned>((dmax + kSliceCh - 1) / kSliceCh));
+  append_kernel<<<grid, kAppendThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -440,6 +440,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
   uint4 qf[NTH][NCH];
   float wv[NTH][2];
   int cur_b = -1;
+  int64_t cur_nv = 0;
   for (int64_t i = group; i < n_units; i += NGROUP) {
     const int s = static_cast<int>(i % NSTAGE);
     const uint32_t round = static_cast<uint32_t>(i / NSTAGE);
@@ -449,6 +450,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     locate(u_begin + i, b, j0);
     if (b != cur_b) {
       cur_b = b;
+      cur_nv = query_visible(p, b);
 #pragma unroll
       for (int nt = 0; nt < NTH; ++nt) {
         const int n = 8 * nt + g;
@@ -463,7 +465,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
         }
       }
     }
-    const int64_t nv = query_visible(p, b);
+    const int64_t nv = cur_nv;
     const int64_t j = j0 + 16 * sub;  // this warp's 16 keys
     if (j < nv) {
       float s0 = -INFINITY, s1 = -INFINITY;

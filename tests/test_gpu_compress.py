@@ -111,7 +111,8 @@ def test_fp8_kv_and_fp4_index_storage(ck, orc):
 
 @pytest.mark.parametrize("kind,m", [("csa", 4), ("hca", 128)])
 def test_append_equals_bulk_and_fills_ring(ck, orc, kind, m):
-    """Token-by-token decode appends produce the same entries, bit for bit, as one bulk fold."""
+    """Token-by-token decode appends produce the entries of one bulk fold (both within the fold
+    tolerance of the oracle: the two paths split the token sum differently) and fill the ring."""
     B, d, d_idx = 2, 128, 64
     n = 3 * 128 + 40  # ends mid-block for HCA
     is_csa = kind == "csa"
@@ -137,10 +138,18 @@ def test_append_equals_bulk_and_fills_ring(ck, orc, kind, m):
     assert ck.cskv_get_status(status) == ck.OK
     for b in range(B):
         s = int(seq[b])
-        ea, eb = La.read_entries(s, n // m), Lb.read_entries(s, n // m)
-        assert torch.equal(ea["kv"], eb["kv"])
-        if is_csa:
-            assert torch.equal(ea["idx"], eb["idx"])
+        nb_e = n // m
+        ref = orc.decode(orc.store(orc.compress(stored_bf16(x[b, :nb_e * m]), stored_bf16(z[b, :nb_e * m]), m),
+                                   orc.BF16))
+        xd = orc.decode(stored_bf16(x[b]))
+        for L, what in ((La, "bulk"), (Lb, "append")):
+            e = layer_entries(L, s, nb_e)
+            assert_fold_close(orc.decode(e["kv"]), ref, xd, m, "%s kv seq %d" % (what, s))
+            if is_csa:
+                ref_i = orc.decode(orc.store(orc.compress(stored_bf16(xi[b, :nb_e * m]),
+                                                          stored_bf16(zi[b, :nb_e * m]), m), orc.BF16))
+                assert_fold_close(orc.decode(e["idx"]), ref_i, orc.decode(stored_bf16(xi[b])), m,
+                                  "%s idx seq %d" % (what, s))
         slots = [p % 128 for p in range(n - 128, n)]
         assert torch.equal(Lb.ring_x[s][slots], x[b, n - 128:])
         assert torch.equal(Lb.ring_z[s][slots], z[b, n - 128:])
@@ -167,8 +176,12 @@ def test_multi_token_append_and_ring_only(ck, orc):
                          z[:, n - 128:].contiguous(), xi[:, n - 128:].contiguous(), zi[:, n - 128:].contiguous(),
                          ring_only=True)
     torch.cuda.synchronize()
-    a, b = L1.read_entries(0, n // m), L2.read_entries(0, n // m)
-    assert torch.equal(a["kv"], b["kv"]) and torch.equal(a["idx"], b["idx"])
+    ref = orc.decode(orc.store(orc.compress(stored_bf16(x[0]), stored_bf16(z[0]), m), orc.BF16))
+    ref_i = orc.decode(orc.store(orc.compress(stored_bf16(xi[0]), stored_bf16(zi[0]), m), orc.BF16))
+    for L in (L1, L2):
+        e = layer_entries(L, 0, n // m)
+        assert_fold_close(orc.decode(e["kv"]), ref, orc.decode(stored_bf16(x[0])), m, "kv")
+        assert_fold_close(orc.decode(e["idx"]), ref_i, orc.decode(stored_bf16(xi[0])), m, "idx")
     assert torch.equal(L1.ring_x, L2.ring_x) and torch.equal(L1.ring_zi, L2.ring_zi)
 
 
