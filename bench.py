@@ -198,8 +198,10 @@ def run_ours(args, rank, world):
                 evb[j][i][0].record(stream)
                 c(s)
                 evb[j][i][1].record(stream)
-    for _ in range(max(1, -(-args.warmup // n_ev))):
-        graph.replay()
+    # graphs replay on the stream the timing events are recorded on
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, -(-args.warmup // n_ev))):
+            graph.replay()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -209,12 +211,13 @@ def run_ours(args, rank, world):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    t0.record(stream)
-    for _ in range(reps):
-        graph.replay()
-    if graph_rem is not None:
-        graph_rem.replay()
-    t1.record(stream)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        if graph_rem is not None:
+            graph_rem.replay()
+        t1.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
     if world > 1:
@@ -222,7 +225,8 @@ def run_ours(args, rank, world):
     steps_timed = args.steps
     ms_total = t0.elapsed_time(t1)
     idx_vals = [ev[j][0].elapsed_time(ev[j][1]) for j in range(n_ev)] if reps else []
-    graph_b.replay()
+    with torch.cuda.stream(stream):
+        graph_b.replay()
     torch.cuda.synchronize()
     op_ms = {}
     for i, c in enumerate(calls):

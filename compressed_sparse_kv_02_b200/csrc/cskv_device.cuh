@@ -62,6 +62,11 @@ __device__ __forceinline__ uint4 ldg16_stream(const void* p) {
   return v;
 }
 
+// Hint the L2 to fetch [p, p + bytes) from DRAM (16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

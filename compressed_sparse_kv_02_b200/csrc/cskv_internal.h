@@ -2,12 +2,17 @@
 // (cskv_abi.cu) and the kernel files. Not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "cskv.h"
 
 namespace cskv {
+
+// cuTensorMapEncodeTiled, looked up once through the runtime (null if unavailable)
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 // One stream of raw tokens folded into compressed entries (the latent-KV
 // stream, or the indexer-key stream of a CSA layer).
@@ -70,6 +75,7 @@ struct IndexParams {
   // workspace
   float* scores;        // [n_q, vis_stride]
   int64_t vis_stride;
+  uint32_t* hist;       // [n_q, 2048] counts of the scores' top 11 key bits (from the scan), or null
   int cluster;          // CTAs per query in the selection kernel
   int slice;            // entries per CTA of the selection kernel
 };

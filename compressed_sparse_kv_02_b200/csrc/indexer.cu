@@ -16,12 +16,18 @@
 // the dot product is unchanged while every load is a full 128-bit access.
 //
 // index_select_kernel picks the top-k per query: a cluster of CTAs holds the
-// query's scores in shared memory (one slice per CTA), runs a 4-pass 8-bit
-// radix select on order-preserving integer keys with the per-CTA histograms
-// summed through distributed shared memory, and writes the chosen indices in
-// ascending order (equal scores prefer the lower index).
+// query's scores in shared memory (one slice per CTA) and runs a radix select
+// on order-preserving integer keys in three digits (11, 11 and 10 bits). The
+// first digit's histogram is counted by the TMA scan as it writes the scores;
+// the later digits are counted over the few keys left in the threshold bin,
+// with the per-CTA histograms summed through distributed shared memory. The
+// chosen indices are written in ascending order (equal scores prefer the
+// lower index).
 #include <cooperative_groups.h>
 #include <cudaTypedefs.h>
+
+#include <mutex>
+#include <vector>
 
 #include "cskv_device.cuh"
 #include "cskv_internal.h"
@@ -36,6 +42,7 @@ constexpr int kMaxQueries = 4096;  // queries per call (prefix table in shared m
 constexpr int kSelThreads = 1024;
 constexpr int kSliceCap = 40960;   // scores per CTA of the selection kernel
 constexpr int kMaxCluster = 16;   // CTAs per query in the selection kernel (above 8: non-portable)
+constexpr int kHistBins = 2048;   // bins of the score-key histogram the TMA scan leaves for the selection
 
 __device__ __forceinline__ int64_t query_visible(const IndexParams& p, int b) {
   const int64_t t = p.q_pos[b];
@@ -334,7 +341,12 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
   int* s_valid = reinterpret_cast<int*>(empty + NSTAGE);
   int* s_pref = s_valid + NSTAGE;
   __shared__ int s_wsum[32];
+  // digit-A histograms (top 11 bits of the score key) of the first and the last
+  // query of this CTA's unit range; a query strictly inside the range (short
+  // contexts) counts straight into the global histogram
+  __shared__ uint32_t s_h[2][kHistBins];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < 2 * kHistBins; i += kTmaThreads) (&s_h[0][0])[i] = 0u;
 
   {  // 64-key units per query, exclusive prefix
     int run = 0;
@@ -376,6 +388,12 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     b = lo;
     j0 = (u - s_pref[lo]) * kUnitKeys;
   };
+  int b_first = 0, b_last = 0;
+  if (n_units > 0) {
+    int64_t jx;
+    locate(u_begin, b_first, jx);
+    locate(u_begin + n_units - 1, b_last, jx);
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -508,31 +526,91 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
       }
       if (c == 0) {
         float* out = p.scores + (int64_t)b * p.vis_stride;
-        if (j + pg < nv) out[j + pg] = s0;
-        if (j + pg + 8 < nv) out[j + pg + 8] = s1;
+        uint32_t* hrow = b == b_first ? s_h[0] : b == b_last ? s_h[1] : nullptr;
+        uint32_t* gh = p.hist + (int64_t)b * kHistBins;
+        if (j + pg < nv) {
+          out[j + pg] = s0;
+          const uint32_t d = f2key(s0) >> 21;
+          atomicAdd(hrow ? hrow + d : gh + d, 1u);
+        }
+        if (j + pg + 8 < nv) {
+          out[j + pg + 8] = s1;
+          const uint32_t d = f2key(s1) >> 21;
+          atomicAdd(hrow ? hrow + d : gh + d, 1u);
+        }
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
   }
+  // consumers only (the producer warp has returned): flush the shared histograms
+  asm volatile("bar.sync 1, %0;\n" ::"r"(kTmaConsumerWarps * 32) : "memory");
+  if (n_units > 0) {
+    for (int i = tid - 32; i < 2 * kHistBins; i += kTmaConsumerWarps * 32) {
+      const int which = i / kHistBins, bin = i % kHistBins;
+      const uint32_t v = s_h[which][bin];
+      if (v) atomicAdd(p.hist + (int64_t)(which ? b_last : b_first) * kHistBins + bin, v);
+    }
+  }
 }
 
 // ---------------------------------------------------------------- top-k
-__device__ __forceinline__ int scan256_inclusive(int v, int* s_w) {
-  // threads 0..255 participate; returns the inclusive prefix over them
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(kFull, x, o);
-    if (lane >= o) x += y;
+// Radix select on 32-bit order-preserving keys with three digits:
+// A = bits 31..21 (2048 bins), B = bits 20..10 (2048 bins), C = bits 9..0
+// (1024 bins). Digit A's histogram comes from the scan (global, per query)
+// when the TMA scan ran, else from one pass over the slices. Keys whose digit
+// A equals the threshold digit are gathered into a short candidate list, and
+// digits B and C are counted over that list only; a threshold bin too large
+// for the list falls back to masked passes over the whole slice.
+constexpr int kBinsA = 2048, kBinsB = 2048, kBinsC = 1024;
+constexpr int kCandCap = 8192;  // candidate keys per CTA held in shared memory
+
+// count digit (key >> shift) & dmask of the keys of src[0, n) with (key & mask) == prefix
+__device__ __forceinline__ void hist_pass(const uint32_t* src, int n, uint32_t mask, uint32_t prefix, int shift,
+                                          uint32_t dmask, uint32_t* hist) {
+  const int lane = threadIdx.x & 31;
+  for (int base = 0; base < n; base += kSelThreads) {
+    const int i = base + threadIdx.x;
+    const uint32_t key = i < n ? src[i] : 0u;
+    const bool ok = i < n && (key & mask) == prefix;
+    const uint32_t dg = (key >> shift) & dmask;
+    const unsigned act = __ballot_sync(kFull, ok);
+    if (ok) {
+      const unsigned peers = __match_any_sync(act, dg);
+      if (lane == __ffs(peers) - 1) atomicAdd(&hist[dg], static_cast<uint32_t>(__popc(peers)));
+    }
   }
-  if (lane == 31) s_w[wid] = x;
-  asm volatile("bar.sync 1, 256;\n" ::);
-  int add = 0;
-  for (int w = 0; w < wid; ++w) add += s_w[w];
-  asm volatile("bar.sync 1, 256;\n" ::);
-  return x + add;
+}
+
+// The digit holding the krem-th largest key, given the count of every bin
+// (count(bin) for bin in [0, nbins)); bins are walked in descending order.
+// Every thread returns the same digit, the rank left inside its bin and the
+// bin's count. Uses every thread of the block.
+template <typename CountFn>
+__device__ __forceinline__ void find_digit(int nbins, int krem, CountFn count, int* s_w, uint32_t* s_res,
+                                           uint32_t& digit, int& krem_out, int& bin_cnt) {
+  const int per = nbins / kSelThreads;  // 1 or 2 bins per thread
+  int c[2] = {0, 0};
+  int tot = 0;
+  for (int e = 0; e < per; ++e) {
+    c[e] = count(nbins - 1 - (threadIdx.x * per + e));
+    tot += c[e];
+  }
+  int all;
+  int run = block_exclusive_scan<kSelThreads>(tot, s_w, all);
+  for (int e = 0; e < per; ++e) {
+    if (run < krem && krem <= run + c[e]) {
+      s_res[0] = static_cast<uint32_t>(nbins - 1 - (threadIdx.x * per + e));
+      s_res[1] = static_cast<uint32_t>(krem - run);
+      s_res[2] = static_cast<uint32_t>(c[e]);
+    }
+    run += c[e];
+  }
+  __syncthreads();
+  digit = s_res[0];
+  krem_out = static_cast<int>(s_res[1]);
+  bin_cnt = static_cast<int>(s_res[2]);
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParams p) {
@@ -541,12 +619,13 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
   const int rank = static_cast<int>(cluster.block_rank());
   const int b = blockIdx.x / CL;
   const int tid = threadIdx.x, lane = tid & 31;
-  extern __shared__ uint32_t s_keys[];
-  __shared__ uint32_t s_hist[4][256];
+  extern __shared__ uint32_t s_keys[];  // [slice] keys, then [kCandCap] candidates
+  uint32_t* s_cand = s_keys + p.slice;
+  __shared__ uint32_t s_hA[kBinsA], s_hB[kBinsB], s_hC[kBinsC];
   __shared__ int s_w[32];
+  __shared__ uint32_t s_res[3];
   __shared__ int s_cnt[2];
-  __shared__ uint32_t s_digit;
-  __shared__ int s_krem;
+  __shared__ int s_ncand;
 
   const int k = p.k;
   int64_t nv = query_visible(p, b);
@@ -567,49 +646,101 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
   const int64_t lo = (int64_t)rank * p.slice;
   const int64_t hi = lo + p.slice < nv ? lo + p.slice : nv;
   const int len = hi > lo ? static_cast<int>(hi - lo) : 0;
-  for (int i = tid; i < len; i += kSelThreads) s_keys[i] = f2key(sc[lo + i]);
-  for (int i = tid; i < 4 * 256; i += kSelThreads) (&s_hist[0][0])[i] = 0u;
+  {  // slice -> keys; four 16-byte loads in flight per thread (lo and the row start are 16-byte aligned)
+    const float4* src4 = reinterpret_cast<const float4*>(sc + lo);
+    const int n4 = len >> 2;
+    for (int base = 0; base < n4; base += 4 * kSelThreads) {
+      float4 v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = base + e * kSelThreads + tid;
+        v[e] = i < n4 ? __ldg(src4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = base + e * kSelThreads + tid;
+        if (i < n4)
+          reinterpret_cast<uint4*>(s_keys)[i] = make_uint4(f2key(v[e].x), f2key(v[e].y), f2key(v[e].z), f2key(v[e].w));
+      }
+    }
+    for (int i = (n4 << 2) + tid; i < len; i += kSelThreads) s_keys[i] = f2key(sc[lo + i]);
+  }
+  for (int i = tid; i < kBinsA; i += kSelThreads) s_hA[i] = 0u;
+  for (int i = tid; i < kBinsB; i += kSelThreads) s_hB[i] = 0u;
+  for (int i = tid; i < kBinsC; i += kSelThreads) s_hC[i] = 0u;
+  if (tid == 0) {
+    s_ncand = 0;
+    s_res[0] = s_res[1] = s_res[2] = 0u;
+  }
   __syncthreads();
 
-  uint32_t prefix = 0u, mask = 0u;
-  int krem = k;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
+  // digit A
+  uint32_t dA;
+  int krem, nA;
+  if (p.hist) {
+    const uint32_t* gh = p.hist + (int64_t)b * kBinsA;
+    find_digit(kBinsA, k, [&](int bin) { return static_cast<int>(__ldg(gh + bin)); }, s_w, s_res, dA, krem, nA);
+  } else {
+    hist_pass(s_keys, len, 0u, 0u, 21, kBinsA - 1, s_hA);
+    cluster.sync();
+    find_digit(kBinsA, k, [&](int bin) {
+      uint32_t part[kMaxCluster];
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r) part[r] = r < CL ? *cluster.map_shared_rank(&s_hA[bin], r) : 0u;
+      int c = 0;
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r) c += static_cast<int>(part[r]);
+      return c;
+    }, s_w, s_res, dA, krem, nA);
+  }
+  uint32_t prefix = dA << 21, mask = 0xFFE00000u;
+
+  // digit B: over the gathered candidates when they fit (the bin's count is the cluster's total)
+  const bool gathered = nA <= kCandCap;
+  if (gathered) {
+    const unsigned below = (1u << lane) - 1u;
     for (int base = 0; base < len; base += kSelThreads) {
       const int i = base + tid;
       const uint32_t key = i < len ? s_keys[i] : 0u;
-      const bool ok = i < len && (key & mask) == prefix;
-      const uint32_t dg = (key >> shift) & 255u;
-      const unsigned act = __ballot_sync(kFull, ok);
-      if (ok) {
-        const unsigned peers = __match_any_sync(act, dg);
-        if (lane == __ffs(peers) - 1) atomicAdd(&s_hist[pass][dg], static_cast<uint32_t>(__popc(peers)));
+      const bool cand = i < len && (key & mask) == prefix;
+      const unsigned m = __ballot_sync(kFull, cand);
+      if (m) {
+        int at = 0;
+        if (lane == __ffs(m) - 1) at = atomicAdd(&s_ncand, __popc(m));
+        at = __shfl_sync(kFull, at, __ffs(m) - 1);
+        at += __popc(m & below);
+        if (cand && at < kCandCap) {  // always true while the scan's histogram matches the scores
+          s_cand[at] = key;
+          atomicAdd(&s_hB[(key >> 10) & (kBinsB - 1)], 1u);
+        }
       }
     }
-    cluster.sync();
-    if (tid < 256) {
-      const int bin = 255 - tid;  // descending digit order
-      int cnt = 0;
+  } else {
+    hist_pass(s_keys, len, mask, prefix, 10, kBinsB - 1, s_hB);
+  }
+  cluster.sync();
+  auto remote_count = [&](const uint32_t* h) {
+    return [&, h](int bin) {
       uint32_t part[kMaxCluster];
 #pragma unroll
-      for (int r = 0; r < kMaxCluster; ++r)  // all remote loads in flight before the sum
-        part[r] = r < CL ? *cluster.map_shared_rank(&s_hist[pass][bin], r) : 0u;
+      for (int r = 0; r < kMaxCluster; ++r) part[r] = r < CL ? *cluster.map_shared_rank(h + bin, r) : 0u;
+      int c = 0;
 #pragma unroll
-      for (int r = 0; r < kMaxCluster; ++r) cnt += static_cast<int>(part[r]);
-      const int incl = scan256_inclusive(cnt, s_w);
-      const int excl = incl - cnt;
-      if (excl < krem && krem <= incl) {
-        s_digit = static_cast<uint32_t>(bin);
-        s_krem = krem - excl;
-      }
-    }
-    __syncthreads();
-    prefix |= s_digit << shift;
-    mask |= 255u << shift;
-    krem = s_krem;
-    __syncthreads();
-  }
-  const uint32_t T = prefix;  // the k-th largest key; take the first krem keys equal to T
+      for (int r = 0; r < kMaxCluster; ++r) c += static_cast<int>(part[r]);
+      return c;
+    };
+  };
+  uint32_t dB, dC;
+  int nB, nC;
+  find_digit(kBinsB, krem, remote_count(s_hB), s_w, s_res, dB, krem, nB);
+  prefix |= dB << 10;
+  mask |= 0x001FFC00u;
+  const uint32_t* src = gathered ? s_cand : s_keys;
+  const int n_src = gathered ? min(s_ncand, kCandCap) : len;
+  hist_pass(src, n_src, mask, prefix, 0, kBinsC - 1, s_hC);
+  cluster.sync();
+  find_digit(kBinsC, krem, remote_count(s_hC), s_w, s_res, dC, krem, nC);
+  const uint32_t T = prefix | dC;  // the k-th largest key; take the first krem keys equal to T
 
   // Ordered output. Warp w owns the contiguous segment [w*seg, (w+1)*seg) of
   // this CTA's slice. Pass 1 counts, per warp, keys above T and equal to T;
@@ -686,6 +817,34 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
   cluster.sync();  // peers may still read this CTA's shared memory
 }
 
+// Clusters of `cl` selection CTAs that can be resident at once on the current
+// device, cached per (device, cl, shared memory); 0 if the shape cannot launch.
+int max_active_clusters(int cl, size_t smem, const cudaLaunchConfig_t* cfg) {
+  struct Entry {
+    int dev, cl;
+    size_t smem;
+    int fit;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& en : cache)
+      if (en.dev == dev && en.cl == cl && en.smem == smem) return en.fit;
+  }
+  if (!cfg) return 0;
+  int fit = 0;
+  if (cudaOccupancyMaxActiveClusters(&fit, index_select_kernel, cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    fit = 0;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  cache.push_back({dev, cl, smem, fit});
+  return fit;
+}
+
 template <int NCH, int NTH, int TPW, bool FP4>
 cudaError_t launch_scan(IndexParams& p, int n_sm, cudaStream_t st) {
   auto kern = index_scan_kernel<NCH, NTH, TPW, FP4>;
@@ -698,19 +857,6 @@ cudaError_t launch_scan(IndexParams& p, int n_sm, cudaStream_t st) {
   if (grid < 1) grid = 1;
   kern<<<static_cast<int>(grid), kScanThreads, smem, st>>>(p);
   return cudaGetLastError();
-}
-
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link)
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }();
-  return fn;
 }
 
 template <int NCH, int NTH>
@@ -740,16 +886,30 @@ cudaError_t launch_scan_tma(IndexParams& p, int n_sm, cudaStream_t st) {
 
 }  // namespace
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link)
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
 size_t index_ws_bytes(int n_q, int64_t max_pos, int m, int n_win) {
   const int64_t nv = visible_entries(max_pos, m, n_win);
   const int64_t stride = (nv + 63) / 64 * 64;
-  return sizeof(float) * static_cast<size_t>(stride) * static_cast<size_t>(n_q) + 256;
+  return (sizeof(float) * static_cast<size_t>(stride) + sizeof(uint32_t) * kHistBins) * static_cast<size_t>(n_q) + 256;
 }
 
 cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st) {
   const int64_t nv_max = visible_entries(p.max_pos, p.m, p.n_win);
   p.vis_stride = (nv_max + 63) / 64 * 64;
   p.scores = static_cast<float*>(ws);
+  p.hist = nullptr;
   if (p.n_q > kMaxQueries) return cudaErrorInvalidValue;
   cudaError_t e = cudaSuccess;
   const bool fp4 = p.idx_dtype == CSKV_FP4_E2M1;
@@ -758,6 +918,9 @@ cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st) {
                       (reinterpret_cast<uintptr_t>(p.idx_pool) & 15u) == 0 &&
                       (int64_t)p.n_pages * p.page_size < (int64_t(1) << 31);
   if (nv_max > 0 && tma_ok) {
+    p.hist = reinterpret_cast<uint32_t*>(p.scores + (size_t)p.n_q * p.vis_stride);
+    e = cudaMemsetAsync(p.hist, 0, sizeof(uint32_t) * kHistBins * (size_t)p.n_q, st);
+    if (e != cudaSuccess) return e;
     if (p.d_idx == 64 && nth == 1) e = launch_scan_tma<2, 1>(p, n_sm, st);
     else if (p.d_idx == 64 && nth == 2) e = launch_scan_tma<2, 2>(p, n_sm, st);
     else if (p.d_idx == 128 && nth == 1) e = launch_scan_tma<4, 1>(p, n_sm, st);
@@ -778,52 +941,54 @@ cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st) {
   int cl_min = static_cast<int>((nv_max + kSliceCap - 1) / kSliceCap);
   if (cl_min < 1) cl_min = 1;
   if (cl_min > kMaxCluster) return cudaErrorNotSupported;
-  int cl_par = n_sm / (p.n_q > 0 ? p.n_q : 1);
-  if (cl_par > kMaxCluster) cl_par = kMaxCluster;
-  int cl = cl_min > cl_par ? cl_min : cl_par;
-  if (cl < 1) cl = 1;
+  if (p.n_q == 0) return cudaSuccess;
+  int cl0 = n_sm / p.n_q;
+  if (cl0 > kMaxCluster) cl0 = kMaxCluster;
+  if (cl0 < cl_min) cl0 = cl_min;
   // no point in CTAs that would hold fewer than 4096 scores
-  while (cl > cl_min && (nv_max + cl - 1) / cl < 4096) --cl;
-  p.cluster = cl;
-  p.slice = static_cast<int>(((nv_max + cl - 1) / cl + 3) / 4 * 4);
-  if (p.slice < 4) p.slice = 4;
-  const size_t smem = sizeof(uint32_t) * static_cast<size_t>(p.slice);
+  while (cl0 > cl_min && (nv_max + cl0 - 1) / cl0 < 4096) --cl0;
   e = cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem));
+                           static_cast<int>(sizeof(uint32_t) * (kSliceCap + kCandCap)));
   if (e != cudaSuccess) return e;
-  if (cl > 8) {
+  if (cl0 > 8) {
     e = cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
-  if (p.n_q == 0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(p.n_q * cl), 1, 1);
   cfg.blockDim = dim3(kSelThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(cl);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cl > 8) {  // a non-portable cluster must fit in one GPC; else fall back to 8
-    int n_clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&n_clusters, index_select_kernel, &cfg) != cudaSuccess || n_clusters < 1) {
-      (void)cudaGetLastError();
-      if (cl_min > 8) return cudaErrorNotSupported;
-      cl = 8;
-      p.cluster = cl;
-      p.slice = static_cast<int>(((nv_max + cl - 1) / cl + 3) / 4 * 4);
-      cfg.gridDim = dim3(static_cast<unsigned>(p.n_q * cl), 1, 1);
-      cfg.dynamicSmemBytes = sizeof(uint32_t) * static_cast<size_t>(p.slice);
-      attr[0].val.clusterDim.x = static_cast<unsigned>(cl);
-      e = cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(cfg.dynamicSmemBytes));
-      if (e != cudaSuccess) return e;
+  auto shape = [&](int cl) {
+    p.cluster = cl;
+    p.slice = static_cast<int>(((nv_max + cl - 1) / cl + 3) / 4 * 4);
+    if (p.slice < 4) p.slice = 4;
+    cfg.gridDim = dim3(static_cast<unsigned>(p.n_q * cl), 1, 1);
+    cfg.dynamicSmemBytes = sizeof(uint32_t) * (static_cast<size_t>(p.slice) + kCandCap);
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cl);
+  };
+  // The largest cluster, down from cl0, whose n_q clusters are all resident at
+  // once (a second wave would double the time); clusters above 8 CTAs must fit
+  // in one GPC, which not every GPC can host. If none fits in one wave, the
+  // largest portable size.
+  int chosen = -1;
+  for (int cl = cl0; cl >= cl_min && chosen < 0; --cl) {
+    shape(cl);
+    const int fit = max_active_clusters(cl, cfg.dynamicSmemBytes, &cfg);
+    if (fit >= p.n_q) chosen = cl;
+  }
+  if (chosen < 0) {
+    chosen = cl0 < 8 ? cl0 : (cl_min > 8 ? cl_min : 8);
+    if (chosen > 8) {
+      shape(chosen);
+      if (max_active_clusters(chosen, cfg.dynamicSmemBytes, &cfg) < 1) return cudaErrorNotSupported;
     }
   }
+  shape(chosen);
   return cudaLaunchKernelEx(&cfg, index_select_kernel, p);
 }
 
