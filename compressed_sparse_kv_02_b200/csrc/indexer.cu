@@ -40,9 +40,17 @@ namespace {
 constexpr int kScanThreads = 256;
 constexpr int kMaxQueries = 4096;  // queries per call (prefix table in shared memory)
 constexpr int kSelThreads = 1024;
-constexpr int kSliceCap = 40960;   // scores per CTA of the selection kernel
+constexpr int kSliceCap = 32768;   // scores per CTA of the selection kernel
 constexpr int kMaxCluster = 16;   // CTAs per query in the selection kernel (above 8: non-portable)
 constexpr int kHistBins = 2048;   // bins of the score-key histogram the TMA scan leaves for the selection
+
+// Programmatic dependent launch: a kernel launched behind this one may start
+// once every CTA here has called grid_dependents_launch (or exited); it calls
+// grid_dependency_wait before it reads anything this grid writes, which waits
+// for this whole grid to finish and its writes to be visible. Both are no-ops
+// for plain launches.
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 
 __device__ __forceinline__ int64_t query_visible(const IndexParams& p, int b) {
   const int64_t t = p.q_pos[b];
@@ -346,6 +354,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
   // contexts) counts straight into the global histogram
   __shared__ uint32_t s_h[2][kHistBins];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  grid_dependents_launch();  // the selection kernel may be scheduled as SMs free up
   for (int i = tid; i < 2 * kHistBins; i += kTmaThreads) (&s_h[0][0])[i] = 0u;
 
   {  // 64-key units per query, exclusive prefix
@@ -582,6 +591,15 @@ __device__ __forceinline__ void hist_pass(const uint32_t* src, int n, uint32_t m
   }
 }
 
+// the same over a short list with keys spread over many bins: one atomic per key
+__device__ __forceinline__ void hist_pass_sparse(const uint32_t* src, int n, uint32_t mask, uint32_t prefix,
+                                                 int shift, uint32_t dmask, uint32_t* hist) {
+  for (int i = threadIdx.x; i < n; i += kSelThreads) {
+    const uint32_t key = src[i];
+    if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
+  }
+}
+
 // The digit holding the krem-th largest key, given the count of every bin
 // (count(bin) for bin in [0, nbins)); bins are walked in descending order.
 // Every thread returns the same digit, the rank left inside its bin and the
@@ -613,26 +631,63 @@ __device__ __forceinline__ void find_digit(int nbins, int krem, CountFn count, i
   __syncthreads();
 }
 
+__device__ __forceinline__ int warp_exclusive_scan(int v, int lane) {
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, x, o);
+    if (lane >= o) x += y;
+  }
+  return x - v;
+}
+
+
 __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParams p) {
   cg::cluster_group cluster = cg::this_cluster();
   const int CL = p.cluster;
   const int rank = static_cast<int>(cluster.block_rank());
   const int b = blockIdx.x / CL;
-  const int tid = threadIdx.x, lane = tid & 31;
-  extern __shared__ uint32_t s_keys[];  // [slice] keys, then [kCandCap] candidates
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  // [slice] keys | [kCandCap] this CTA's candidates | [kCandCap] the cluster's candidates
+  extern __shared__ __align__(16) uint32_t s_keys[];
   uint32_t* s_cand = s_keys + p.slice;
+  uint32_t* s_all = s_cand + kCandCap;
   __shared__ uint32_t s_hA[kBinsA], s_hB[kBinsB], s_hC[kBinsC];
   __shared__ int s_w[32];
   __shared__ uint32_t s_res[3];
   __shared__ int s_cnt[2];
   __shared__ int s_ncand;
+  __shared__ __align__(8) uint64_t s_bar;
+  __shared__ int s_peer[2 * kMaxCluster];
+  constexpr int NW = kSelThreads / 32;
+  __shared__ int s_wgt[NW], s_weq[NW];
 
+  for (int i = tid; i < kBinsA; i += kSelThreads) s_hA[i] = 0u;
+  for (int i = tid; i < kBinsB; i += kSelThreads) s_hB[i] = 0u;
+  for (int i = tid; i < kBinsC; i += kSelThreads) s_hC[i] = 0u;
+  if (tid == 0) {
+    s_ncand = 0;
+    s_res[0] = s_res[1] = s_res[2] = 0u;
+    mbar_init(&s_bar, 1);
+    fence_barrier_init();
+  }
   const int k = p.k;
   int64_t nv = query_visible(p, b);
   if (nv < 0) nv = 0;
   const float* sc = p.scores + (int64_t)b * p.vis_stride;
   int32_t* oidx = p.out_idx + (int64_t)b * k;
   float* osc = p.out_scores ? p.out_scores + (int64_t)b * k : nullptr;
+  const int64_t lo = (int64_t)rank * p.slice;
+  const int64_t hi = lo + p.slice < nv ? lo + p.slice : nv;
+  const int len = hi > lo ? static_cast<int>(hi - lo) : 0;
+  grid_dependency_wait();  // the scores and the digit-A histogram come from the scan
+  __syncthreads();
+  // the slice's scores (whole 16-byte pieces) land by one bulk copy while digit A is found
+  const int n4 = nv > k ? len >> 2 : 0;
+  if (tid == 0 && n4 > 0) {
+    mbar_arrive_expect_tx(&s_bar, static_cast<uint32_t>(n4) * 16u);
+    bulk_load(s_keys, sc + lo, static_cast<uint32_t>(n4) * 16u, &s_bar);
+  }
 
   if (nv <= k) {  // everything visible is chosen (uniform across the cluster)
     for (int64_t i = (int64_t)rank * kSelThreads + tid; i < k; i += (int64_t)CL * kSelThreads) {
@@ -643,44 +698,57 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
     return;
   }
 
-  const int64_t lo = (int64_t)rank * p.slice;
-  const int64_t hi = lo + p.slice < nv ? lo + p.slice : nv;
-  const int len = hi > lo ? static_cast<int>(hi - lo) : 0;
-  {  // slice -> keys; four 16-byte loads in flight per thread (lo and the row start are 16-byte aligned)
-    const float4* src4 = reinterpret_cast<const float4*>(sc + lo);
-    const int n4 = len >> 2;
-    for (int base = 0; base < n4; base += 4 * kSelThreads) {
-      float4 v[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = base + e * kSelThreads + tid;
-        v[e] = i < n4 ? __ldg(src4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = base + e * kSelThreads + tid;
-        if (i < n4)
-          reinterpret_cast<uint4*>(s_keys)[i] = make_uint4(f2key(v[e].x), f2key(v[e].y), f2key(v[e].z), f2key(v[e].w));
-      }
-    }
-    for (int i = (n4 << 2) + tid; i < len; i += kSelThreads) s_keys[i] = f2key(sc[lo + i]);
-  }
-  for (int i = tid; i < kBinsA; i += kSelThreads) s_hA[i] = 0u;
-  for (int i = tid; i < kBinsB; i += kSelThreads) s_hB[i] = 0u;
-  for (int i = tid; i < kBinsC; i += kSelThreads) s_hC[i] = 0u;
-  if (tid == 0) {
-    s_ncand = 0;
-    s_res[0] = s_res[1] = s_res[2] = 0u;
-  }
-  __syncthreads();
-
-  // digit A
-  uint32_t dA;
-  int krem, nA;
+  // digit A from the scan's histogram, when there is one (identical in every CTA)
+  uint32_t dA = 0u;
+  int krem = k, nA = 0;
   if (p.hist) {
     const uint32_t* gh = p.hist + (int64_t)b * kBinsA;
-    find_digit(kBinsA, k, [&](int bin) { return static_cast<int>(__ldg(gh + bin)); }, s_w, s_res, dA, krem, nA);
-  } else {
+    find_digit(kBinsA, k, [&](int bin) { return static_cast<int>(gh[bin]); }, s_w, s_res, dA, krem, nA);
+  }
+  const uint32_t maskA = 0xFFE00000u;
+  const unsigned below = (1u << lane) - 1u;
+  // appends the keys of digit dA among the flagged ones to this CTA's candidate list
+  auto gather = [&](uint32_t key, bool cand) {
+    const unsigned m = __ballot_sync(kFull, cand);
+    if (m) {
+      int at = 0;
+      if (lane == __ffs(m) - 1) at = atomicAdd(&s_ncand, __popc(m));
+      at = __shfl_sync(kFull, at, __ffs(m) - 1) + __popc(m & below);
+      if (cand && at < kCandCap) s_cand[at] = key;  // always true while the histogram matches the scores
+    }
+  };
+  {  // scores -> keys in place; the candidates of digit dA are gathered on the way
+    const bool gather_now = p.hist && nA <= kCandCap;
+    const uint32_t pre = dA << 21;
+    if (n4 > 0 && !mbar_wait(&s_bar, 0u, p.status)) {
+      // the copy never completed: leave the (undefined) slice as it is; the status word says why
+    }
+    uint4* k4 = reinterpret_cast<uint4*>(s_keys);
+    for (int base = 0; base < n4; base += kSelThreads) {
+      const int i = base + tid;
+      uint4 kv = make_uint4(0u, 0u, 0u, 0u);
+      if (i < n4) {
+        const uint4 fv = k4[i];
+        kv = make_uint4(f2key(__uint_as_float(fv.x)), f2key(__uint_as_float(fv.y)), f2key(__uint_as_float(fv.z)),
+                        f2key(__uint_as_float(fv.w)));
+        k4[i] = kv;
+      }
+      if (gather_now) {
+        gather(kv.x, i < n4 && (kv.x & maskA) == pre);
+        gather(kv.y, i < n4 && (kv.y & maskA) == pre);
+        gather(kv.z, i < n4 && (kv.z & maskA) == pre);
+        gather(kv.w, i < n4 && (kv.w & maskA) == pre);
+      }
+    }
+    for (int base = n4 << 2; base < len; base += kSelThreads) {  // the last 0..3 keys
+      const int i = base + tid;
+      const uint32_t key = i < len ? f2key(sc[lo + i]) : 0u;
+      if (i < len) s_keys[i] = key;
+      if (gather_now) gather(key, i < len && (key & maskA) == pre);
+    }
+  }
+  __syncthreads();
+  if (!p.hist) {  // digit A over the slices, then the candidates
     hist_pass(s_keys, len, 0u, 0u, 21, kBinsA - 1, s_hA);
     cluster.sync();
     find_digit(kBinsA, k, [&](int bin) {
@@ -692,72 +760,114 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
       for (int r = 0; r < kMaxCluster; ++r) c += static_cast<int>(part[r]);
       return c;
     }, s_w, s_res, dA, krem, nA);
+    if (nA <= kCandCap)
+      for (int base = 0; base < len; base += kSelThreads) {
+        const int i = base + tid;
+        const uint32_t key = i < len ? s_keys[i] : 0u;
+        gather(key, i < len && (key & maskA) == (dA << 21));
+      }
   }
-  uint32_t prefix = dA << 21, mask = 0xFFE00000u;
-
-  // digit B: over the gathered candidates when they fit (the bin's count is the cluster's total)
-  const bool gathered = nA <= kCandCap;
-  if (gathered) {
-    const unsigned below = (1u << lane) - 1u;
-    for (int base = 0; base < len; base += kSelThreads) {
-      const int i = base + tid;
-      const uint32_t key = i < len ? s_keys[i] : 0u;
-      const bool cand = i < len && (key & mask) == prefix;
-      const unsigned m = __ballot_sync(kFull, cand);
-      if (m) {
-        int at = 0;
-        if (lane == __ffs(m) - 1) at = atomicAdd(&s_ncand, __popc(m));
-        at = __shfl_sync(kFull, at, __ffs(m) - 1);
-        at += __popc(m & below);
-        if (cand && at < kCandCap) {  // always true while the scan's histogram matches the scores
-          s_cand[at] = key;
-          atomicAdd(&s_hB[(key >> 10) & (kBinsB - 1)], 1u);
-        }
+  uint32_t prefix = dA << 21, mask = maskA;
+  uint32_t dB = 0u, dC = 0u;
+  int nB = 0, nC = 0;
+  if (nA <= kCandCap) {
+    // every CTA copies the cluster's candidates (nA keys in all) and finishes the select alone
+    cluster.sync();
+    __shared__ int s_pn[kMaxCluster + 1], s_pq[kMaxCluster + 1];  // prefix of keys / 16-byte pieces per peer
+    if (tid == 0) {
+      int nk = 0, nq = 0;
+      for (int r = 0; r < CL; ++r) {
+        s_pn[r] = nk;
+        s_pq[r] = nq;
+        const int n_r = min(*cluster.map_shared_rank(&s_ncand, r), kCandCap);
+        nk += n_r;
+        nq += (n_r + 3) >> 2;
+      }
+      s_pn[CL] = nk;
+      s_pq[CL] = nq;
+    }
+    __syncthreads();
+    const int n_all = min(s_pn[CL], kCandCap);
+    for (int t = tid; t < s_pq[CL]; t += kSelThreads) {  // one 16-byte piece of a peer's list per thread
+      int r = 0;
+      while (r + 1 < CL && s_pq[r + 1] <= t) ++r;
+      const int piece = t - s_pq[r];
+      const int n_r = s_pn[r + 1] - s_pn[r];
+      const uint4 v = reinterpret_cast<const uint4*>(cluster.map_shared_rank(s_cand, r))[piece];
+      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = piece * 4 + e, o = s_pn[r] + j;
+        if (j < n_r && o < kCandCap) s_all[o] = vv[e];
       }
     }
+    __syncthreads();
+    hist_pass_sparse(s_all, n_all, mask, prefix, 10, kBinsB - 1, s_hB);
+    __syncthreads();
+    find_digit(kBinsB, krem, [&](int bin) { return static_cast<int>(s_hB[bin]); }, s_w, s_res, dB, krem, nB);
+    prefix |= dB << 10;
+    mask |= 0x001FFC00u;
+    hist_pass_sparse(s_all, n_all, mask, prefix, 0, kBinsC - 1, s_hC);
+    __syncthreads();
+    find_digit(kBinsC, krem, [&](int bin) { return static_cast<int>(s_hC[bin]); }, s_w, s_res, dC, krem, nC);
   } else {
-    hist_pass(s_keys, len, mask, prefix, 10, kBinsB - 1, s_hB);
-  }
-  cluster.sync();
-  auto remote_count = [&](const uint32_t* h) {
-    return [&, h](int bin) {
-      uint32_t part[kMaxCluster];
+    // a threshold bin too large for the lists: masked passes over the slices, histograms summed over the cluster
+    auto remote_count = [&](const uint32_t* h) {
+      return [&, h](int bin) {
+        uint32_t part[kMaxCluster];
 #pragma unroll
-      for (int r = 0; r < kMaxCluster; ++r) part[r] = r < CL ? *cluster.map_shared_rank(h + bin, r) : 0u;
-      int c = 0;
+        for (int r = 0; r < kMaxCluster; ++r) part[r] = r < CL ? *cluster.map_shared_rank(h + bin, r) : 0u;
+        int c = 0;
 #pragma unroll
-      for (int r = 0; r < kMaxCluster; ++r) c += static_cast<int>(part[r]);
-      return c;
+        for (int r = 0; r < kMaxCluster; ++r) c += static_cast<int>(part[r]);
+        return c;
+      };
     };
-  };
-  uint32_t dB, dC;
-  int nB, nC;
-  find_digit(kBinsB, krem, remote_count(s_hB), s_w, s_res, dB, krem, nB);
-  prefix |= dB << 10;
-  mask |= 0x001FFC00u;
-  const uint32_t* src = gathered ? s_cand : s_keys;
-  const int n_src = gathered ? min(s_ncand, kCandCap) : len;
-  hist_pass(src, n_src, mask, prefix, 0, kBinsC - 1, s_hC);
-  cluster.sync();
-  find_digit(kBinsC, krem, remote_count(s_hC), s_w, s_res, dC, krem, nC);
+    hist_pass(s_keys, len, mask, prefix, 10, kBinsB - 1, s_hB);
+    cluster.sync();
+    find_digit(kBinsB, krem, remote_count(s_hB), s_w, s_res, dB, krem, nB);
+    prefix |= dB << 10;
+    mask |= 0x001FFC00u;
+    hist_pass(s_keys, len, mask, prefix, 0, kBinsC - 1, s_hC);
+    cluster.sync();
+    find_digit(kBinsC, krem, remote_count(s_hC), s_w, s_res, dC, krem, nC);
+  }
   const uint32_t T = prefix | dC;  // the k-th largest key; take the first krem keys equal to T
 
   // Ordered output. Warp w owns the contiguous segment [w*seg, (w+1)*seg) of
-  // this CTA's slice. Pass 1 counts, per warp, keys above T and equal to T;
-  // the counts are scanned over the warps of the CTA and then over the CTAs
-  // of the cluster; pass 2 writes the chosen ids in index order.
-  constexpr int NW = kSelThreads / 32;
-  const int wid = tid >> 5;
-  const int seg = ((len + NW - 1) / NW + 31) / 32 * 32;
+  // this CTA's slice (seg a multiple of 128: 4 keys per lane per step). Pass
+  // 1 counts, per warp, keys above T and equal to T; the counts are scanned
+  // over the warps of the CTA and then over the CTAs of the cluster; pass 2
+  // writes the chosen ids in index order.
+  const int seg = ((len + NW - 1) / NW + 127) / 128 * 128;
   const int s_lo = wid * seg, s_hi = min(len, s_lo + seg);
+  auto keys4 = [&](int i, uint32_t (&kk)[4], unsigned& valid) {
+    if (i + 3 < s_hi) {
+      const uint4 v = *reinterpret_cast<const uint4*>(s_keys + i);
+      kk[0] = v.x; kk[1] = v.y; kk[2] = v.z; kk[3] = v.w;
+      valid = 15u;
+    } else {
+      valid = 0u;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        kk[e] = i + e < s_hi ? s_keys[i + e] : 0u;
+        valid |= (i + e < s_hi ? 1u : 0u) << e;
+      }
+    }
+  };
   int gt = 0, eq = 0;
-  for (int base = s_lo; base < s_hi; base += 32) {
-    const int i = base + lane;
-    const uint32_t key = i < s_hi ? s_keys[i] : 0u;
-    gt += __popc(__ballot_sync(kFull, i < s_hi && key > T));
-    eq += __popc(__ballot_sync(kFull, i < s_hi && key == T));
+  for (int base = s_lo; base < s_hi; base += 128) {
+    uint32_t kk[4];
+    unsigned valid;
+    keys4(base + 4 * lane, kk, valid);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      gt += ((valid >> e) & 1u) && kk[e] > T;
+      eq += ((valid >> e) & 1u) && kk[e] == T;
+    }
   }
-  __shared__ int s_wgt[NW], s_weq[NW];
+  gt = __reduce_add_sync(kFull, gt);
+  eq = __reduce_add_sync(kFull, eq);
   if (lane == 0) {
     s_wgt[wid] = gt;
     s_weq[wid] = eq;
@@ -773,11 +883,13 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
     s_cnt[1] = te;
   }
   cluster.sync();
+  if (tid < 2 * CL) s_peer[tid] = *cluster.map_shared_rank(&s_cnt[tid & 1], tid >> 1);  // one remote read each
+  __syncthreads();
   // ties are taken in index order: CTA r may take krem minus the ties of CTAs before it
   int eq_before = 0, sel_before = 0, take_eq = 0;
   for (int r = 0; r < CL; ++r) {
-    const int g_r = *cluster.map_shared_rank(&s_cnt[0], r);
-    const int e_r = *cluster.map_shared_rank(&s_cnt[1], r);
+    const int g_r = s_peer[2 * r];
+    const int e_r = s_peer[2 * r + 1];
     int t_r = krem - eq_before;
     t_r = t_r < 0 ? 0 : (t_r > e_r ? e_r : t_r);
     if (r < rank) {
@@ -797,21 +909,42 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
     w_eq_before += s_weq[w];
   }
   int run_eq = w_eq_before, run_sel = w_sel_before;
-  const unsigned lt = (1u << lane) - 1u;
-  for (int base = s_lo; base < s_hi; base += 32) {
-    const int i = base + lane;
-    const uint32_t key = i < s_hi ? s_keys[i] : 0u;
-    const unsigned m_eq = __ballot_sync(kFull, i < s_hi && key == T);
-    const int eq_rank = run_eq + __popc(m_eq & lt);
-    const bool sel = (i < s_hi && key > T) || ((m_eq >> lane) & 1u && eq_rank < take_eq);
-    const unsigned m_sel = __ballot_sync(kFull, sel);
-    const int at = run_sel + __popc(m_sel & lt);
-    if (sel && at < k) {
-      oidx[at] = static_cast<int32_t>(lo + i);
-      if (osc) osc[at] = key2f(key);
+  for (int base = s_lo; base < s_hi; base += 128) {
+    const int i = base + 4 * lane;
+    uint32_t kk[4];
+    unsigned valid;
+    keys4(i, kk, valid);
+    int e_l = 0, g_l = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      e_l += ((valid >> e) & 1u) && kk[e] == T;
+      g_l += ((valid >> e) & 1u) && kk[e] > T;
     }
-    run_eq += __popc(m_eq);
-    run_sel += __popc(m_sel);
+    if (!__any_sync(kFull, (e_l | g_l) != 0)) continue;  // nothing chosen in these 128 keys
+    int eq_rank = run_eq + warp_exclusive_scan(e_l, lane);
+    bool sel[4];
+    int s_l = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const bool v = (valid >> e) & 1u;
+      const bool is_eq = v && kk[e] == T;
+      sel[e] = (v && kk[e] > T) || (is_eq && eq_rank < take_eq);
+      eq_rank += is_eq;
+      s_l += sel[e];
+    }
+    int at = run_sel + warp_exclusive_scan(s_l, lane);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (sel[e]) {
+        if (at < k) {
+          oidx[at] = static_cast<int32_t>(lo + i + e);
+          if (osc) osc[at] = key2f(kk[e]);
+        }
+        ++at;
+      }
+    }
+    run_eq += __reduce_add_sync(kFull, e_l);
+    run_sel += __reduce_add_sync(kFull, s_l);
   }
   if (rank == 0 && tid == 0) p.out_cnt[b] = k;
   cluster.sync();  // peers may still read this CTA's shared memory
@@ -948,7 +1081,7 @@ cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st) {
   // no point in CTAs that would hold fewer than 4096 scores
   while (cl0 > cl_min && (nv_max + cl0 - 1) / cl0 < 4096) --cl0;
   e = cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(sizeof(uint32_t) * (kSliceCap + kCandCap)));
+                           static_cast<int>(sizeof(uint32_t) * (kSliceCap + 2 * kCandCap)));
   if (e != cudaSuccess) return e;
   if (cl0 > 8) {
     e = cudaFuncSetAttribute(index_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -957,18 +1090,22 @@ cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kSelThreads, 1, 1);
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent launch: CTAs start on SMs the scan has left and wait
+  // (griddepcontrol.wait) for its scores before reading them
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   auto shape = [&](int cl) {
     p.cluster = cl;
     p.slice = static_cast<int>(((nv_max + cl - 1) / cl + 3) / 4 * 4);
     if (p.slice < 4) p.slice = 4;
     cfg.gridDim = dim3(static_cast<unsigned>(p.n_q * cl), 1, 1);
-    cfg.dynamicSmemBytes = sizeof(uint32_t) * (static_cast<size_t>(p.slice) + kCandCap);
+    cfg.dynamicSmemBytes = sizeof(uint32_t) * (static_cast<size_t>(p.slice) + 2 * kCandCap);
     attr[0].val.clusterDim.x = static_cast<unsigned>(cl);
   };
   // The largest cluster, down from cl0, whose n_q clusters are all resident at
