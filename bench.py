@@ -138,6 +138,27 @@ def bytes_per_query(cfg):
             "total": idx + csa + hca + app + qio}
 
 
+# ----------------------------------------------------------------- ranks
+def rank_config(cfg, rank):
+    """Each rank decodes its own batch of sequences: same shapes, its own seed."""
+    from compressed_sparse_kv_02_b200 import synth
+    return cfg if rank == 0 else synth.Config(**{**cfg.__dict__, "seed": cfg.seed + 17 * rank})
+
+
+def max_over_ranks(x, device, world):
+    """The slowest rank's figure (a MAX all-reduce; every rank gets it)."""
+    if world == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, ms_max):
+    """Units of all ranks per second of the slowest rank."""
+    return units_per_rank * world / (ms_max * 1e-3)
+
+
 # ----------------------------------------------------------------- our arm
 def run_ours(args, rank, world):
     import compressed_sparse_kv_02_b200 as ck
@@ -147,8 +168,7 @@ def run_ours(args, rank, world):
     cfg = synth.CONFIGS[args.config]
     if args.batch:
         cfg = synth.Config(**{**cfg.__dict__, "batch": args.batch})
-    if rank:
-        cfg = synth.Config(**{**cfg.__dict__, "seed": cfg.seed + 17 * rank})
+    cfg = rank_config(cfg, rank)
     model = decode.DecodeModel(cfg, device="cuda")
     model.fill_synthetic()
     model.prepare()
@@ -236,12 +256,8 @@ def run_ours(args, rank, world):
     st = model.check_status()
     if st != ck.OK:
         raise RuntimeError("device status after the timed region: %s" % ck.status_string(st))
-    ms_step = ms_total / steps_timed
-    if world > 1:
-        t = torch.tensor([ms_step], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_step = float(t.item())
-    value = nq * world / (ms_step * 1e-3)
+    ms_step = max_over_ranks(ms_total / steps_timed, dev, world)
+    value = whole_job_rate(nq, world, ms_step)
 
     # end to end: host (pinned) inputs copied in, outputs copied out, every step
     host_in = model.step_inputs_like(device="cpu", pin=True)
@@ -273,11 +289,7 @@ def run_ours(args, rank, world):
             e2e_step()
         e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev, world)
 
     bq = bytes_per_query(cfg)
     hbm, src = peaks()
@@ -332,7 +344,7 @@ def run_ours(args, rank, world):
             "bound": "hbm", "achieved": round(path_gbs, 1), "peak": hbm, "unit": "GB/s",
             "frac": round(path_gbs / hbm, 4), "bytes_per_query": bq,
         },
-        "e2e": {"value": round(nq * world / (e2e_ms * 1e-3), 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": round(whole_job_rate(nq, world, e2e_ms), 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": kernels_per_step * steps_timed,
     }

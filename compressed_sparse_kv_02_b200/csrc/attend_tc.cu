@@ -6,61 +6,78 @@
 // by every head).
 //
 // With 128 heads on one 576-wide latent every key carries 2 x 128 x 1088
-// flops: the product is a real dense contraction, with the heads as M = 128.
-// Work item = (query, 128-head group, key split, half of d_v). Per item:
-//   - Q [128 heads x 576] sits in shared memory as nine 128-byte-swizzled
-//     K-major blocks of 64 channels (one TMA load per block); 32-key tiles of
-//     K stream through two swizzled buffers: by TMA when the tile's rows are
-//     contiguous (window rows of the ring, HCA entries of one page), by
-//     cp.async through a row table otherwise (the CSA selection);
-//   - S = Q K^T (M 128, N 32, K 576) lands in tensor memory as three partial
-//     sums over 192 channels each, so consecutive MMAs never wait on one
-//     accumulator;
-//   - four warps take one head row each from S (tcgen05.ld), run the online
-//     softmax in fp32 and write P (bf16) back to tensor memory;
-//   - O[:, half] += P V (M 128, N 256, K 32) with P as the tensor-memory A
-//     operand and V read MN-major from the same K tile (V = the first d_v
-//     channels of each key);
+// flops against 1152 bytes: the product sits at the B200's ridge point, so the
+// kernel must stream keys at HBM speed and keep the tensor core busy at once.
+// Work item = (query, 128-head group, key split), run by a cluster of two CTAs
+// that split the key channels:
+//   rank 0 holds Q channels 0..319 and loads key channels 0..319;
+//   rank 1 holds Q channels 320..575 and loads key channels 256..575;
+// each computes a partial S = Q K^T over its channels (heads as M = 128, 32
+// keys as N) in tensor memory, sends it to the other CTA through distributed
+// shared memory and adds the one it receives, so both hold the full S and run
+// the same online softmax (fp32; identical results, since a + b == b + a).
+// Each then accumulates O for its half of d_v: O[:, 256 r .. 256 r + 255] +=
+// P V, with P (bf16) as the tensor-memory A operand and V read MN-major from
+// the first four channel blocks of its key tile (V = the first d_v channels of
+// every key). No tensor work is duplicated. Each CTA keeps its last three Q
+// blocks in tensor memory (an MMA's A operand may come from there) and the
+// rest in shared memory, which leaves room for five key-tile stages and the
+// exchange buffers, so the loads run well ahead of the math.
+//   - key tiles arrive by TMA when their rows are contiguous (window rows of
+//     the ring, HCA entries of one page), by cp.async through a row table
+//     otherwise (the CSA selection);
+//   - each thread of the softmax warpgroup owns one head row; it sends tile
+//     t + 1's partial (asynchronous stores counted on the receiver's
+//     mbarrier) before it waits for tile t's, hiding the exchange;
 //   - O is rescaled only when a row's running max rises by more than 2^8 (the
 //     probabilities stay below 256 in bf16), so most tiles skip it.
 // Window keys are taken in ring-slot order (the softmax does not depend on the
-// order of its keys), which makes a window tile 32 consecutive ring rows.
-// The two d_v halves of a (query, split) run in two CTAs that both compute S
-// (the accumulator for all 512 output channels would fill the whole tensor
-// memory). Each item writes its normalised partial output and log-sum-exp;
+// order of its keys), which makes a window tile 32 consecutive ring rows. Each
+// item writes its normalised partial output and log-sum-exp;
 // attend_merge_kernel combines the splits.
+#include <cooperative_groups.h>
+
 #include "cskv_device.cuh"
 #include "cskv_internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace cskv {
 namespace {
 
 constexpr int kDqk = 576, kDv = 512, kM = 128, kNk = 32;
-constexpr int kKb = kDqk / 64;                // 64-channel (128-byte) blocks per row
-constexpr int kQBytes = kKb * kM * 128;       // 147456
-constexpr int kKBytes = kKb * kNk * 128;      // 36864 per key tile
-constexpr int kThreads = 256;                 // warps 0-3 softmax, warp 4 MMA, warps 5-7 loads
+constexpr int kNb = 5;                         // 64-channel blocks of a key row loaded by each CTA
+constexpr int kStageBytes = kNb * kNk * 128;   // 20480 per key-tile stage
+// Q blocks of a CTA: the first kQSmem (rank 0: 2, rank 1: 1) in shared memory,
+// the last three in tensor memory (the A operand of an MMA may come from either)
+constexpr int kQTmem = 3;
+constexpr int kQBytes = 2 * kM * 128;          // 32768
+constexpr int kNS = 5;                         // key-tile stages
+constexpr int kRecvBytes = kM * kNk * 4;       // one partial S tile from the other CTA
+constexpr int kThreads = 256;                  // warps 0-3 softmax, warp 4 MMA, warps 5-7 loads
 constexpr int kMmaThread = 128;
 constexpr int kLoadThread0 = 160;
 constexpr int kLoaders = kThreads - kLoadThread0;  // 96
-constexpr int kRowCap = 1024;                 // keys per work item (row table in shared memory)
-constexpr int kSAcc = 3;                      // partial sums of S (K = 3 x 192)
+constexpr int kRowCap = 1024;                  // keys per work item (row table in shared memory)
 constexpr uint32_t kTmemCols = 512;
-// O 256 | S 2 buffers x 3 partials x 32 | P 2 buffers x 16 (bf16 pairs)
-constexpr uint32_t kColO = 0, kColS = 256, kColP = 256 + 2 * kSAcc * kNk;
+// O 256 | S 3 buffers x 32 | P 3 buffers x 16 (bf16 pairs) | Q 3 blocks x 32 (bf16 pairs)
+constexpr int kNSP = 3;  // S and P buffers
+constexpr uint32_t kColO = 0, kColS = 256, kColP = kColS + kNSP * 32, kColQ = kColP + kNSP * 16;
+static_assert(kColQ + kQTmem * 32 <= kTmemCols, "tensor memory budget");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleThreshold = 8.0f;     // log2 units
-constexpr int kPrefetchTiles = 6;             // L2 prefetch distance of gathered key rows
-static_assert(kColP + 32 <= kTmemCols, "tensor memory budget");
+constexpr float kRescaleThreshold = 8.0f;      // log2 units
+constexpr int kPrefetchTiles = 6;              // L2 prefetch distance of gathered key rows
 
 struct Smem {
   static constexpr int Q = 0;
-  static constexpr int K = kQBytes;                  // two tile buffers (also the epilogue staging)
-  static constexpr int BAR = K + 2 * kKBytes;        // mbarriers
-  static constexpr int MASK = BAR + 128;             // valid-key bits, one word per tile
-  static constexpr int ROWS = MASK + kRowCap / 8;    // source row of every key of the item
-  static constexpr int TMEM = ROWS + kRowCap * 8;    // allocated tensor-memory address
+  static constexpr int K = kQBytes;                     // kNS stages (also the epilogue staging)
+  static constexpr int RECV = K + kNS * kStageBytes;    // two slots of the other CTA's partial S
+  static constexpr int SEND = RECV + 2 * kRecvBytes;    // two slots of this CTA's partial S on its way out
+  static constexpr int BAR = SEND + 2 * kRecvBytes;     // mbarriers
+  static constexpr int MASK = BAR + 256;                // valid-key bits, one word per tile
+  static constexpr int ROWS = MASK + kRowCap / 8;       // source row of every key of the item
+  static constexpr int TMEM = ROWS + kRowCap * 8;       // allocated tensor-memory address
   static constexpr int FLAGS = TMEM + 16;
   static constexpr int PREF = FLAGS + 16;
   static size_t bytes(int n_q) { return 1024 + PREF + sizeof(int) * (size_t)(n_q + 1); }
@@ -113,8 +130,8 @@ __device__ __forceinline__ const uint16_t* key_src(const AttendParams& p, int b,
   return static_cast<const uint16_t*>(p.kv_pool) + ((int64_t)page * p.page_size + j % p.page_size) * kDqk;
 }
 
-// byte offset of 16-byte chunk `ch` (0..71) of row `r` in a swizzled block set
-// whose 64-channel blocks are `block_bytes` apart
+// byte offset of 16-byte chunk `ch` of row `r` in a swizzled block set whose
+// 64-channel (128-byte) blocks are `block_bytes` apart
 __device__ __forceinline__ uint32_t swz(int r, int ch, int block_bytes) {
   return (ch >> 3) * block_bytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
 }
@@ -123,14 +140,48 @@ __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
 }
 
-// Pipeline (per CTA, tiles numbered gt across its items; buffer gt & 1):
-//   loaders  : wait kempty[buf] (P V of tile gt-2 done) -> TMA, or cp.async +
-//              proxy fence, into buf -> kfull[buf]
-//   MMA      : wait kfull -> S(gt) = Q K^T into S[buf] -> commit sfull[buf];
-//              then wait pfull of tile gt-1 -> O += P V -> commit kempty, obar
-//   softmax  : wait sfull[buf] -> S row -> P row into P[buf] (+ rare O rescale
-//              after obar of tile gt-1) -> arrive pfull[buf]
-// S(gt) is issued before P V (gt-1), so the tensor core overlaps the softmax.
+// ---------------------------------------------------------------- cluster helpers
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+  return r;
+}
+// shared::cluster address of `local` in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t peer_addr(const void* local, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(a) : "r"(smem_u32(local)), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ void st_peer_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;\n" ::"r"(addr), "r"(v) : "memory");
+}
+// arrive on an mbarrier of another CTA (after this thread's reads of the slot
+// it frees; the other CTA only writes into that slot again after seeing it)
+__device__ __forceinline__ void mbar_arrive_peer(uint32_t addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];\n" ::"r"(addr) : "memory");
+}
+// bulk copy (by the TMA engine) of `bytes` from this CTA's shared memory into
+// another CTA's, counted as transaction bytes on that CTA's mbarrier (dst and
+// mbar are shared::cluster addresses). The source may be rewritten once that
+// mbarrier's phase has completed.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                   dst),
+               "r"(smem_u32(src)), "r"(bytes), "r"(mbar)
+               : "memory");
+}
+// Pipeline (per CTA; tiles numbered gt across the items of the cluster, the
+// same in both CTAs; stage gt % kNS, S / P buffer gt % 3, exchange slot gt & 1):
+//   loaders  : wait kempty (P V of tile gt - kNS done) -> TMA, or cp.async +
+//              proxy fence, into the stage -> kfull
+//   MMA      : wait kfull -> partial S(gt) -> commit sfull; then wait pfull of
+//              tile gt - 2 -> O += P V -> commit kempty, obar
+//   softmax  : wait sfull(gt + 1) -> send its partial to the other CTA (async
+//              stores that count bytes on the receiver's rfull); wait rfull(gt)
+//              -> S(gt) = own + received -> free the slot (remote rempty) ->
+//              P(gt) (+ rare O rescale after P V of tile gt - 1) -> arrive pfull
+// S(gt) needs the softmax only up to tile gt - 3 and the softmax needs S only
+// one tile ahead, so neither waits on the other's latest step.
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ring,
                      const __grid_constant__ CUtensorMap tm_kv, AttendParams p) {
@@ -138,34 +189,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = sm + Smem::Q;
   uint8_t* sK = sm + Smem::K;
+  uint8_t* sRecv = sm + Smem::RECV;
+  uint8_t* sSend = sm + Smem::SEND;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Smem::BAR);
-  uint64_t* kfull = bars;       // [2] loaders -> MMA
-  uint64_t* kempty = bars + 2;  // [2] MMA -> loaders (commit)
-  uint64_t* sfull = bars + 4;   // [2] MMA -> softmax (commit)
-  uint64_t* pfull = bars + 6;   // [2] softmax -> MMA (128 arrivals)
-  uint64_t* obar = bars + 8;    //     MMA -> softmax (commit after each P V)
-  uint64_t* qbar = bars + 9;    //     Q landed (TMA)
-  uint64_t* dbar = bars + 10;   //     MMA -> epilogue (commit after the item's last P V)
+  uint64_t* kfull = bars;             // [kNS] loaders -> MMA
+  uint64_t* kempty = bars + kNS;      // [kNS] MMA -> loaders (commit)
+  uint64_t* sfull = bars + 2 * kNS;   // [3] MMA -> softmax (commit)
+  uint64_t* pfull = sfull + kNSP;     // [3] softmax -> MMA (128 arrivals)
+  uint64_t* obar = pfull + kNSP;      // [3] MMA -> softmax (commit after the P V of that P buffer)
+  uint64_t* rfull = obar + kNSP;      // [2] other CTA's partial S landed (one arrival + 16 KB of bytes)
+  uint64_t* rempty = rfull + 2;       // [2] other CTA has read what this one sent (4 remote arrivals)
+  uint64_t* qbar = rempty + 2;        //     Q landed (TMA)
+  uint64_t* dbar = qbar + 1;          //     MMA -> epilogue (commit after the item's last P V)
   uint32_t* sMask = reinterpret_cast<uint32_t*>(sm + Smem::MASK);
   const uint16_t** sRow = reinterpret_cast<const uint16_t**>(sm + Smem::ROWS);
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + Smem::TMEM);
-  int* sAbort = reinterpret_cast<int*>(sm + Smem::FLAGS);
-  volatile int* sLdOk = reinterpret_cast<int*>(sm + Smem::FLAGS) + 1;  // [2], loader wait results
+  volatile int* sAbort = reinterpret_cast<int*>(sm + Smem::FLAGS);
+  volatile int* sLdOk = reinterpret_cast<int*>(sm + Smem::FLAGS) + 1;  // [2] loader wait results, then [1] send flag
   int* sPref = reinterpret_cast<int*>(sm + Smem::PREF);
   __shared__ int s_wsum[32];
 
+  cg::cluster_group cluster = cg::this_cluster();
+  const uint32_t rank = cluster_rank(), peer = rank ^ 1u;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int groups = p.n_heads / kM;
   const int kps = p.keys_per_split;
+  const int kb_load0 = rank ? 4 : 0;  // first 64-channel block of the key rows this CTA loads
+  const int n_sblk = rank ? 4 : 5;    // blocks of its S partial (Q blocks 0.. of this CTA)
+  const int n_qs = n_sblk - kQTmem;   // of which in shared memory
+  const int qkb0 = rank ? 5 : 0;      // channel block of its Q block 0
+  const int s_blk0 = rank ? 1 : 0;    // first S block inside a stage (blocks 0..3 are V)
 
-  {  // items per query: splits x head groups x 2 halves of d_v
+  {  // items per query: splits x head groups
     int run = 0;
     for (int base = 0; base < p.n_q; base += kThreads) {
       const int b = base + tid;
       int v = 0;
       if (b < p.n_q) {
         const Keys k = keys_of(p, b);
-        v = static_cast<int>((k.n + kps - 1) / kps) * groups * 2;
+        v = static_cast<int>((k.n + kps - 1) / kps) * groups;
       }
       int tot;
       const int ex = block_exclusive_scan<kThreads>(v, s_wsum, tot);
@@ -175,14 +237,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) sPref[p.n_q] = run;
   }
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kNS; ++i) {
       mbar_init(&kfull[i], 1);
       mbar_init(&kempty[i], 1);
+    }
+    for (int i = 0; i < kNSP; ++i) {
       mbar_init(&sfull[i], 1);
       mbar_init(&pfull[i], kM);
+      mbar_init(&obar[i], 1);
     }
-    mbar_init(obar, 1);
-    mbar_init(qbar, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&rfull[i], 1);
+      mbar_init(&rempty[i], 4);
+    }
+    mbar_init(qbar, 1 + kM);  // the TMA's arrival and one per softmax thread (tensor-memory blocks)
     mbar_init(dbar, 1);
     fence_barrier_init();
     *sAbort = 0;
@@ -197,17 +265,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster.sync();  // barriers of both CTAs initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem = *sTmem;
   if (blockIdx.x == 0)
     for (int b = tid; b < p.n_q; b += kThreads)
       if (p.q_pos[b] < 0 || p.q_pos[b] > p.max_pos) report(p.status, CSKV_ERR_INVALID_ARG);
   const int total = sPref[p.n_q];
-  uint32_t g = 0;       // tiles processed by this CTA before the current item
-  uint32_t n_item = 0;  // items processed by this CTA before the current one (qbar phase)
+  const int n_clusters = gridDim.x / 2;
+  uint32_t g = 0;       // tiles processed by this cluster before the current item
+  uint32_t n_item = 0;  // items processed before the current one (qbar / dbar phase)
 
-  for (int item = blockIdx.x; item < total; item += gridDim.x, ++n_item) {
+  for (int item = blockIdx.x / 2; item < total; item += n_clusters, ++n_item) {
     int lo = 0, hi = p.n_q - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -215,9 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const int b = lo;
     const int r = item - sPref[b];
-    const int vh = r & 1;
-    const int grp = (r >> 1) % groups;
-    const int split = (r >> 1) / groups;
+    const int grp = r % groups;
+    const int split = r / groups;
     const Keys kk = keys_of(p, b);
     const int seq = p.q_seq[b];
     const bool seq_ok = seq >= 0 && seq < p.n_seqs_layer;
@@ -238,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int q = 0; q < 4; ++q) {
         const int i = i0 + q * kThreads + tid;
         if (i < nk) {
-          if (!src[q]) report(p.status, CSKV_ERR_OUT_OF_RANGE);
+          if (!src[q] && rank == 0) report(p.status, CSKV_ERR_OUT_OF_RANGE);
           sRow[i] = src[q];
         }
         const unsigned bits = __ballot_sync(kFull, src[q] != nullptr);
@@ -250,10 +318,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid >= kLoadThread0) {
       // ------------------------------------------------------------ loaders
       const int lt = tid - kLoadThread0;
-      if (lt == 0) {  // Q of this head group: nine 128-row TMA boxes
-        mbar_arrive_expect_tx(qbar, kQBytes);
+      if (lt == 0) {  // this CTA's shared-memory Q blocks of the head group: 128-row TMA boxes
+        mbar_arrive_expect_tx(qbar, n_qs * kM * 128);
         const int qrow = b * p.n_heads + grp * kM;
-        for (int kb = 0; kb < kKb; ++kb) tma_load_2d(sQ + kb * (kM * 128), &tm_q, kb * 64, qrow, qbar);
+        for (int j = 0; j < n_qs; ++j) tma_load_2d(sQ + j * (kM * 128), &tm_q, (qkb0 + j) * 64, qrow, qbar);
       }
       // TMA source of tile it: 0 = ring rows, 1 = pool rows, -1 = gathered (cp.async)
       auto tile_src = [&](int it, int& row0) -> int {
@@ -278,43 +346,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto prefetch_tile = [&](int it) {
         if (lt < kNk && it < ntiles) {
           const int i = it * kNk + lt;
-          if (i < nk && sRow[i]) prefetch_l2(sRow[i], kDqk * 2);
+          if (i < nk && sRow[i]) prefetch_l2(sRow[i] + kb_load0 * 64, kNb * 128);
         }
       };
-      for (int it = 0; it < kPrefetchTiles; ++it) prefetch_tile(it);
+      const bool gathered_item = p.is_csa || p.x_chunk;
+      if (gathered_item)
+        for (int it = 0; it < kPrefetchTiles; ++it) prefetch_tile(it);
       for (int it = 0; it < ntiles; ++it) {
         const uint32_t gt = g + it;
-        const int buf = gt & 1;
-        prefetch_tile(it + kPrefetchTiles);
+        const int st = gt % kNS;
+        if (gathered_item) prefetch_tile(it + kPrefetchTiles);
         // one thread waits and the loaders agree on its result, so no loader can
         // leave the loop while another waits at a named barrier below
-        if (lt == 0) sLdOk[it & 1] = gt < 2 || mbar_wait(&kempty[buf], ((gt >> 1) - 1) & 1u, p.status);
+        if (lt == 0)
+          sLdOk[it & 1] = !*sAbort && (gt < (uint32_t)kNS || mbar_wait(&kempty[st], ((gt / kNS) - 1) & 1u, p.status));
         named_sync(3, kLoaders);
         if (!sLdOk[it & 1]) { *sAbort = 1; break; }
-        uint8_t* dst = sK + buf * kKBytes;
+        uint8_t* dst = sK + st * kStageBytes;
         int row0 = 0;
         const int mode = tile_src(it, row0);
         if (mode >= 0) {
           if (lt == 0) {
-            mbar_arrive_expect_tx(&kfull[buf], kKBytes);
+            mbar_arrive_expect_tx(&kfull[st], kStageBytes);
             const CUtensorMap* map = mode == 0 ? &tm_ring : &tm_kv;
-            for (int kb = 0; kb < kKb; ++kb) tma_load_2d(dst + kb * (kNk * 128), map, kb * 64, row0, &kfull[buf]);
+            for (int j = 0; j < kNb; ++j)
+              tma_load_2d(dst + j * (kNk * 128), map, (kb_load0 + j) * 64, row0, &kfull[st]);
           }
         } else {
           // consecutive threads take consecutive 16-byte chunks of a row (coalesced)
 #pragma unroll 4
-          for (int id = lt; id < kNk * 72; id += kLoaders) {
-            const int kr = id / 72, c = id % 72;
+          for (int id = lt; id < kNk * kNb * 8; id += kLoaders) {
+            const int kr = id / (kNb * 8), c = id % (kNb * 8);
             const int i = it * kNk + kr;
             const uint16_t* src = i < nk ? sRow[i] : nullptr;
-            cp_async16(dst + swz(kr, c, kNk * 128), src ? static_cast<const void*>(src + c * 8) : p.q,
-                       src ? 16 : 0);
+            cp_async16(dst + swz(kr, c, kNk * 128),
+                       src ? static_cast<const void*>(src + kb_load0 * 64 + c * 8) : p.q, src ? 16 : 0);
           }
           cp_async_commit();
           cp_async_wait<0>();
           fence_proxy_async_smem();
           named_sync(3, kLoaders);
-          if (lt == 0) mbar_arrive(&kfull[buf]);
+          if (lt == 0) mbar_arrive(&kfull[st]);
         }
       }
     } else if (tid == kMmaThread) {
@@ -322,44 +394,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_s = umma_idesc_bf16(kM, kNk, false);
       const uint32_t idesc_pv = umma_idesc_bf16(kM, 256, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK);
+      // descriptors differ only in the start address (low 14 bits, in 16-byte units)
+      const uint64_t dq0 = umma_desc_sw128(sQa, 16, 1024);
+      const uint64_t dk0 = umma_desc_sw128(sKa + s_blk0 * (kNk * 128), 16, 1024);
+      const uint64_t dv0 = umma_desc_sw128(sKa, kNk * 128, 1024);
       bool ok = mbar_wait(qbar, n_item & 1u, p.status);
-      for (int it = 0; it <= ntiles && ok; ++it) {
+      for (int it = 0; it <= ntiles + 1 && ok && !*sAbort; ++it) {
         if (it < ntiles) {
           const uint32_t gt = g + it;
-          const int buf = gt & 1;
-          if (!(ok = mbar_wait(&kfull[buf], (gt >> 1) & 1u, p.status))) break;
+          const int st = gt % kNS, buf = gt % kNSP;
+          if (!(ok = mbar_wait(&kfull[st], (gt / kNS) & 1u, p.status))) break;
           tc_fence_after();
-          const uint32_t kb_base = sKa + buf * kKBytes;
-          const uint32_t d = tmem + kColS + buf * (kSAcc * kNk);
-          // 36 MMAs (9 blocks x 4 k-steps), round-robin over three accumulators
+          const uint64_t dk = dk0 + ((st * kStageBytes) >> 4);
+          const uint32_t d = tmem + kColS + buf * kNk;
+          // 16 or 20 MMAs (issue-bound at N = 32, so one accumulator costs nothing)
 #pragma unroll 1
-          for (int kb3 = 0; kb3 < kKb / kSAcc; ++kb3) {
+          for (int j = 0; j < n_sblk; ++j) {
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-#pragma unroll
-              for (int a = 0; a < kSAcc; ++a) {
-                const int kb = a * (kKb / kSAcc) + kb3;
-                const uint64_t da = umma_desc_sw128(sQa + kb * (kM * 128) + ks * 32, 16, 1024);
-                const uint64_t db = umma_desc_sw128(kb_base + kb * (kNk * 128) + ks * 32, 16, 1024);
-                umma_ss(d + a * kNk, da, db, idesc_s, (kb3 | ks) != 0);
-              }
+              const uint64_t db = dk + ((j * (kNk * 128) + ks * 32) >> 4);
+              const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
+              if (j < n_qs)
+                umma_ss(d, dq0 + ((j * (kM * 128) + ks * 32) >> 4), db, idesc_s, acc);
+              else
+                umma_ts(d, tmem + kColQ + (j - n_qs) * 32 + ks * 8, db, idesc_s, acc);
             }
           }
           umma_commit(&sfull[buf]);
         }
-        if (it >= 1) {
-          const uint32_t gp = g + it - 1;
-          const int pb = gp & 1;
-          if (!(ok = mbar_wait(&pfull[pb], (gp >> 1) & 1u, p.status))) break;
+        if (it >= 2) {
+          const uint32_t gp = g + it - 2;
+          const int pb = gp % kNSP, sp = gp % kNS;
+          if (!(ok = mbar_wait(&pfull[pb], (gp / kNSP) & 1u, p.status))) break;
           tc_fence_after();
-          const uint32_t v_base = sKa + pb * kKBytes + vh * 4 * (kNk * 128);
+          const uint64_t dv = dv0 + ((sp * kStageBytes) >> 4);  // blocks 0..3 of the stage: this CTA's V
 #pragma unroll
-          for (int k2 = 0; k2 < 2; ++k2) {
-            const uint64_t db = umma_desc_sw128(v_base + k2 * 16 * 128, kNk * 128, 1024);
-            umma_ts(tmem + kColO, tmem + kColP + pb * 16 + k2 * 8, db, idesc_pv, (it > 1 || k2 > 0) ? 1u : 0u);
-          }
-          umma_commit(&kempty[pb]);
-          umma_commit(obar);
+          for (int k2 = 0; k2 < 2; ++k2)
+            umma_ts(tmem + kColO, tmem + kColP + pb * 16 + k2 * 8, dv + ((k2 * 16 * 128) >> 4), idesc_pv,
+                    (it > 2 || k2 > 0) ? 1u : 0u);
+          umma_commit(&kempty[sp]);
+          umma_commit(&obar[pb]);
         }
       }
       umma_commit(dbar);  // one completion per item, also after an abort
@@ -368,28 +442,94 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------------ softmax (one head row per thread)
       const float sl2 = p.sm_scale * kLog2e;
       const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+      const uint32_t recv_peer = peer_addr(sRecv, peer);
+      const uint32_t rfull_peer = peer_addr(rfull, peer);
+      const uint32_t rempty_peer = peer_addr(rempty, peer);
+      const int rr = tid;  // head row
       float m_used = -INFINITY, l_run = 0.f;
+      // Loop control stays uniform over the 128 threads (they meet at named
+      // barriers inside produce): it changes only through the flag read after
+      // produce's second barrier. A failed wait elsewhere raises the abort flag
+      // and lets the iteration finish on whatever data is there.
       bool ok = true;
+      float part[32];
+      volatile int* sSendOk = sLdOk + 2;  // [1] published by thread 0 inside produce
+      // own partial of tile gt into part[], and one bulk copy of it into the other CTA's slot gt & 1
+      auto produce = [&](uint32_t gt) -> bool {
+        const int buf = gt % kNSP, slot = gt & 1;
+        if (!__all_sync(kFull, mbar_wait(&sfull[buf], (gt / kNSP) & 1u, p.status))) *sAbort = 1;
+        tc_fence_after();
+        uint32_t s0[32];
+        tmem_ld32(tmem + lane_base + kColS + buf * kNk, s0);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) part[j] = __uint_as_float(s0[j]);
+        // slot gt & 1 of the send buffers here and of the receive slots there held
+        // tile gt - 2: both are free once the other CTA has read that tile
+        if (tid == 0) *sSendOk = !*sAbort && (gt < 2 || mbar_wait(&rempty[slot], ((gt >> 1) - 1) & 1u, p.status));
+        named_sync(1, kM);
+        const bool sent = *sSendOk != 0;
+        uint8_t* sbuf = sSend + slot * kRecvBytes;
+        if (sent) {
+          uint8_t* row = sbuf + rr * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(row + ((c ^ (rr & 7)) << 4)) =
+                make_uint4(__float_as_uint(part[4 * c]), __float_as_uint(part[4 * c + 1]),
+                           __float_as_uint(part[4 * c + 2]), __float_as_uint(part[4 * c + 3]));
+          fence_proxy_async_smem();
+        }
+        named_sync(1, kM);
+        if (sent && tid == 0) bulk_copy_to_peer(recv_peer + slot * kRecvBytes, sbuf, kRecvBytes, rfull_peer + slot * 8);
+        return sent;
+      };
+      {  // this thread's head row of the tensor-memory Q blocks (bf16 pairs, low half first)
+        const uint16_t* qg = p.q + ((int64_t)b * p.n_heads + grp * kM + rr) * kDqk + (qkb0 + n_qs) * 64;
+#pragma unroll 1
+        for (int t = 0; t < kQTmem; ++t) {
+          uint32_t qv[32];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v = ldg16(qg + t * 64 + c * 8);
+            qv[4 * c] = v.x;
+            qv[4 * c + 1] = v.y;
+            qv[4 * c + 2] = v.z;
+            qv[4 * c + 3] = v.w;
+          }
+          tmem_st32(tmem + lane_base + kColQ + t * 32, qv);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(qbar);
+      }
+      if (ntiles > 0) ok = produce(g);
       for (int it = 0; it < ntiles && ok; ++it) {
         const uint32_t gt = g + it;
-        const int buf = gt & 1;
-        // warp-uniform results keep the warp-wide votes below well defined
-        ok = __all_sync(kFull, mbar_wait(&sfull[buf], (gt >> 1) & 1u, p.status));
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t s0[32], s1[32], s2[32];
-        const uint32_t sbase = tmem + lane_base + kColS + buf * (kSAcc * kNk);
-        tmem_ld32(sbase, s0);
-        tmem_ld32(sbase + kNk, s1);
-        tmem_ld32(sbase + 2 * kNk, s2);
-        tmem_ld_wait();
+        const int buf = gt % kNSP, slot = gt & 1;
+        float cur[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) cur[j] = part[j];
+        if (it + 1 < ntiles && !(ok = produce(gt + 1))) break;
+        // the other CTA's partial of tile gt: one arrival (here) and 16 KB of its bulk copy
+        if (tid == 0) mbar_arrive_expect_tx(&rfull[slot], kRecvBytes);
+        if (!__all_sync(kFull, mbar_wait(&rfull[slot], (gt >> 1) & 1u, p.status))) *sAbort = 1;
+        const uint8_t* src = sRecv + slot * kRecvBytes + rr * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v = lds16(src + ((c ^ (rr & 7)) << 4));
+          cur[4 * c] += __uint_as_float(v.x);
+          cur[4 * c + 1] += __uint_as_float(v.y);
+          cur[4 * c + 2] += __uint_as_float(v.z);
+          cur[4 * c + 3] += __uint_as_float(v.w);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_peer(rempty_peer + slot * 8);
         const uint32_t valid = sMask[it];
         float v[32];
         float mt = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float sv = __uint_as_float(s0[j]) + __uint_as_float(s1[j]) + __uint_as_float(s2[j]);
-          v[j] = ((valid >> j) & 1u) ? sv * sl2 : -INFINITY;  // keys past nk have no row
+          v[j] = ((valid >> j) & 1u) ? cur[j] * sl2 : -INFINITY;  // keys past nk have no row
           mt = fmaxf(mt, v[j]);
         }
         float corr = 1.f;
@@ -408,10 +548,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           l_run += p0 + p1;
           pp[j] = pack_bf16(p0, p1);
         }
+        // P buffer gt % 3 was read by the P V of tile gt - 3
+        if (gt >= (uint32_t)kNSP && !__all_sync(kFull, mbar_wait(&obar[buf], ((gt / kNSP) - 1) & 1u, p.status)))
+          *sAbort = 1;
         if (__any_sync(kFull, rescale)) {
-          // O is being accumulated by P V of tile gt-1: rescale after it lands
-          // completions of obar so far: gt-1 or gt (P V of tile gt needs this warp's arrival)
-          ok = __all_sync(kFull, mbar_wait(obar, (gt - 1) & 1u, p.status));
+          // O takes the rescale once the P V of tile gt - 1 (and so every earlier one) has landed
+          const uint32_t gq = gt - 1;
+          if (!__all_sync(kFull, mbar_wait(&obar[gq % kNSP], (gq / kNSP) & 1u, p.status))) *sAbort = 1;
           tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < 256; c += 32) {
@@ -435,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int head0 = grp * kM;
       const int64_t prow0 = ((int64_t)b * p.max_splits + split) * p.n_heads + head0;
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      // staged through the (now idle) key buffers: each thread parks 32 values of its
+      // staged through the (now idle) key stages: each thread parks 32 values of its
       // row, then each warp stores 32 whole rows of 128 bytes
       float* stage = reinterpret_cast<float*>(sK);  // [128 rows][33]
 #pragma unroll 1
@@ -448,25 +591,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 32; ++j) stage[tid * 33 + j] = ok ? __uint_as_float(orow[j]) * inv : 0.f;
         named_sync(2, kM);
-        for (int rr = 0; rr < 32; ++rr) {
-          const int row = warp * 32 + rr;
-          p.part_o[(prow0 + row) * kDv + vh * 256 + c + lane] = stage[row * 33 + lane];
+        for (int q = 0; q < 32; ++q) {
+          const int row = warp * 32 + q;
+          p.part_o[(prow0 + row) * kDv + rank * 256 + c + lane] = stage[row * 33 + lane];
         }
         named_sync(2, kM);
       }
-      if (vh == 0) p.part_lse[prow0 + tid] = l_run > 0.f ? (m_used + log2f(l_run)) * kLn2 : -INFINITY;
+      if (rank == 0) p.part_lse[prow0 + tid] = l_run > 0.f ? (m_used + log2f(l_run)) * kLn2 : -INFINITY;
     }
     g += ntiles;
     tc_fence_before();
     __syncthreads();  // shared and tensor memory are reused by the next item
     tc_fence_after();
-    if (*sAbort) break;
+    if (*sAbort) {
+      if (tid == 0) st_peer_u32(peer_addr(const_cast<int*>(sAbort), peer), 1u);  // stop the other CTA too
+      break;
+    }
   }
   // after an abort, give tensor-core work in flight a bounded chance to land before freeing
   if (*sAbort && tid == kMmaThread) mbar_wait(dbar, n_item & 1u, nullptr);
   cp_async_wait<0>();
   tc_fence_before();
-  __syncthreads();
+  cluster.sync();  // the other CTA may still write into this one's shared memory until here
   tc_fence_after();
   if (warp == 4) tmem_dealloc(tmem, kTmemCols);
 }
@@ -490,11 +636,11 @@ bool attend_tc_supported(int d_qk, int d_v, int n_heads, int kv_dtype, int n_q) 
          Smem::bytes(n_q) <= 232448;  // the per-query prefix table shares shared memory with the tiles
 }
 
-// keys per split: queries x head groups x splits x 2 halves ~ one CTA per SM
+// keys per split: queries x head groups x splits ~ one CTA pair per two SMs
 void attend_tc_plan(AttendParams& p, int n_sm) {
   const int64_t groups = p.n_heads / kM;
   const int64_t n_max = (int64_t)p.n_win + (p.is_csa ? p.k : visible_entries(p.max_pos, p.m, p.n_win));
-  int64_t splits = n_sm / ((int64_t)p.n_q * groups * 2);
+  int64_t splits = (n_sm / 2) / ((int64_t)p.n_q * groups);
   if (splits < 1) splits = 1;
   int64_t kps = (n_max + splits - 1) / splits;
   kps = (kps + kNk - 1) / kNk * kNk;
@@ -517,11 +663,22 @@ cudaError_t launch_attend_tc(AttendParams& p, int n_sm, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int64_t upper = (int64_t)p.n_q * p.max_splits * (p.n_heads / kM) * 2;
-  int64_t grid = upper < n_sm ? upper : n_sm;
-  if (grid < 1) grid = 1;
-  attend_tc_kernel<<<static_cast<int>(grid), kThreads, smem, st>>>(tm_q, tm_ring, tm_kv, p);
-  e = cudaGetLastError();
+  const int64_t upper = (int64_t)p.n_q * p.max_splits * (p.n_heads / kM);
+  int64_t clusters = upper < n_sm / 2 ? upper : n_sm / 2;
+  if (clusters < 1) clusters = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, attend_tc_kernel, tm_q, tm_ring, tm_kv, p);
   if (e != cudaSuccess) return e;
   return launch_attend_merge(p, st);
 }

@@ -256,14 +256,14 @@ cskv_status csa_index_score_topk(const cskv_index_args* args, void* workspace, s
  *     fp32 values (16 MiB) inside libcskv.so. Every GPU that loads the
  *     library holds it until the process exits.
  *   - Limit: a call needs csa_index_ws_bytes() bytes of it; a larger request
- *     (n_q x the visible entries of max_pos, rounded up to 64) returns
- *     CSKV_ERR_WORKSPACE and launches nothing.
+ *     (n_q x (the visible entries of max_pos rounded up to 64, plus 2048
+ *     histogram counters)) returns CSKV_ERR_WORKSPACE and launches nothing.
  *   - Set-up: the first call on each device looks up the array's device
  *     address (cudaGetSymbolAddress) with that device current; make that
  *     first call before any stream capture.
  *   - Sharing: every call uses the same array and leaves its contents
  *     behind. Nothing in it needs clearing (each call writes every score it
- *     reads), but two calls that can run on the GPU at the same time -- on
+ *     reads and zeroes the counters it uses), but two calls that can run on the GPU at the same time -- on
  *     unordered streams, or from several host threads -- race on it and
  *     corrupt each other's results; order them on one stream or with events.
  *   - Arguments, outputs and errors are otherwise those of
