@@ -322,37 +322,122 @@ __global__ void __launch_bounds__(kBlockFoldThreads) fold_bulk_block_kernel(Fold
   }
 }
 
-constexpr int kAppendThreads = 256;
-constexpr int kSliceCh = 64;  // channels per CTA of the append kernel
+constexpr int kAppendWarps = 4;
+constexpr int kAppendThreads = 32 * kAppendWarps;
+constexpr int kSliceCh = 64;       // channels per CTA of the append kernel (whole row for FP8)
+constexpr int kAppendMaxD = 1024;  // channels of the row buffer
 
-// Grid (sequence, 64-channel slice). Each CTA copies its slice of the new rows
-// into the rings, then folds its slice of every block the new tokens complete
-// (old rows from the ring, new rows from the input; the slots written and the
-// slots read never coincide because n_new + m - 1 <= n_win). An FP8 stream
-// needs the whole row for its scale, so slice 0 folds all of it.
+// Online-softmax state (max of the base-2 logits, denominator, weighted sum)
+// of 16 channels, merged from another lane's state.
+__device__ __forceinline__ void merge16(float (&mx)[16], float (&den)[16], float (&acc)[16], int o) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const float m2 = __shfl_xor_sync(kFull, mx[e], o);
+    const float d2 = __shfl_xor_sync(kFull, den[e], o);
+    const float a2 = __shfl_xor_sync(kFull, acc[e], o);
+    const float M = fmaxf(mx[e], m2);
+    const float f1 = mx[e] == -INFINITY ? 0.f : exp2f(mx[e] - M);
+    const float f2 = m2 == -INFINITY ? 0.f : exp2f(m2 - M);
+    den[e] = den[e] * f1 + d2 * f2;
+    acc[e] = acc[e] * f1 + a2 * f2;
+    mx[e] = M;
+  }
+}
+
+// Store channels [c_lo, c_hi) of one folded entry from the row buffer `sv`
+// (fp32, indexed by channel) into pool row `row` in the stream's storage type:
+// bf16 (RNE), FP8 E4M3 with the row scale amax / 448 (the range is the whole
+// row), or FP4 E2M1 with one E4M3 scale per 16 channels.
+__device__ void store_row(const FoldStream& S, int64_t row, const float* sv, int c_lo, int c_hi, float* s_red) {
+  const int t = threadIdx.x;
+  if (S.out_dtype == CSKV_BF16) {
+    uint16_t* dst = static_cast<uint16_t*>(S.pool) + row * S.d;
+    for (int c = c_lo + 8 * t; c < c_hi; c += 8 * kAppendThreads) {
+      uint4 o;
+      o.x = pack_bf16(sv[c], sv[c + 1]);
+      o.y = pack_bf16(sv[c + 2], sv[c + 3]);
+      o.z = pack_bf16(sv[c + 4], sv[c + 5]);
+      o.w = pack_bf16(sv[c + 6], sv[c + 7]);
+      *reinterpret_cast<uint4*>(dst + c) = o;
+    }
+  } else if (S.out_dtype == CSKV_FP8_E4M3) {
+    float a = 0.f;
+    for (int c = c_lo + t; c < c_hi; c += kAppendThreads) a = fmaxf(a, fabsf(sv[c]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o));
+    if ((t & 31) == 0) s_red[t >> 5] = a;
+    __syncthreads();
+    float amax = 0.f;
+    for (int w = 0; w < kAppendWarps; ++w) amax = fmaxf(amax, s_red[w]);
+    const float sc = amax > 0.f ? amax / 448.0f : 1.0f;
+    uint8_t* dst = static_cast<uint8_t*>(S.pool) + row * S.d;
+    for (int c = c_lo + 8 * t; c < c_hi; c += 8 * kAppendThreads) {
+      uint32_t w[2] = {0u, 0u};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t code = __nv_cvt_float_to_fp8(sv[c + e] / sc, __NV_SATFINITE, __NV_E4M3);
+        w[e >> 2] |= code << (8 * (e & 3));
+      }
+      *reinterpret_cast<uint2*>(dst + c) = make_uint2(w[0], w[1]);
+    }
+    if (t == 0) S.scale_f32[row] = sc;
+    __syncthreads();  // s_red is reused
+  } else {  // FP4: 16-channel blocks, element 2i in the low nibble of byte i
+    uint8_t* dst = static_cast<uint8_t*>(S.pool) + row * (S.d / 2);
+    for (int c = c_lo + 16 * t; c < c_hi; c += 16 * kAppendThreads) {
+      float a = 0.f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) a = fmaxf(a, fabsf(sv[c + e]));
+      const __nv_fp8_storage_t sb = __nv_cvt_float_to_fp8(a / 6.0f, __NV_SATFINITE, __NV_E4M3);
+      const float sd = __half2float(__half(__nv_cvt_fp8_to_halfraw(sb, __NV_E4M3)));
+      uint32_t w[2] = {0u, 0u};
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        uint32_t code = 0u;
+        if (sd > 0.f) code = __nv_cvt_float_to_fp4(sv[c + e] / sd, __NV_E2M1, cudaRoundNearest) & 0xfu;
+        w[e >> 3] |= code << (4 * (e & 7));
+      }
+      *reinterpret_cast<uint2*>(dst + c / 2) = make_uint2(w[0], w[1]);
+      S.scale_e4m3[row * (S.d / 16) + c / 16] = sb;
+    }
+  }
+}
+
+// Grid (sequence, 64-channel slice, stream); an FP8 stream is handled whole by
+// slice 0 (its scale is the row's amax). Each CTA copies its channels of the
+// new rows into the rings, then folds its channels of every block the new
+// tokens complete (old rows from the ring, new rows from the input; the slots
+// written and the slots read never coincide because n_new + m - 1 <= n_win).
+// A warp folds 16 channels at a time: each lane runs the online softmax over
+// tokens lane, lane + 32, ... of the block, and the 32 partial states merge
+// by shuffles; the entry is stored from a shared-memory row buffer.
 __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
-  __shared__ float sm[3 * kAppendThreads * 8];
-  const int b = blockIdx.x, slice = blockIdx.y;
+  __shared__ float sv[kAppendMaxD];
+  __shared__ float s_red[kAppendWarps];
+  const int b = blockIdx.x, slice = blockIdx.y, si = blockIdx.z;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int seq = p.seq_ids[b];
   if (seq < 0 || seq >= p.n_seqs_layer) {
-    if (threadIdx.x == 0 && slice == 0) report(p.status, CSKV_ERR_OUT_OF_RANGE);
+    if (t == 0 && slice == 0 && si == 0) report(p.status, CSKV_ERR_OUT_OF_RANGE);
     return;
   }
+  const FoldStream& S = p.s[si];
+  const bool whole = S.out_dtype == CSKV_FP8_E4M3;
+  const int c_lo = whole ? 0 : slice * kSliceCh;
+  const int c_hi = whole ? S.d : min(S.d, c_lo + kSliceCh);
+  if (c_lo >= S.d || (whole && slice != 0)) return;
   const int64_t pos = p.pos[b];
-  for (int si = 0; si < p.n_streams; ++si) {
-    const FoldStream& S = p.s[si];
-    const int c_lo = slice * kSliceCh, c_hi = min(S.d, c_lo + kSliceCh);
-    if (c_lo >= S.d) continue;
-    const int cx = (c_hi - c_lo) / 8;  // 16-byte chunks of this slice per row
-    for (int t = threadIdx.x; t < p.n_new * cx; t += blockDim.x) {
-      const int i = t / cx, ch = t % cx;
+  {  // ring rows of the new tokens (this CTA's channels; gate logits: a per-token logit goes with c_lo == 0)
+    const int cx = (c_hi - c_lo) / 8;
+    for (int k = t; k < p.n_new * cx; k += kAppendThreads) {
+      const int i = k / cx, ch = k % cx;
       const int64_t slot = (pos + i) % p.n_win;
       *reinterpret_cast<uint4*>(S.ring_x_w + ((int64_t)seq * p.n_win + slot) * S.d + c_lo + ch * 8) =
           ldg16(S.x + ((int64_t)b * p.n_new + i) * S.d + c_lo + ch * 8);
     }
-    const int z_lo = S.gc == 1 ? (slice == 0 ? 0 : 1) : c_lo, z_hi = S.gc == 1 ? 1 : c_hi;
-    for (int t = threadIdx.x; t < p.n_new * (z_hi - z_lo); t += blockDim.x) {
-      const int i = t / (z_hi - z_lo), c = z_lo + t % (z_hi - z_lo);
+    const int z_lo = S.gc == 1 ? (c_lo == 0 ? 0 : 1) : c_lo, z_hi = S.gc == 1 ? 1 : c_hi;
+    for (int k = t; k < p.n_new * (z_hi - z_lo); k += kAppendThreads) {
+      const int i = k / (z_hi - z_lo), c = z_lo + k % (z_hi - z_lo);
       const int64_t slot = (pos + i) % p.n_win;
       S.ring_z_w[((int64_t)seq * p.n_win + slot) * S.gc + c] = S.z[((int64_t)b * p.n_new + i) * S.gc + c];
     }
@@ -361,28 +446,75 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
   // blocks completed by positions pos .. pos+n_new-1
   const int64_t j_first = pos / p.m;                 // first block ending at or after pos
   const int64_t j_last = (pos + p.n_new) / p.m - 1;  // last block ending before pos+n_new
-  const int64_t nb = j_last >= j_first ? j_last - j_first + 1 : 0;
-  for (int64_t it = 0; it < nb * p.n_streams; ++it) {
-    const int si = static_cast<int>(it / nb);
-    const int64_t j = j_first + it % nb;
-    const FoldStream& S = p.s[si];
-    const bool whole = S.out_dtype == CSKV_FP8_E4M3;
-    const int c_lo = whole ? 0 : slice * kSliceCh;
-    const int c_hi = whole ? S.d : min(S.d, c_lo + kSliceCh);
-    if (c_lo >= S.d || (whole && slice != 0)) continue;  // uniform across the block
-    const int64_t row = entry_row(p, seq, j);
-    auto rows = [&](int i, const uint16_t*& xr, const uint16_t*& zr) {
-      const int64_t q = j * p.m + i;
-      if (q >= pos) {
-        xr = S.x + ((int64_t)b * p.n_new + (q - pos)) * S.d;
-        zr = S.z + ((int64_t)b * p.n_new + (q - pos)) * S.gc;
-      } else {
-        const int64_t slot = q % p.n_win;
-        xr = S.ring_x + ((int64_t)seq * p.n_win + slot) * S.d;
-        zr = S.ring_z + ((int64_t)seq * p.n_win + slot) * S.gc;
+  for (int64_t j = j_first; j <= j_last; ++j) {
+    const int64_t row = entry_row(p, seq, j);  // uniform across the block
+    for (int c0 = c_lo + 16 * warp; c0 < c_hi; c0 += 16 * kAppendWarps) {
+      float mx[16], den[16], acc[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        mx[e] = -INFINITY;
+        den[e] = 0.f;
+        acc[e] = 0.f;
       }
-    };
-    if (row >= 0) fold_entry_block(S, p.m, row, rows, sm, c_lo, c_hi);  // row is uniform across the block
+      for (int i = lane; i < p.m; i += 32) {
+        const int64_t q = j * p.m + i;
+        const uint16_t* xr;
+        const uint16_t* zr;
+        if (q >= pos) {
+          xr = S.x + ((int64_t)b * p.n_new + (q - pos)) * S.d;
+          zr = S.z + ((int64_t)b * p.n_new + (q - pos)) * S.gc;
+        } else {
+          const int64_t slot = q % p.n_win;
+          xr = S.ring_x + ((int64_t)seq * p.n_win + slot) * S.d;
+          zr = S.ring_z + ((int64_t)seq * p.n_win + slot) * S.gc;
+        }
+        float xf[16], zl[16];
+        {
+          float h[8];
+          unpack8(ldg16(xr + c0), h);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xf[e] = h[e];
+          unpack8(ldg16(xr + c0 + 8), h);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xf[8 + e] = h[e];
+        }
+        if (S.gc == 1) {
+          const float zz = bf16_bits_to_f32(zr[0]);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) zl[e] = zz;
+        } else {
+          float h[8];
+          unpack8(ldg16(zr + c0), h);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) zl[e] = h[e];
+          unpack8(ldg16(zr + c0 + 8), h);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) zl[8 + e] = h[e];
+        }
+        if (S.bias) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) zl[e] += S.bias[(int64_t)i * S.d + c0 + e];
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float l2 = zl[e] * kLog2e;  // base-2 weights: 2^(l2 - max) = e^(z - max_z)
+          const float M = fmaxf(mx[e], l2);
+          const float corr = mx[e] == -INFINITY ? 0.f : exp2f(mx[e] - M);
+          const float pw = exp2f(l2 - M);
+          den[e] = den[e] * corr + pw;
+          acc[e] = acc[e] * corr + pw * xf[e];
+          mx[e] = M;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) merge16(mx, den, acc, o);
+      if (lane == 0)
+#pragma unroll
+        for (int e = 0; e < 16; ++e) sv[c0 + e] = acc[e] / den[e];
+    }
+    __syncthreads();
+    if (row >= 0) store_row(S, row, sv, c_lo, c_hi, s_red);
+    __syncthreads();  // the row buffer is reused by the next block
   }
 }
 
@@ -408,8 +540,12 @@ cudaError_t launch_fold_bulk(const FoldParams& p, cudaStream_t st) {
 cudaError_t launch_append(const FoldParams& p, cudaStream_t st) {
   if (p.n_seq == 0 || p.n_new == 0) return cudaSuccess;
   int dmax = 0;
-  for (int si = 0; si < p.n_streams; ++si) dmax = p.s[si].d > dmax ? p.s[si].d : dmax;
-  dim3 grid(static_cast<unsigned>(p.n_seq), static_cast<unsigned>((dmax + kSliceCh - 1) / kSliceCh));
+  for (int si = 0; si < p.n_streams; ++si) {
+    if (p.s[si].d > kAppendMaxD) return cudaErrorInvalidValue;
+    dmax = p.s[si].d > dmax ? p.s[si].d : dmax;
+  }
+  dim3 grid(static_cast<unsigned>(p.n_seq), static_cast<unsigned>((dmax + kSliceCh - 1) / kSliceCh),
+            static_cast<unsigned>(p.n_streams));
   append_kernel<<<grid, kAppendThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
