@@ -138,6 +138,18 @@ def bytes_per_query(cfg):
             "total": idx + csa + hca + app + qio}
 
 
+# DRAM bytes (read + write) of the indexer op per query, from one ncu capture of
+# the scan and select kernels on the Pro workload at batch 2, scaled by queries
+# (profiles/decode_pro_b2_kernels_full.md); None for other workloads or once
+# those kernels change.
+INDEX_OP_DRAM_BYTES_PER_QUERY = {"pro": (134.303232e6 + 4.073728e6 + 2.179328e6) / 2}
+
+
+def index_op_traffic(cfg, nq):
+    per_q = INDEX_OP_DRAM_BYTES_PER_QUERY.get(cfg.name)
+    return None if per_q is None else round(per_q * nq)
+
+
 # ----------------------------------------------------------------- ranks
 def rank_config(cfg, rank):
     """Each rank decodes its own batch of sequences: same shapes, its own seed."""
@@ -335,7 +347,7 @@ def run_ours(args, rank, world):
             "peak_source": src,
             "unit": "GB/s",
             "frac": round(achieved / hbm, 4),
-            "traffic": None,
+            "traffic": index_op_traffic(cfg, nq),
             "algorithmic_bytes_per_launch": bq["index"] * nq,
             "avg_launch_ms": round(idx_ms_avg, 5),
         },
