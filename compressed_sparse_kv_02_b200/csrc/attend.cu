@@ -386,6 +386,52 @@ __global__ void __launch_bounds__(256) attend_merge_kernel(AttendParams p) {
   }
 }
 
+// The same merge over head-minor partial outputs ([query x split][d_v / 4][heads][4],
+// written by attend_tc_kernel): a CTA takes 128 consecutive heads x 2 groups of 4
+// channels, so every partial-output load is a warp's 512 contiguous bytes.
+__global__ void __launch_bounds__(256) attend_merge_t_kernel(AttendParams p) {
+  const int b = blockIdx.x;
+  const QueryKeys qk = query_keys(p, b);
+  const int ns = static_cast<int>((qk.n + p.keys_per_split - 1) / p.keys_per_split);
+  const int h = blockIdx.z * 128 + (threadIdx.x & 127);
+  const int g4 = blockIdx.y * 2 + (threadIdx.x >> 7);  // group of 4 output channels
+  if (h >= p.n_heads || g4 >= p.d_v / 4) return;
+  const int64_t lbase = (int64_t)b * p.max_splits * p.n_heads + h;
+  float L = -INFINITY;
+  for (int s = 0; s < ns; ++s) L = fmaxf(L, p.part_lse[lbase + (int64_t)s * p.n_heads]);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float wsum = 0.f;
+  if (L != -INFINITY) {
+    const float4* po = reinterpret_cast<const float4*>(p.part_o);
+    for (int s0 = 0; s0 < ns; s0 += 8) {
+      float wg[8];
+      float4 o[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int s = s0 + j;
+        wg[j] = 0.f;
+        o[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (s < ns) {
+          wg[j] = expf(p.part_lse[lbase + (int64_t)s * p.n_heads] - L);
+          o[j] = po[(((int64_t)b * p.max_splits + s) * (p.d_v / 4) + g4) * p.n_heads + h];
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        wsum += wg[j];
+        acc[0] += wg[j] * o[j].x;
+        acc[1] += wg[j] * o[j].y;
+        acc[2] += wg[j] * o[j].z;
+        acc[3] += wg[j] * o[j].w;
+      }
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  const uint2 packed = make_uint2(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv));
+  *reinterpret_cast<uint2*>(p.out + ((int64_t)b * p.n_heads + h) * p.d_v + g4 * 4) = packed;
+  if (p.lse && g4 == 0) p.lse[(int64_t)b * p.n_heads + h] = wsum > 0.f ? L + logf(wsum) : -INFINITY;
+}
+
 struct Plan {
   int mt, vs;
 };
@@ -428,6 +474,12 @@ Plan plan_for(int d_qk, int d_v, int n_heads) {
 }  // namespace
 
 cudaError_t launch_attend_merge(AttendParams& p, cudaStream_t st) {
+  if (p.part_t) {
+    dim3 mg(static_cast<unsigned>(p.n_q), static_cast<unsigned>((p.d_v / 4 + 1) / 2),
+            static_cast<unsigned>((p.n_heads + 127) / 128));
+    attend_merge_t_kernel<<<mg, 256, 0, st>>>(p);
+    return cudaGetLastError();
+  }
   const int hb = 256 / (p.d_v / 4);
   dim3 mg(static_cast<unsigned>(p.n_q), static_cast<unsigned>((p.n_heads + hb - 1) / hb));
   attend_merge_kernel<<<mg, 256, 0, st>>>(p);

@@ -578,9 +578,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int head0 = grp * kM;
       const int64_t prow0 = ((int64_t)b * p.max_splits + split) * p.n_heads + head0;
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      // staged through the (now idle) key stages: each thread parks 32 values of its
-      // row, then each warp stores 32 whole rows of 128 bytes
-      float* stage = reinterpret_cast<float*>(sK);  // [128 rows][33]
+      // each thread writes its head row straight from tensor memory: part_o is
+      // head-minor ([query x split][d_v / 4][heads][4]), so a warp's 16-byte
+      // stores cover 32 consecutive heads, 512 contiguous bytes
+      float4* po = reinterpret_cast<float4*>(p.part_o) +
+                   (((int64_t)b * p.max_splits + split) * (kDv / 4) + rank * 64) * p.n_heads + head0 + rr;
 #pragma unroll 1
       for (int c = 0; c < 256; c += 32) {
         uint32_t orow[32];
@@ -589,13 +591,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait();
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) stage[tid * 33 + j] = ok ? __uint_as_float(orow[j]) * inv : 0.f;
-        named_sync(2, kM);
-        for (int q = 0; q < 32; ++q) {
-          const int row = warp * 32 + q;
-          p.part_o[(prow0 + row) * kDv + rank * 256 + c + lane] = stage[row * 33 + lane];
+        for (int k = 0; k < 8; ++k) {
+          const float4 v = ok ? make_float4(__uint_as_float(orow[4 * k]) * inv, __uint_as_float(orow[4 * k + 1]) * inv,
+                                            __uint_as_float(orow[4 * k + 2]) * inv, __uint_as_float(orow[4 * k + 3]) * inv)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+          po[(int64_t)(c / 4 + k) * p.n_heads] = v;
         }
-        named_sync(2, kM);
       }
       if (rank == 0) p.part_lse[prow0 + tid] = l_run > 0.f ? (m_used + log2f(l_run)) * kLn2 : -INFINITY;
     }
@@ -678,6 +679,7 @@ cudaError_t launch_attend_tc(AttendParams& p, int n_sm, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  p.part_t = 1;
   e = cudaLaunchKernelEx(&cfg, attend_tc_kernel, tm_q, tm_ring, tm_kv, p);
   if (e != cudaSuccess) return e;
   return launch_attend_merge(p, st);

@@ -107,7 +107,8 @@ struct AttendParams {
   int64_t chunk_pos0, chunk_len;
   int32_t* status;
   // workspace / plan
-  float* part_o;   // [n_q * max_splits * n_heads, d_v]
+  float* part_o;   // [n_q * max_splits * n_heads, d_v], or with part_t: [n_q * max_splits, d_v / 4, n_heads, 4]
+  int part_t;      // part_o in the head-minor layout (written by attend_tc_kernel)
   float* part_lse; // [n_q * max_splits * n_heads]
   int max_splits;
   int keys_per_split;

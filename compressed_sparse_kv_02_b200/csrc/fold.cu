@@ -446,6 +446,8 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
   // blocks completed by positions pos .. pos+n_new-1
   const int64_t j_first = pos / p.m;                 // first block ending at or after pos
   const int64_t j_last = (pos + p.n_new) / p.m - 1;  // last block ending before pos+n_new
+  int merge_span = 1;  // power of two >= min(m, 32)
+  while (merge_span < 32 && merge_span < p.m) merge_span <<= 1;
   for (int64_t j = j_first; j <= j_last; ++j) {
     const int64_t row = entry_row(p, seq, j);  // uniform across the block
     for (int c0 = c_lo + 16 * warp; c0 < c_hi; c0 += 16 * kAppendWarps) {
@@ -506,8 +508,8 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
           mx[e] = M;
         }
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) merge16(mx, den, acc, o);
+      // lanes >= m hold nothing: merge only across the lanes that ran tokens
+      for (int o = merge_span >> 1; o > 0; o >>= 1) merge16(mx, den, acc, o);
       if (lane == 0)
 #pragma unroll
         for (int e = 0; e < 16; ++e) sv[c0 + e] = acc[e] / den[e];
