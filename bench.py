@@ -117,25 +117,62 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- workload bytes
-def bytes_per_query(cfg):
-    """Algorithmic HBM bytes of one decode query through one CSA and one HCA layer (bf16 caches)."""
-    t = cfg.ctx - 1
-    nv = -(-(t + 1 - cfg.n_win) // cfg.m_csa)
-    nv_h = -(-(t + 1 - cfg.n_win) // cfg.m_hca)
-    row = cfg.d_qk * 2
-    idx = nv * cfg.d_idx * 2
-    csa = (cfg.n_win + cfg.k) * row
-    hca = (cfg.n_win + nv_h) * row
-    # appends: the new token's rows (read, written to the ring) and, when a block completes, its m rows of
-    # latent + gate logits read back for the fold and one entry written
-    app = 2 * (2 * row) + 2 * (2 * cfg.d_idx * 2)
-    if (t + 1) % cfg.m_csa == 0:
-        app += cfg.m_csa * (2 * row + 2 * cfg.d_idx * 2) + row + cfg.d_idx * 2
-    if (t + 1) % cfg.m_hca == 0:
-        app += cfg.m_hca * 2 * row + row
-    qio = 2 * cfg.heads * row + cfg.heads_idx * cfg.d_idx * 2 + 2 * cfg.heads * cfg.d_v * 2
-    return {"index": idx, "csa_attend": csa, "hca_attend": hca, "append": app, "io": qio,
-            "total": idx + csa + hca + app + qio}
+def _visible(t, m, n_win):
+    return max(0, -(-(t + 1 - n_win) // m))
+
+
+def bytes_per_query(cfg, ctx_lens=None, n_pairs=1):
+    """Algorithmic HBM bytes of one decode query through n_pairs (CSA, HCA) layer pairs, averaged over the
+    batch: the visible indexer keys, the attended keys (window rows are bf16, compressed entries in the
+    cache's storage type), the append traffic and the query / output I/O."""
+    lens = [cfg.ctx] * cfg.batch if ctx_lens is None else list(ctx_lens)
+    row = cfg.d_qk * 2  # bf16 raw / window row
+    ent = cfg.d_qk * 2 if cfg.kv_dtype == "bf16" else cfg.d_qk + 4  # stored entry (FP8: codes + fp32 scale)
+    key_i = cfg.d_idx * 2 if cfg.idx_dtype == "bf16" else cfg.d_idx // 2 + cfg.d_idx // 16
+    q_i = cfg.heads_idx * key_i
+    tot = {"index": 0.0, "csa_attend": 0.0, "hca_attend": 0.0, "append": 0.0, "io": 0.0}
+    for n in lens:
+        t = n - 1
+        nv, nv_h = _visible(t, cfg.m_csa, cfg.n_win), _visible(t, cfg.m_hca, cfg.n_win)
+        n_w = min(cfg.n_win, t + 1)
+        tot["index"] += nv * key_i
+        tot["csa_attend"] += n_w * row + min(cfg.k, nv) * ent
+        tot["hca_attend"] += n_w * row + nv_h * ent
+        # appends: the new token's rows (read, written to the ring) and, when a block completes, its m rows
+        # of latent + gate logits read back for the fold and one entry written
+        app = 2 * (2 * row) + 2 * (2 * cfg.d_idx * 2)
+        if (t + 1) % cfg.m_csa == 0:
+            app += cfg.m_csa * (2 * row + 2 * cfg.d_idx * 2) + ent + key_i
+        if (t + 1) % cfg.m_hca == 0:
+            app += cfg.m_hca * 2 * row + ent
+        tot["append"] += app
+        tot["io"] += 2 * cfg.heads * row + q_i + 2 * cfg.heads * cfg.d_v * 2
+    out = {k: int(round(v * n_pairs / len(lens))) for k, v in tot.items()}
+    out["total"] = sum(out.values())
+    return out
+
+
+def workload_model(cfg, device="cuda"):
+    """The decode model of a workload: uniform lengths and one layer pair, or (mixed) per-sequence
+    log-uniform lengths and two layer pairs (CSA, HCA, CSA, HCA)."""
+    from compressed_sparse_kv_02_b200 import decode, synth
+    if cfg.name == "mixed":
+        return decode.DecodeModel(cfg, device=device, ctx_lens=synth.mixed_lengths(cfg), n_pairs=2)
+    return decode.DecodeModel(cfg, device=device)
+
+
+def workload_text(cfg, nq, model):
+    if cfg.name == "pro":
+        return ("pro-like decode at 1M context: B=%d, t=%d, H=%d, d_qk=%d, d_v=%d, indexer %dx%d, CSA m=4 top-%d, "
+                "HCA m'=128, window 128, one CSA + one HCA layer"
+                % (nq, cfg.ctx - 1, cfg.heads, cfg.d_qk, cfg.d_v, cfg.heads_idx, cfg.d_idx, cfg.k))
+    if cfg.name == "mixed":
+        L = model.ctx_lens
+        return ("mixed paged decode: B=%d, lengths log-uniform %d..%d (mean %d), H=%d, d_qk=%d, d_v=%d, FP8 e4m3 "
+                "KV + fp32 scale per entry, FP4 e2m1 indexer %dx%d with e4m3 scales per 16, top-%d, layers CSA, "
+                "HCA, CSA, HCA" % (nq, min(L), max(L), sum(L) // len(L), cfg.heads, cfg.d_qk, cfg.d_v,
+                                   cfg.heads_idx, cfg.d_idx, cfg.k))
+    return "%s decode: B=%d, t=%d, H=%d, d=%d" % (cfg.name, nq, cfg.ctx - 1, cfg.heads, cfg.d_qk)
 
 
 # DRAM bytes (read + write) of the indexer op per query, from one ncu capture of
@@ -181,7 +218,7 @@ def run_ours(args, rank, world):
     if args.batch:
         cfg = synth.Config(**{**cfg.__dict__, "batch": args.batch})
     cfg = rank_config(cfg, rank)
-    model = decode.DecodeModel(cfg, device="cuda")
+    model = workload_model(cfg)
     model.fill_synthetic()
     model.prepare()
     stream = torch.cuda.Stream()
@@ -303,9 +340,10 @@ def run_ours(args, rank, world):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev, world)
 
-    bq = bytes_per_query(cfg)
+    bq = bytes_per_query(cfg, model.ctx_lens, model.n_pairs)
     hbm, src = peaks()
-    achieved = bq["index"] * nq / (idx_ms_avg * 1e-3) / 1e9
+    idx_bytes = bq["index"] * nq // model.n_pairs  # one indexer call (the first CSA layer's)
+    achieved = idx_bytes / (idx_ms_avg * 1e-3) / 1e9
     path_gbs = bq["total"] * nq / (ms_step * 1e-3) / 1e9
     kernels_per_step = 0
     for c in calls:
@@ -322,16 +360,14 @@ def run_ours(args, rank, world):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
-        "data": "synthetic (seeded Gaussian caches, 1% planted indexer keys)",
+        "dtype": "bf16" if cfg.kv_dtype == "bf16" else "fp8 KV / fp4 indexer",
+        "data": "synthetic (seeded Gaussian caches%s)" % (", 1% planted indexer keys" if cfg.planted_frac else
+                                                           ", random FP8 / FP4 codes" if cfg.kv_dtype != "bf16" else ""),
         "config": {
-            "workload": "pro-like decode at 1M context: B=%d, t=%d, H=%d, d_qk=%d, d_v=%d, indexer %dx%d, "
-                        "CSA m=4 top-%d, HCA m'=128, window 128, one CSA + one HCA layer"
-                        % (nq, cfg.ctx - 1, cfg.heads, cfg.d_qk, cfg.d_v, cfg.heads_idx, cfg.d_idx, cfg.k)
-            if cfg.name == "pro" else cfg.name,
+            "workload": workload_text(cfg, nq, model),
             "config_name": cfg.name,
             "batch_per_gpu": nq,
-            "context": cfg.ctx,
+            "context": max(model.ctx_lens),
             "parallelism": "replicas" if world == 1 else "dp%d (independent sequences per GPU)" % world,
             "l2": "inputs larger than L2 (%.0f MB read per step)" % (bq["total"] * nq / 1e6),
             "timing": "CUDA graph of %d steps replayed %d times (+%d); CUDA events on the launching stream"
@@ -348,7 +384,7 @@ def run_ours(args, rank, world):
             "unit": "GB/s",
             "frac": round(achieved / hbm, 4),
             "traffic": index_op_traffic(cfg, nq),
-            "algorithmic_bytes_per_launch": bq["index"] * nq,
+            "algorithmic_bytes_per_launch": idx_bytes,
             "avg_launch_ms": round(idx_ms_avg, 5),
         },
         "op_ms_untimed_breakdown": op_ms,
@@ -370,15 +406,17 @@ def _oracle_inputs(model, cfg, b):
     """Host copies (oracle storage views) of sequence b's caches and query, read from the device."""
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     import oracle
-    from gpu_helpers import layer_entries, ring_window, stored_bf16
-    t = cfg.ctx - 1
+    from gpu_helpers import layer_entries, ring_window, stored_bf16, stored_fp4
+    t = model.ctx_lens[b] - 1
     csa, hca = model.layers[0], model.layers[1]
     nv = oracle.visible_entries(t, cfg.m_csa, cfg.n_win)
     nv_h = oracle.visible_entries(t, cfg.m_hca, cfg.n_win)
     ent = layer_entries(csa, b, nv)
     inp = model.inputs[0]
+    qi = (stored_bf16(inp["q_idx"][b]) if cfg.idx_dtype == "bf16" else
+          stored_fp4(inp["q_idx"][b], inp["q_idx_scale"][b]))
     return dict(t=t, win=ring_window(csa, b, t), kv=ent["kv"], ki=ent["idx"], q=stored_bf16(inp["q_csa"][b]),
-                qi=stored_bf16(inp["q_idx"][b]), w=inp["w"][b].double().cpu().numpy(),
+                qi=qi, w=inp["w"][b].double().cpu().numpy(),
                 win_h=ring_window(hca, b, t), kv_h=layer_entries(hca, b, nv_h)["kv"],
                 q_h=stored_bf16(inp["q_hca"][b]))
 
@@ -398,15 +436,16 @@ def cpu_baseline(model, cfg, budget_s=20.0):
     oracle.set_threads(cores)
     done, t_cpu = 0, 0.0
     xs = [_oracle_inputs(model, cfg, b) for b in range(min(2, cfg.batch))]
+    # a query goes through n_pairs layer pairs; the sample runs the first pair and charges n_pairs of it
     while t_cpu < budget_s and done < 4 * cfg.batch:
         x = xs[done % len(xs)]
         t0 = time.perf_counter()
         _oracle_query(cfg, x)
-        t_cpu += time.perf_counter() - t0
+        t_cpu += (time.perf_counter() - t0) * model.n_pairs
         done += 1
     return {"value": round(done / t_cpu, 4), "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": "%d full decode queries (CSA indexer+top-k+attention and HCA attention, fp64) of the "
-                      "same workload, %.1f s of host time" % (done, t_cpu)}
+            "sample": "%d full decode queries (CSA indexer+top-k+attention and HCA attention, fp64, %d layer "
+                      "pair(s)) of the same workload, %.1f s of host time" % (done, model.n_pairs, t_cpu)}
 
 
 def run_reference(args, rank, world):
@@ -416,7 +455,7 @@ def run_reference(args, rank, world):
     import oracle
     oracle.build()
     cfg = synth.CONFIGS[args.config]
-    model = decode.DecodeModel(cfg, device="cuda")
+    model = workload_model(cfg)
     model.fill_synthetic()
     model.step()
     torch.cuda.synchronize()

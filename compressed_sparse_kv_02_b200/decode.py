@@ -123,10 +123,12 @@ class DecodeModel:
         return inp
 
     def fill_synthetic(self):
-        """Synthesise every layer's cache and ring in stored form, plus the step inputs (bf16 caches)."""
+        """Synthesise every layer's cache and ring in stored form, plus the step inputs."""
         cfg = self.cfg
+        if cfg.kv_dtype == "fp8" and cfg.idx_dtype == "fp4":
+            return self._fill_synthetic_quantised()
         if cfg.kv_dtype != "bf16" or cfg.idx_dtype != "bf16" or len(set(self.ctx_lens)) != 1:
-            raise NotImplementedError("fill_synthetic covers uniform-length bf16 workloads")
+            raise NotImplementedError("fill_synthetic covers uniform-length bf16 and FP8 / FP4 workloads")
         self.inputs = self.step_inputs_like()
         self.planted = {}
         for li in range(self.n_pairs):
@@ -150,6 +152,31 @@ class DecodeModel:
                     inp["w"].copy_(st["w"])
                     self.planted[li] = st["planted"]
                 del st
+        torch.cuda.synchronize()
+
+    def _fill_synthetic_quantised(self):
+        """FP8 KV and FP4 indexer caches, per-sequence lengths: one sequence at a time (bounded temporaries)."""
+        cfg = self.cfg
+        self.inputs = self.step_inputs_like()
+        self.planted = {}
+        for li in range(self.n_pairs):
+            csa, hca = self.layers[2 * li], self.layers[2 * li + 1]
+            for kind, L in (("csa", csa), ("hca", hca)):
+                for b, n_b in enumerate(self.ctx_lens):
+                    st = synth.stored_sequence_state(cfg, kind, b, n_b, self.device, stream_base=1000 * li)
+                    if st["kv_codes"].shape[0]:
+                        L.write_entries(b, 0, kv=st["kv_codes"], kv_scale=st["kv_scale"],
+                                        idx=st.get("idx_codes"), idx_scale=st.get("idx_scales"))
+                    L.ring_x[b].copy_(st["ring_x"])
+                    L.ring_z[b].copy_(st["ring_z"])
+                    if kind == "csa":
+                        L.ring_xi[b].copy_(st["ring_xi"])
+                        L.ring_zi[b].copy_(st["ring_zi"])
+                    del st
+            x = synth.stored_step_inputs(cfg, self.device, stream_base=1000 * li)
+            for k_, v in x.items():
+                self.inputs[li][k_].copy_(v.view(self.inputs[li][k_].shape))
+            self.planted[li] = [torch.empty(0, dtype=torch.int64) for _ in range(cfg.batch)]
         torch.cuda.synchronize()
 
     def prepare(self, inputs: Optional[dict] = None):

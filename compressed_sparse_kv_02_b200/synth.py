@@ -160,3 +160,74 @@ def decode_layer_state(cfg: Config, kind: str, device="cpu", stream_base: int = 
         out["ring_zi"][:, slots] = rzi
         out["new_xi"], out["new_zi"] = raw_stream(B, 1, cfg.d_idx, s, base + 11, device)
     return out
+
+
+def mixed_lengths(cfg: Config, lo: int = 4096, hi: int = None) -> list:
+    """Per-sequence stream lengths n_b = round(exp(U(ln lo, ln hi))) (hi defaults to cfg.ctx)."""
+    hi = cfg.ctx if hi is None else hi
+    u = torch.rand(cfg.batch, generator=generator(cfg.seed, 900, "cpu"), dtype=torch.float64)
+    return [int(round(math.exp(math.log(lo) + float(x) * (math.log(hi) - math.log(lo))))) for x in u]
+
+
+def e4m3_codes(shape, std: float, g: torch.Generator, device="cpu") -> torch.Tensor:
+    """E4M3 code bytes of ~N(0, std^2) values (torch's float8_e4m3fn rounding; never NaN)."""
+    v = (torch.randn(tuple(shape), generator=g, device=device) * std).clamp(-448.0, 448.0)
+    return v.to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def e2m1_codes(shape, g: torch.Generator, device="cpu") -> torch.Tensor:
+    """Random bytes of two E2M1 codes each (every 4-bit pattern is a finite value)."""
+    return torch.randint(0, 256, tuple(shape), generator=g, device=device, dtype=torch.int32).to(torch.uint8)
+
+
+def e4m3_block_scales(shape, g: torch.Generator, device="cpu") -> torch.Tensor:
+    """Positive E4M3 scale bytes between 0.5 and 2 (codes 0x30 .. 0x40)."""
+    return torch.randint(0x30, 0x41, tuple(shape), generator=g, device=device, dtype=torch.int32).to(torch.uint8)
+
+
+def stored_sequence_state(cfg: Config, kind: str, b: int, n_b: int, device="cpu", stream_base: int = 0) -> dict:
+    """Synthesised quantised state of one sequence of one decode layer at t = n_b - 1 (FP8 KV, FP4 indexer).
+
+    kv_codes [E, d_qk] E4M3 bytes with kv_scale [E] fp32 (stored value = code x scale, ~N(0,1)/sqrt(d_qk));
+    CSA also idx_codes [E, d_idx/2] E2M1 bytes with idx_scales [E, d_idx/16] E4M3 bytes;
+    ring_x / ring_z [n_win, d] bf16 rows of positions t-128 .. t-1 at slot p % n_win (CSA: ring_xi / ring_zi).
+    """
+    m = cfg.m_csa if kind == "csa" else cfg.m_hca
+    E = n_b // m
+    t = n_b - 1
+    s = cfg.seed
+    base = stream_base + (0 if kind == "csa" else 100) + 1000 * (b + 1)
+    out = {"kv_codes": e4m3_codes((E, cfg.d_qk), 1.0, generator(s, base + 1, device), device),
+           "kv_scale": torch.full((E,), 1.0 / math.sqrt(cfg.d_qk), dtype=torch.float32, device=device)}
+    slots = torch.tensor([(t - cfg.n_win + i) % cfg.n_win for i in range(cfg.n_win)], device=device)
+    rx, rz = raw_stream(1, cfg.n_win, cfg.d_qk, s, base + 3, device)
+    out["ring_x"] = torch.empty_like(rx[0])
+    out["ring_x"][slots] = rx[0]
+    out["ring_z"] = torch.empty_like(rz[0])
+    out["ring_z"][slots] = rz[0]
+    if kind == "csa":
+        out["idx_codes"] = e2m1_codes((E, cfg.d_idx // 2), generator(s, base + 2, device), device)
+        out["idx_scales"] = e4m3_block_scales((E, cfg.d_idx // 16), generator(s, base + 4, device), device)
+        rxi, rzi = raw_stream(1, cfg.n_win, cfg.d_idx, s, base + 9, device)
+        out["ring_xi"] = torch.empty_like(rxi[0])
+        out["ring_xi"][slots] = rxi[0]
+        out["ring_zi"] = torch.empty_like(rzi[0])
+        out["ring_zi"][slots] = rzi[0]
+    return out
+
+
+def stored_step_inputs(cfg: Config, device="cpu", stream_base: int = 0) -> dict:
+    """New rows and decode queries of one step for a quantised layer pair (FP4 indexer queries)."""
+    B, s = cfg.batch, cfg.seed
+    base = stream_base + 5000
+    out = {}
+    out["csa_x"], out["csa_z"] = raw_stream(B, 1, cfg.d_qk, s, base + 1, device)
+    out["csa_xi"], out["csa_zi"] = raw_stream(B, 1, cfg.d_idx, s, base + 3, device)
+    out["hca_x"], out["hca_z"] = raw_stream(B, 1, cfg.d_qk, s, base + 5, device)
+    out["q_csa"] = normal((B, cfg.heads, cfg.d_qk), 1.0, generator(s, base + 7, device), device)
+    out["q_hca"] = normal((B, cfg.heads, cfg.d_qk), 1.0, generator(s, base + 8, device), device)
+    out["q_idx"] = e2m1_codes((B, cfg.heads_idx, cfg.d_idx // 2), generator(s, base + 9, device), device)
+    out["q_idx_scale"] = e4m3_block_scales((B, cfg.heads_idx, cfg.d_idx // 16), generator(s, base + 10, device),
+                                           device)
+    out["w"] = uniform((B, cfg.heads_idx), 0.0, 1.0, generator(s, base + 11, device), device)
+    return out

@@ -8,6 +8,9 @@
 * flash (B = 32 x 128K) and pro (B = 8 x 1M, 1% planted keys): the full-size
   workloads in the launch configuration the benchmark times (DecodeModel),
   with the oracle run on sampled queries and heads.
+* mixed: the quantised, mixed-length workload (FP8 KV with a scale per entry,
+  FP4 indexer keys and queries, per-sequence lengths, layers CSA, HCA, CSA,
+  HCA) at a reduced batch and length, every query and both layer pairs.
 """
 import math
 
@@ -16,8 +19,8 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import (ATOL_BF16, REL_BF16, assert_close, assert_fold_close, check_topk, layer_entries,
-                         make_layer, ring_window, stored_bf16)
+from gpu_helpers import (ATOL_BF16, ATOL_LP, REL_BF16, REL_LP, assert_close, assert_fold_close, check_topk, layer_entries,
+                         make_layer, ring_window, stored_bf16, stored_fp4)
 
 pytestmark = pytest.mark.gpu
 
@@ -169,3 +172,40 @@ def test_flash_fullsize_sampled(ck, orc):
 
 def test_pro_fullsize_sampled(ck, orc):
     _fullsize(ck, orc, "pro", sample_b=[0, 7], sample_heads=[0, 1, 63, 64, 127])
+
+
+def test_mixed_fp8_fp4_two_pairs(ck, orc):
+    from compressed_sparse_kv_02_b200 import decode, synth
+    cfg = synth.Config("mixed_small", 4, 1 << 16, 128, 576, 512, 8, 128, 1024, seed=4, kv_dtype="fp8",
+                       idx_dtype="fp4")
+    lens = synth.mixed_lengths(cfg, lo=4096, hi=1 << 16)
+    lens[0] = 4096  # a sequence whose last token completes an HCA block (the append emits an entry)
+    model = decode.DecodeModel(cfg, ctx_lens=lens, n_pairs=2)
+    model.fill_synthetic()
+    model.step()
+    torch.cuda.synchronize()
+    assert model.check_status() == ck.OK
+    scale = 1.0 / math.sqrt(cfg.d_qk)
+    heads = np.array([0, 5, 64, 127])
+    for li in range(2):
+        csa, hca = model.layers[2 * li], model.layers[2 * li + 1]
+        out, inp = model.out[li], model.inputs[li]
+        for b, n_b in enumerate(lens):
+            t = n_b - 1
+            nv = orc.visible_entries(t, 4, 128)
+            nv_h = orc.visible_entries(t, 128, 128)
+            ent = layer_entries(csa, b, nv)
+            qi = stored_fp4(inp["q_idx"][b], inp["q_idx_scale"][b])
+            sc = orc.index_scores(qi, inp["w"][b].double().cpu().numpy(), ent["idx"], nv)
+            idx = out["idx"][b].cpu().numpy()
+            cnt = int(out["cnt"][b])
+            check_topk(idx, cnt, sc, cfg.k)
+            keys = np.vstack([orc.decode(ring_window(csa, b, t)), orc.decode(ent["kv"].take_rows(idx[:cnt]))])
+            o, _ = orc.attend(stored_bf16(inp["q_csa"][b][heads]), orc.f64(keys), cfg.d_v, scale)
+            assert_close(out["o_csa"][b][heads].float().cpu().numpy(), o, ATOL_LP, REL_LP,
+                         "csa pair %d b=%d" % (li, b))
+            hent = layer_entries(hca, b, nv_h)["kv"]
+            o, _ = orc.hca_query(t, 128, 128, stored_bf16(inp["q_hca"][b][heads]), ring_window(hca, b, t), hent,
+                                 cfg.d_v, scale)
+            assert_close(out["o_hca"][b][heads].float().cpu().numpy(), o, ATOL_LP, REL_LP,
+                         "hca pair %d b=%d" % (li, b))
