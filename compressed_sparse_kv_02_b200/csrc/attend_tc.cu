@@ -77,7 +77,8 @@ struct Smem {
   static constexpr int BAR = SEND + 2 * kRecvBytes;     // mbarriers
   static constexpr int MASK = BAR + 256;                // valid-key bits, one word per tile
   static constexpr int ROWS = MASK + kRowCap / 8;       // source row of every key of the item
-  static constexpr int TMEM = ROWS + kRowCap * 8;       // allocated tensor-memory address
+  static constexpr int SCALE = ROWS + kRowCap * 8;      // FP8 entries: the per-entry scale of every key
+  static constexpr int TMEM = SCALE + kRowCap * 4;      // allocated tensor-memory address
   static constexpr int FLAGS = TMEM + 16;
   static constexpr int PREF = FLAGS + 16;
   static size_t bytes(int n_q) { return 1024 + PREF + sizeof(int) * (size_t)(n_q + 1); }
@@ -111,9 +112,11 @@ __device__ __forceinline__ Keys keys_of(const AttendParams& p, int b) {
 
 // Source row of key u. Window keys come first: in ring-slot order (slot u)
 // when every window row is in the ring, in position order when a prefill chunk
-// supplies some of them; then the compressed entries. Null if invalid.
-__device__ __forceinline__ const uint16_t* key_src(const AttendParams& p, int b, int seq, const Keys& k,
-                                                   int64_t u) {
+// supplies some of them; then the compressed entries (bf16 rows, or FP8 rows
+// with their scale in `sc`). Null if invalid.
+__device__ __forceinline__ const void* key_src(const AttendParams& p, int b, int seq, const Keys& k, int64_t u,
+                                               float& sc) {
+  sc = 1.f;
   if (u < k.n_w) {
     if (!p.x_chunk) return p.ring_x + ((int64_t)seq * p.n_win + u) * kDqk;
     const int64_t pos = k.ws + u;
@@ -127,7 +130,25 @@ __device__ __forceinline__ const uint16_t* key_src(const AttendParams& p, int b,
   if (pi >= p.max_pages_per_seq) return nullptr;
   const int32_t page = p.page_table[(int64_t)seq * p.max_pages_per_seq + pi];
   if (page < 0 || page >= p.n_pages) return nullptr;
-  return static_cast<const uint16_t*>(p.kv_pool) + ((int64_t)page * p.page_size + j % p.page_size) * kDqk;
+  const int64_t row = (int64_t)page * p.page_size + j % p.page_size;
+  if (p.kv_dtype == CSKV_FP8_E4M3) {
+    sc = p.kv_scale[row];
+    return static_cast<const uint8_t*>(p.kv_pool) + row * kDqk;
+  }
+  return static_cast<const uint16_t*>(p.kv_pool) + row * kDqk;
+}
+
+// 8 E4M3 codes -> 8 bf16 (exact: every E4M3 value is a bf16 value)
+__device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 c) {
+  uint32_t o[4];
+  const uint32_t w[2] = {c.x, c.y};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_fp8x2_storage_t v = static_cast<__nv_fp8x2_storage_t>((w[i >> 1] >> (16 * (i & 1))) & 0xffffu);
+    const float2 f = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(v, __NV_E4M3)));
+    o[i] = pack_bf16(f.x, f.y);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // byte offset of 16-byte chunk `ch` of row `r` in a swizzled block set whose
@@ -202,7 +223,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* qbar = rempty + 2;        //     Q landed (TMA)
   uint64_t* dbar = qbar + 1;          //     MMA -> epilogue (commit after the item's last P V)
   uint32_t* sMask = reinterpret_cast<uint32_t*>(sm + Smem::MASK);
-  const uint16_t** sRow = reinterpret_cast<const uint16_t**>(sm + Smem::ROWS);
+  const void** sRow = reinterpret_cast<const void**>(sm + Smem::ROWS);
+  float* sScale = reinterpret_cast<float*>(sm + Smem::SCALE);
+  const bool fp8 = p.kv_dtype == CSKV_FP8_E4M3;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + Smem::TMEM);
   volatile int* sAbort = reinterpret_cast<int*>(sm + Smem::FLAGS);
   volatile int* sLdOk = reinterpret_cast<int*>(sm + Smem::FLAGS) + 1;  // [2] loader wait results, then [1] send flag
@@ -296,11 +319,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // source rows of this item's keys and one valid-bit word per tile, visible
     // to every role after the barrier; four independent lookups per thread
     for (int i0 = 0; i0 < ntiles * kNk; i0 += 4 * kThreads) {
-      const uint16_t* src[4];
+      const void* src[4];
+      float sc[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int i = i0 + q * kThreads + tid;
-        src[q] = (i < nk && seq_ok) ? key_src(p, b, seq, kk, u0 + i) : nullptr;
+        sc[q] = 0.f;
+        src[q] = (i < nk && seq_ok) ? key_src(p, b, seq, kk, u0 + i, sc[q]) : nullptr;
       }
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -309,6 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!src[q] && rank == 0) report(p.status, CSKV_ERR_OUT_OF_RANGE);
           sRow[i] = src[q];
         }
+        if (i < ntiles * kNk) sScale[i] = src[q] ? sc[q] : 0.f;  // finite for every slot of every tile
         const unsigned bits = __ballot_sync(kFull, src[q] != nullptr);
         if (lane == 0 && i < ntiles * kNk) sMask[i >> 5] = bits;
       }
@@ -331,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           row0 = static_cast<int>((int64_t)seq * p.n_win + a);
           return 0;
         }
-        if (!p.is_csa && a >= kk.n_w) {
+        if (!p.is_csa && !fp8 && a >= kk.n_w) {
           const int64_t j0 = a - kk.n_w;
           const int64_t pi = j0 / p.page_size;
           // whole tile inside one page and inside the item (rows past the end are not zero)
@@ -346,10 +372,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto prefetch_tile = [&](int it) {
         if (lt < kNk && it < ntiles) {
           const int i = it * kNk + lt;
-          if (i < nk && sRow[i]) prefetch_l2(sRow[i] + kb_load0 * 64, kNb * 128);
+          if (i < nk && sRow[i]) {
+            const bool row8 = fp8 && u0 + i >= kk.n_w;  // FP8 entry (window rows are bf16)
+            prefetch_l2(static_cast<const uint8_t*>(sRow[i]) + kb_load0 * 64 * (row8 ? 1 : 2), kNb * (row8 ? 64 : 128));
+          }
         }
       };
-      const bool gathered_item = p.is_csa || p.x_chunk;
+      const bool gathered_item = p.is_csa || p.x_chunk || fp8;
       if (gathered_item)
         for (int it = 0; it < kPrefetchTiles; ++it) prefetch_tile(it);
       for (int it = 0; it < ntiles; ++it) {
@@ -373,14 +402,41 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_2d(dst + j * (kNk * 128), map, (kb_load0 + j) * 64, row0, &kfull[st]);
           }
         } else {
-          // consecutive threads take consecutive 16-byte chunks of a row (coalesced)
-#pragma unroll 4
-          for (int id = lt; id < kNk * kNb * 8; id += kLoaders) {
-            const int kr = id / (kNb * 8), c = id % (kNb * 8);
-            const int i = it * kNk + kr;
-            const uint16_t* src = i < nk ? sRow[i] : nullptr;
-            cp_async16(dst + swz(kr, c, kNk * 128),
-                       src ? static_cast<const void*>(src + kb_load0 * 64 + c * 8) : p.q, src ? 16 : 0);
+          // consecutive threads take consecutive 16-byte chunks of a row (coalesced); bf16 rows go
+          // by cp.async, FP8 entries are loaded into registers first (all of this thread's loads in
+          // flight at once) and then widened to bf16 into the tile
+          constexpr int kItems = kNk * kNb * 8;
+          constexpr int kPer = (kItems + kLoaders - 1) / kLoaders;
+          uint2 codes[kPer];
+#pragma unroll
+          for (int q = 0; q < kPer; ++q) {
+            const int id = lt + q * kLoaders;
+            codes[q] = make_uint2(0u, 0u);
+            if (id < kItems) {
+              const int kr = id / (kNb * 8), c = id % (kNb * 8);
+              const int i = it * kNk + kr;
+              const void* src = i < nk ? sRow[i] : nullptr;
+              if (src && fp8 && u0 + i >= kk.n_w)
+                codes[q] = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(src) + kb_load0 * 64 +
+                                                                c * 8));
+              else
+                cp_async16(dst + swz(kr, c, kNk * 128),
+                           src ? static_cast<const void*>(static_cast<const uint16_t*>(src) + kb_load0 * 64 + c * 8)
+                               : p.q,
+                           src ? 16 : 0);
+            }
+          }
+          if (fp8) {
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) {
+              const int id = lt + q * kLoaders;
+              if (id < kItems) {
+                const int kr = id / (kNb * 8), c = id % (kNb * 8);
+                const int i = it * kNk + kr;
+                if (i < nk && sRow[i] && u0 + i >= kk.n_w)
+                  *reinterpret_cast<uint4*>(dst + swz(kr, c, kNk * 128)) = e4m3x8_to_bf16x8(codes[q]);
+              }
+            }
           }
           cp_async_commit();
           cp_async_wait<0>();
@@ -527,6 +583,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t valid = sMask[it];
         float v[32];
         float mt = -INFINITY;
+        if (fp8) {  // an FP8 entry's logit and value carry its scale
+#pragma unroll
+          for (int j = 0; j < 32; ++j) cur[j] *= sScale[it * kNk + j];
+        }
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           v[j] = ((valid >> j) & 1u) ? cur[j] * sl2 : -INFINITY;  // keys past nk have no row
@@ -546,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 16; ++j) {
           const float p0 = exp2f(v[2 * j] - msub), p1 = exp2f(v[2 * j + 1] - msub);
           l_run += p0 + p1;
-          pp[j] = pack_bf16(p0, p1);
+          pp[j] = fp8 ? pack_bf16(p0 * sScale[it * kNk + 2 * j], p1 * sScale[it * kNk + 2 * j + 1]) : pack_bf16(p0, p1);
         }
         // P buffer gt % 3 was read by the P V of tile gt - 3
         if (gt >= (uint32_t)kNSP && !__all_sync(kFull, mbar_wait(&obar[buf], ((gt / kNSP) - 1) & 1u, p.status)))
@@ -633,7 +693,7 @@ bool encode_rows(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box
 }  // namespace
 
 bool attend_tc_supported(int d_qk, int d_v, int n_heads, int kv_dtype, int n_q) {
-  return d_qk == kDqk && d_v == kDv && n_heads % kM == 0 && kv_dtype == CSKV_BF16 &&
+  return d_qk == kDqk && d_v == kDv && n_heads % kM == 0 && (kv_dtype == CSKV_BF16 || kv_dtype == CSKV_FP8_E4M3) &&
          Smem::bytes(n_q) <= 232448;  // the per-query prefix table shares shared memory with the tiles
 }
 
@@ -658,7 +718,10 @@ cudaError_t launch_attend_tc(AttendParams& p, int n_sm, cudaStream_t st) {
   const uint64_t ring_rows = static_cast<uint64_t>(p.n_seqs_layer) * p.n_win;
   if (kv_rows >= (1ull << 31) || ring_rows >= (1ull << 31)) return cudaErrorNotSupported;
   if (!encode_rows(&tm_q, p.q, static_cast<uint64_t>(p.n_q) * p.n_heads, kM) ||
-      !encode_rows(&tm_ring, p.ring_x, ring_rows, kNk) || !encode_rows(&tm_kv, p.kv_pool, kv_rows, kNk))
+      !encode_rows(&tm_ring, p.ring_x, ring_rows, kNk) ||
+      // an FP8 pool is never read by TMA (its tiles are widened by the loaders)
+      !encode_rows(&tm_kv, p.kv_dtype == CSKV_FP8_E4M3 ? static_cast<const void*>(p.ring_x) : p.kv_pool,
+                   p.kv_dtype == CSKV_FP8_E4M3 ? ring_rows : kv_rows, kNk))
     return cudaErrorNotSupported;
   const size_t smem = Smem::bytes(p.n_q);
   cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

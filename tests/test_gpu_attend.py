@@ -119,8 +119,10 @@ def test_short_selection_and_no_lse(ck, orc):
 
 
 @pytest.mark.parametrize("kind", ["csa", "hca"])
-def test_fp8_kv(ck, orc, kind):
-    _run(ck, orc, kind, 576, 512, 64, [127 + 128 * 30 + 3, 129], fp8=True, k=256, seed=14)
+@pytest.mark.parametrize("H", [64, 128])  # 128 heads take the tensor-memory kernel, 64 the generic one
+def test_fp8_kv(ck, orc, kind, H):
+    _run(ck, orc, kind, 576, 512, H, [127 + 128 * 30 + 3, 129, 127 + 128 * 90 + 64], fp8=True, k=256, seed=14)
+    _run(ck, orc, kind, 576, 512, H, [127 + 128 * 40 + 5], fp8=True, k=512, sharp=True, seed=15)
 
 
 def test_prefill_chunk_window(ck, orc):
