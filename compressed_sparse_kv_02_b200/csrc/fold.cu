@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(kBlockFoldThreads) fold_bulk_block_kernel(Fold
   }
 }
 
-constexpr int kAppendWarps = 4;
+constexpr int kAppendWarps = 16;  // an FP8 entry is folded whole by one CTA: 36 units of 16 channels at d = 576
 constexpr int kAppendThreads = 32 * kAppendWarps;
 constexpr int kSliceCh = 64;       // channels per CTA of the append kernel (whole row for FP8)
 constexpr int kAppendMaxD = 1024;  // channels of the row buffer
@@ -408,9 +408,11 @@ __device__ void store_row(const FoldStream& S, int64_t row, const float* sv, int
 // new rows into the rings, then folds its channels of every block the new
 // tokens complete (old rows from the ring, new rows from the input; the slots
 // written and the slots read never coincide because n_new + m - 1 <= n_win).
-// A warp folds 16 channels at a time: each lane runs the online softmax over
-// tokens lane, lane + 32, ... of the block, and the 32 partial states merge
-// by shuffles; the entry is stored from a shared-memory row buffer.
+// A group of lanes folds 16 channels: each lane runs the online softmax over
+// its tokens of the block and the group's partial states merge by shuffles
+// (a group is 32 lanes for m >= 32, else the next power of two >= m, so a warp
+// folds several 16-channel units at once); the entry is stored from a
+// shared-memory row buffer.
 __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
   __shared__ float sv[kAppendMaxD];
   __shared__ float s_red[kAppendWarps];
@@ -450,7 +452,13 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
   while (merge_span < 32 && merge_span < p.m) merge_span <<= 1;
   for (int64_t j = j_first; j <= j_last; ++j) {
     const int64_t row = entry_row(p, seq, j);  // uniform across the block
-    for (int c0 = c_lo + 16 * warp; c0 < c_hi; c0 += 16 * kAppendWarps) {
+    // lanes in groups of merge_span (a power of two >= min(m, 32)): group g of the warp folds
+    // 16-channel unit (base + g) with one lane per token
+    const int per_warp = 32 / merge_span;
+    const int grp = lane / merge_span, tok = lane % merge_span;
+    for (int u0 = c_lo / 16 + warp * per_warp; u0 < c_hi / 16; u0 += kAppendWarps * per_warp) {
+      const int c0 = (u0 + grp) * 16;
+      const bool active = c0 < c_hi;
       float mx[16], den[16], acc[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
@@ -458,7 +466,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
         den[e] = 0.f;
         acc[e] = 0.f;
       }
-      for (int i = lane; i < p.m; i += 32) {
+      for (int i = tok; active && i < p.m; i += merge_span) {
         const int64_t q = j * p.m + i;
         const uint16_t* xr;
         const uint16_t* zr;
@@ -510,7 +518,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
       }
       // lanes >= m hold nothing: merge only across the lanes that ran tokens
       for (int o = merge_span >> 1; o > 0; o >>= 1) merge16(mx, den, acc, o);
-      if (lane == 0)
+      if (active && tok == 0)
 #pragma unroll
         for (int e = 0; e < 16; ++e) sv[c0 + e] = acc[e] / den[e];
     }
