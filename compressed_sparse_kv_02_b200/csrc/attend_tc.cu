@@ -381,6 +381,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool gathered_item = p.is_csa || p.x_chunk || fp8;
       if (gathered_item)
         for (int it = 0; it < kPrefetchTiles; ++it) prefetch_tile(it);
+      // Gathered tiles are pipelined by one: tile it's loads are issued before tile it-1 is finished
+      // (its FP8 rows widened, its cp.async group waited for) and signalled.
+      constexpr int kItems = kNk * kNb * 8;
+      constexpr int kPer = (kItems + kLoaders - 1) / kLoaders;
+      uint2 pend_codes[kPer];
+      int pend_it = -1;  // gathered tile still to be finished
+      bool stopped = false;  // uniform over the loaders (decided after a named barrier)
+      auto finish = [&](int pit, bool newer_group) {
+        const uint32_t pgt = g + pit;
+        uint8_t* pdst = sK + (pgt % kNS) * kStageBytes;
+        if (fp8) {
+#pragma unroll
+          for (int q = 0; q < kPer; ++q) {
+            const int id = lt + q * kLoaders;
+            if (id < kItems) {
+              const int kr = id / (kNb * 8), c = id % (kNb * 8);
+              const int i = pit * kNk + kr;
+              if (i < nk && sRow[i] && u0 + i >= kk.n_w)
+                *reinterpret_cast<uint4*>(pdst + swz(kr, c, kNk * 128)) = e4m3x8_to_bf16x8(pend_codes[q]);
+            }
+          }
+        }
+        if (newer_group) cp_async_wait<1>(); else cp_async_wait<0>();
+        fence_proxy_async_smem();
+        named_sync(3, kLoaders);
+        if (lt == 0) mbar_arrive(&kfull[pgt % kNS]);
+      };
       for (int it = 0; it < ntiles; ++it) {
         const uint32_t gt = g + it;
         const int st = gt % kNS;
@@ -390,7 +417,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lt == 0)
           sLdOk[it & 1] = !*sAbort && (gt < (uint32_t)kNS || mbar_wait(&kempty[st], ((gt / kNS) - 1) & 1u, p.status));
         named_sync(3, kLoaders);
-        if (!sLdOk[it & 1]) { *sAbort = 1; break; }
+        if (!sLdOk[it & 1]) {
+          *sAbort = 1;
+          stopped = true;
+          break;
+        }
         uint8_t* dst = sK + st * kStageBytes;
         int row0 = 0;
         const int mode = tile_src(it, row0);
@@ -401,12 +432,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < kNb; ++j)
               tma_load_2d(dst + j * (kNk * 128), map, (kb_load0 + j) * 64, row0, &kfull[st]);
           }
+          if (pend_it >= 0) finish(pend_it, false);
+          pend_it = -1;
         } else {
           // consecutive threads take consecutive 16-byte chunks of a row (coalesced); bf16 rows go
-          // by cp.async, FP8 entries are loaded into registers first (all of this thread's loads in
-          // flight at once) and then widened to bf16 into the tile
-          constexpr int kItems = kNk * kNb * 8;
-          constexpr int kPer = (kItems + kLoaders - 1) / kLoaders;
+          // by cp.async, FP8 entries into registers (widened into the tile when it is finished)
           uint2 codes[kPer];
 #pragma unroll
           for (int q = 0; q < kPer; ++q) {
@@ -426,25 +456,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                            src ? 16 : 0);
             }
           }
-          if (fp8) {
-#pragma unroll
-            for (int q = 0; q < kPer; ++q) {
-              const int id = lt + q * kLoaders;
-              if (id < kItems) {
-                const int kr = id / (kNb * 8), c = id % (kNb * 8);
-                const int i = it * kNk + kr;
-                if (i < nk && sRow[i] && u0 + i >= kk.n_w)
-                  *reinterpret_cast<uint4*>(dst + swz(kr, c, kNk * 128)) = e4m3x8_to_bf16x8(codes[q]);
-              }
-            }
-          }
           cp_async_commit();
-          cp_async_wait<0>();
-          fence_proxy_async_smem();
-          named_sync(3, kLoaders);
-          if (lt == 0) mbar_arrive(&kfull[st]);
+          if (pend_it >= 0) finish(pend_it, true);
+#pragma unroll
+          for (int q = 0; q < kPer; ++q) pend_codes[q] = codes[q];
+          pend_it = it;
         }
       }
+      if (pend_it >= 0 && !stopped) finish(pend_it, false);
     } else if (tid == kMmaThread) {
       // ------------------------------------------------------------ MMA issue
       const uint32_t idesc_s = umma_idesc_bf16(kM, kNk, false);
