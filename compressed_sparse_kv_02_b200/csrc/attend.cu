@@ -390,6 +390,8 @@ __global__ void __launch_bounds__(256) attend_merge_kernel(AttendParams p) {
 // written by attend_tc_kernel): a CTA takes 128 consecutive heads x 2 groups of 4
 // channels, so every partial-output load is a warp's 512 contiguous bytes.
 __global__ void __launch_bounds__(256) attend_merge_t_kernel(AttendParams p) {
+  grid_dependency_wait();  // the partial outputs come from the attention kernel ahead of this one
+  grid_dependents_launch();
   const int b = blockIdx.x;
   const QueryKeys qk = query_keys(p, b);
   const int ns = static_cast<int>((qk.n + p.keys_per_split - 1) / p.keys_per_split);
@@ -477,8 +479,7 @@ cudaError_t launch_attend_merge(AttendParams& p, cudaStream_t st) {
   if (p.part_t) {
     dim3 mg(static_cast<unsigned>(p.n_q), static_cast<unsigned>((p.d_v / 4 + 1) / 2),
             static_cast<unsigned>((p.n_heads + 127) / 128));
-    attend_merge_t_kernel<<<mg, 256, 0, st>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(attend_merge_t_kernel, mg, dim3(256), 0, st, p);
   }
   const int hb = 256 / (p.d_v / 4);
   dim3 mg(static_cast<unsigned>(p.n_q), static_cast<unsigned>((p.n_heads + hb - 1) / hb));

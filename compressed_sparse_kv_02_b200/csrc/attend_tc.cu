@@ -243,22 +243,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int qkb0 = rank ? 5 : 0;      // channel block of its Q block 0
   const int s_blk0 = rank ? 1 : 0;    // first S block inside a stage (blocks 0..3 are V)
 
-  {  // items per query: splits x head groups
-    int run = 0;
-    for (int base = 0; base < p.n_q; base += kThreads) {
-      const int b = base + tid;
-      int v = 0;
-      if (b < p.n_q) {
-        const Keys k = keys_of(p, b);
-        v = static_cast<int>((k.n + kps - 1) / kps) * groups;
-      }
-      int tot;
-      const int ex = block_exclusive_scan<kThreads>(v, s_wsum, tot);
-      if (b < p.n_q) sPref[b] = run + ex;
-      run += tot;
-    }
-    if (tid == 0) sPref[p.n_q] = run;
-  }
   if (tid == 0) {
     for (int i = 0; i < kNS; ++i) {
       mbar_init(&kfull[i], 1);
@@ -291,6 +275,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster.sync();  // barriers of both CTAs initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem = *sTmem;
+  // the set-up above overlaps the tail of the kernel launched before this one; its
+  // outputs (the selection, new cache rows) are read only from here on
+  grid_dependency_wait();
+  grid_dependents_launch();
+  {  // items per query: splits x head groups
+    int run = 0;
+    for (int base = 0; base < p.n_q; base += kThreads) {
+      const int b = base + tid;
+      int v = 0;
+      if (b < p.n_q) {
+        const Keys k = keys_of(p, b);
+        v = static_cast<int>((k.n + kps - 1) / kps) * groups;
+      }
+      int tot;
+      const int ex = block_exclusive_scan<kThreads>(v, s_wsum, tot);
+      if (b < p.n_q) sPref[b] = run + ex;
+      run += tot;
+    }
+    if (tid == 0) sPref[p.n_q] = run;
+  }
+  __syncthreads();
   if (blockIdx.x == 0)
     for (int b = tid; b < p.n_q; b += kThreads)
       if (p.q_pos[b] < 0 || p.q_pos[b] > p.max_pos) report(p.status, CSKV_ERR_INVALID_ARG);
@@ -754,13 +759,15 @@ cudaError_t launch_attend_tc(AttendParams& p, int n_sm, cudaStream_t st) {
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   p.part_t = 1;
   e = cudaLaunchKernelEx(&cfg, attend_tc_kernel, tm_q, tm_ring, tm_kv, p);
   if (e != cudaSuccess) return e;

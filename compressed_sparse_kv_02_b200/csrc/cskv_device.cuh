@@ -45,6 +45,14 @@ __device__ __forceinline__ float key2f(uint32_t k) {
   return __uint_as_float(u);
 }
 
+// Programmatic dependent launch: a kernel launched behind this one may start
+// once every CTA here has called grid_dependents_launch (or exited); it calls
+// grid_dependency_wait before it reads anything this grid writes, which waits
+// for this whole grid to finish and its writes to be visible. Both are no-ops
+// for plain launches.
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
 // ---------------------------------------------------------------- loads
 __device__ __forceinline__ uint4 ldg16(const void* p) {
   uint4 v;

@@ -11,6 +11,24 @@
 
 namespace cskv {
 
+// Launch `kern` with programmatic dependent launch allowed: it may be scheduled
+// before the kernel ahead of it on the stream has finished, and must call
+// grid_dependency_wait() before it reads anything that kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // cuTensorMapEncodeTiled, looked up once through the runtime (null if unavailable)
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 

@@ -418,6 +418,8 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
   __shared__ float s_red[kAppendWarps];
   const int b = blockIdx.x, slice = blockIdx.y, si = blockIdx.z;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  grid_dependency_wait();  // every input may come from the kernel launched before this one
+  grid_dependents_launch();
   const int seq = p.seq_ids[b];
   if (seq < 0 || seq >= p.n_seqs_layer) {
     if (t == 0 && slice == 0 && si == 0) report(p.status, CSKV_ERR_OUT_OF_RANGE);
@@ -556,8 +558,7 @@ cudaError_t launch_append(const FoldParams& p, cudaStream_t st) {
   }
   dim3 grid(static_cast<unsigned>(p.n_seq), static_cast<unsigned>((dmax + kSliceCh - 1) / kSliceCh),
             static_cast<unsigned>(p.n_streams));
-  append_kernel<<<grid, kAppendThreads, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(append_kernel, grid, dim3(kAppendThreads), 0, st, p);
 }
 
 }  // namespace cskv

@@ -44,14 +44,6 @@ constexpr int kSliceCap = 32768;   // scores per CTA of the selection kernel
 constexpr int kMaxCluster = 16;   // CTAs per query in the selection kernel (above 8: non-portable)
 constexpr int kHistBins = 2048;   // bins of the score-key histogram the TMA scan leaves for the selection
 
-// Programmatic dependent launch: a kernel launched behind this one may start
-// once every CTA here has called grid_dependents_launch (or exited); it calls
-// grid_dependency_wait before it reads anything this grid writes, which waits
-// for this whole grid to finish and its writes to be visible. Both are no-ops
-// for plain launches.
-__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
-__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
-
 __device__ __forceinline__ int64_t query_visible(const IndexParams& p, int b) {
   const int64_t t = p.q_pos[b];
   if (t < 0 || t > p.max_pos) return -1;
@@ -354,6 +346,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
   // contexts) counts straight into the global histogram
   __shared__ uint32_t s_h[2][kHistBins];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  grid_dependency_wait();     // the keys may have been written by the kernel launched before this one
   grid_dependents_launch();  // the selection kernel may be scheduled as SMs free up
   for (int i = tid; i < 2 * kHistBins; i += kTmaThreads) (&s_h[0][0])[i] = 0u;
 
@@ -681,6 +674,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
   const int64_t hi = lo + p.slice < nv ? lo + p.slice : nv;
   const int len = hi > lo ? static_cast<int>(hi - lo) : 0;
   grid_dependency_wait();  // the scores and the digit-A histogram come from the scan
+  grid_dependents_launch();
   __syncthreads();
   // the slice's scores (whole 16-byte pieces) land by one bulk copy while digit A is found
   const int n4 = nv > k ? len >> 2 : 0;
@@ -1013,8 +1007,7 @@ cudaError_t launch_scan_tma(IndexParams& p, int n_sm, cudaStream_t st) {
   int64_t grid = units_max * p.n_q;
   if (grid > n_sm) grid = n_sm;
   if (grid < 1) grid = 1;
-  kern<<<static_cast<int>(grid), kTmaThreads, smem, st>>>(map, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(kTmaThreads), smem, st, map, p);
 }
 
 }  // namespace
