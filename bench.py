@@ -38,6 +38,7 @@ import torch  # noqa: E402
 METRIC = "CSA/HCA decode queries/s at 1M ctx; HBM GB/s vs peak; prefill tok/s"
 UNIT = "queries/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1400.0  # sustained under the power cap (earlier measurement on this machine)
 EVENT_STEPS = 32  # steps per captured graph (each with its own timing events)
 
 
@@ -206,6 +207,173 @@ def max_over_ranks(x, device, world):
 def whole_job_rate(units_per_rank, world, ms_max):
     """Units of all ranks per second of the slowest rank."""
     return units_per_rank * world / (ms_max * 1e-3)
+
+
+def bf16_peak_sustained():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops_sustained" in d:
+            return float(d["bf16_tflops_sustained"]), "measured (sustained)"
+    return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+# ----------------------------------------------------------------- prefill arm
+PREFILL_CACHED = 65536
+PREFILL_CHUNK = 65536
+
+
+def run_prefill(args, rank, world):
+    """One step = one prefill pass of a 65,536-token chunk onto 65,536 cached tokens through a CSA and an HCA
+    layer (compression, indexer + top-k and both attentions for every position of the chunk)."""
+    import compressed_sparse_kv_02_b200 as ck
+    from compressed_sparse_kv_02_b200 import prefill, synth
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    cfg = rank_config(synth.CONFIGS["prefill"], rank)
+    model = prefill.PrefillModel(cfg, cached=PREFILL_CACHED, chunk=PREFILL_CHUNK, device="cuda")
+    model.fill_synthetic()
+    model.prepare()
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            model.step(stream)
+    stream.synchronize()
+    if model.check_status() != ck.OK:
+        raise RuntimeError("device status after warm-up: %s" % ck.status_string(model.check_status()))
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = ClockSampler()
+    clocks.start()
+    time.sleep(0.2)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(args.steps):
+            model.step(stream)
+        t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    if model.check_status() != ck.OK:
+        raise RuntimeError("device status after the timed region: %s" % ck.status_string(model.check_status()))
+    ms_step = max_over_ranks(t0.elapsed_time(t1) / args.steps, dev, world)
+    value = whole_job_rate(PREFILL_CHUNK, world, ms_step)
+    fl = model.flops()
+    peak, src = bf16_peak_sustained()
+    achieved = fl["total"] / (ms_step * 1e-3) / 1e12
+
+    # end to end: the chunk's inputs copied in from pinned host memory and the outputs copied out, every pass
+    names = ("x", "z", "xi", "zi", "x_h", "z_h", "q", "q_h", "q_idx", "w")
+    host = {k_: torch.empty(model.inputs[k_].shape, dtype=model.inputs[k_].dtype, pin_memory=True) for k_ in names}
+    for k_ in names:
+        host[k_].copy_(model.inputs[k_].cpu())
+    outs = (model.idx, model.o_csa, model.o_hca)
+    host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    h2d = sum(host[k_].numel() * host[k_].element_size() for k_ in names)
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    e2e_steps = 2
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            for k_ in names:
+                model.inputs[k_].copy_(host[k_], non_blocking=True)
+            model.step(stream)
+            for o, ho in zip(outs, host_out):
+                ho.copy_(o, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev, world)
+    n_blocks = -(-PREFILL_CHUNK // model.q_block)
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded Gaussian caches, raw chunk and queries)",
+        "config": {
+            "workload": "prefill chunk: %d new tokens on %d cached (one sequence), H=%d, d=%d (K=V), indexer "
+                        "%dx%d, CSA m=4 top-%d, HCA m'=128, window 128, one CSA + one HCA layer"
+                        % (PREFILL_CHUNK, PREFILL_CACHED, cfg.heads, cfg.d_qk, cfg.heads_idx, cfg.d_idx, cfg.k),
+            "config_name": cfg.name,
+            "parallelism": "replicas" if world == 1 else "dp%d (independent sequences per GPU)" % world,
+            "l2": "inputs larger than L2 (queries alone %.0f MB)" % (2 * model.inputs["q"].numel() * 2 / 1e6),
+            "timing": "%d eager passes between CUDA events on the launching stream" % args.steps,
+        },
+        "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"],
+                   "samples": clk["samples"]},
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "whole prefill pass (indexer scan + top-k + CSA and HCA attention)",
+            "achieved": round(achieved, 1),
+            "peak": peak,
+            "peak_source": src,
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": None,
+            "algorithmic_flops_per_step": fl,
+        },
+        "e2e": {"value": round(whole_job_rate(PREFILL_CHUNK, world, e2e_ms), 2), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": (6 + 6 * n_blocks) * args.steps,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = prefill_cpu_baseline(model, cfg, budget_s=args.cpu_budget)
+    return out
+
+
+def prefill_cpu_baseline(model, cfg, budget_s=20.0):
+    """The oracle on sampled chunk positions (window rows from the chunk), scaled to tokens/s."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import oracle
+    from gpu_helpers import layer_entries, stored_bf16
+    oracle.build()
+    cores = os.cpu_count() or 1
+    oracle.set_threads(cores)
+    csa, hca = model.layers
+    inp, c0 = model.inputs, model.cached
+    sm = 1.0 / math.sqrt(cfg.d_qk)
+    g = torch.Generator().manual_seed(cfg.seed)
+    pos = [c0 + 127, c0 + model.chunk - 1] + torch.randint(c0 + 128, c0 + model.chunk - 1, (4096,),
+                                                             generator=g).tolist()
+    ent = layer_entries(csa, 0, oracle.visible_entries(c0 + model.chunk - 1, cfg.m_csa, cfg.n_win))
+    ent_h = layer_entries(hca, 0, oracle.visible_entries(c0 + model.chunk - 1, cfg.m_hca, cfg.n_win))["kv"]
+    done, t_cpu = 0, 0.0
+    for t in pos:
+        if t_cpu >= budget_s:
+            break
+        i = t - c0
+        nv = oracle.visible_entries(t, cfg.m_csa, cfg.n_win)
+        nvh = oracle.visible_entries(t, cfg.m_hca, cfg.n_win)
+        win = stored_bf16(inp["x"][0, max(0, i - 127):i + 1])
+        win_h = stored_bf16(inp["x_h"][0, max(0, i - 127):i + 1])
+        if i < 127:
+            continue  # keep the sample to positions whose window lies inside the chunk
+        x = dict(q=stored_bf16(inp["q"][i]), qi=stored_bf16(inp["q_idx"][i]), w=inp["w"][i].double().cpu().numpy(),
+                 kv=ent["kv"].rows_subset(0, nv), ki=ent["idx"].rows_subset(0, nv), kvh=ent_h.rows_subset(0, nvh),
+                 qh=stored_bf16(inp["q_h"][i]))
+        t0 = time.perf_counter()
+        oracle.csa_query(t, cfg.m_csa, cfg.n_win, cfg.k, x["q"], x["qi"], x["w"], win, x["kv"], x["ki"], cfg.d_v, sm)
+        oracle.hca_query(t, cfg.m_hca, cfg.n_win, x["qh"], win_h, x["kvh"], cfg.d_v, sm)
+        t_cpu += time.perf_counter() - t0
+        done += 1
+    return {"value": round(done / t_cpu, 4), "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "%d sampled chunk positions (indexer + top-k + CSA and HCA attention per position, fp64; "
+                      "compression not timed), %.1f s of host time, extrapolated to tokens/s" % (done, t_cpu)}
 
 
 # ----------------------------------------------------------------- our arm
@@ -528,7 +696,7 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        out = run_ours(args, rank, world)
+        out = run_prefill(args, rank, world) if args.config == "prefill" else run_ours(args, rank, world)
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:
