@@ -203,6 +203,9 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, const void* src,
 //              P(gt) (+ rare O rescale after P V of tile gt - 1) -> arrive pfull
 // S(gt) needs the softmax only up to tile gt - 3 and the softmax needs S only
 // one tile ahead, so neither waits on the other's latest step.
+// FP8: the pool holds E4M3 entries with an fp32 scale each (a separate instantiation keeps
+// the bf16 kernel's code, and so its instruction-cache footprint, small)
+template <bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ring,
                      const __grid_constant__ CUtensorMap tm_kv, AttendParams p) {
@@ -225,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* sMask = reinterpret_cast<uint32_t*>(sm + Smem::MASK);
   const void** sRow = reinterpret_cast<const void**>(sm + Smem::ROWS);
   float* sScale = reinterpret_cast<float*>(sm + Smem::SCALE);
-  const bool fp8 = p.kv_dtype == CSKV_FP8_E4M3;
+  constexpr bool fp8 = FP8;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + Smem::TMEM);
   volatile int* sAbort = reinterpret_cast<int*>(sm + Smem::FLAGS);
   volatile int* sLdOk = reinterpret_cast<int*>(sm + Smem::FLAGS) + 1;  // [2] loader wait results, then [1] send flag
@@ -483,8 +486,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (it < ntiles) {
           const uint32_t gt = g + it;
           const int st = gt % kNS, buf = gt % kNSP;
+          // the tile is shared memory written by TMA or fenced cp.async / stores: the mbarrier
+          // orders it; tensor memory reuse is ordered by the fence after the P waits below
           if (!(ok = mbar_wait(&kfull[st], (gt / kNS) & 1u, p.status))) break;
-          tc_fence_after();
           const uint64_t dk = dk0 + ((st * kStageBytes) >> 4);
           const uint32_t d = tmem + kColS + buf * kNk;
           // 16 or 20 MMAs (issue-bound at N = 32, so one accumulator costs nothing)
@@ -748,7 +752,9 @@ cudaError_t launch_attend_tc(AttendParams& p, int n_sm, cudaStream_t st) {
                    p.kv_dtype == CSKV_FP8_E4M3 ? ring_rows : kv_rows, kNk))
     return cudaErrorNotSupported;
   const size_t smem = Smem::bytes(p.n_q);
-  cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const bool fp8 = p.kv_dtype == CSKV_FP8_E4M3;
+  auto kern = fp8 ? attend_tc_kernel<true> : attend_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int64_t upper = (int64_t)p.n_q * p.max_splits * (p.n_heads / kM);
@@ -769,7 +775,7 @@ cudaError_t launch_attend_tc(AttendParams& p, int n_sm, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   p.part_t = 1;
-  e = cudaLaunchKernelEx(&cfg, attend_tc_kernel, tm_q, tm_ring, tm_kv, p);
+  e = cudaLaunchKernelEx(&cfg, kern, tm_q, tm_ring, tm_kv, p);
   if (e != cudaSuccess) return e;
   return launch_attend_merge(p, st);
 }
