@@ -180,7 +180,7 @@ def workload_text(cfg, nq, model):
 # the scan and select kernels on the Pro workload at batch 2, scaled by queries
 # (profiles/decode_pro_b2_kernels_full.md); None for other workloads or once
 # those kernels change.
-INDEX_OP_DRAM_BYTES_PER_QUERY = {"pro": (134.303232e6 + 4.073728e6 + 2.179328e6) / 2}
+INDEX_OP_DRAM_BYTES_PER_QUERY = {"pro": (134.301440e6 + 4.370944e6 + 2.179840e6) / 2}
 
 
 def index_op_traffic(cfg, nq):
