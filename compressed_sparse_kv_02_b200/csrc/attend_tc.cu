@@ -191,6 +191,23 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, const void* src,
                "r"(smem_u32(src)), "r"(bytes), "r"(mbar)
                : "memory");
 }
+// Partial S of one key tile: NB channel blocks, the first NQS with Q in shared memory, the rest
+// with Q in tensor memory; fully unrolled, every descriptor built from its 32-bit address (the
+// constant upper half then folds away, which keeps the issue loop short).
+template <int NB, int NQS>
+__device__ __forceinline__ void issue_s(uint32_t d, uint32_t q_smem, uint32_t q_tmem, uint32_t k_smem,
+                                        uint32_t idesc) {
+#pragma unroll
+  for (int k = 0; k < 4 * NB; ++k) {
+    const int j = k >> 2, ks = k & 3;
+    const uint64_t db = umma_desc_sw128(k_smem + j * (kNk * 128) + ks * 32, 16, 1024);
+    if (j < NQS)
+      umma_ss(d, umma_desc_sw128(q_smem + j * (kM * 128) + ks * 32, 16, 1024), db, idesc, k > 0 ? 1u : 0u);
+    else
+      umma_ts(d, q_tmem + (j - NQS) * 32 + ks * 8, db, idesc, k > 0 ? 1u : 0u);
+  }
+}
+
 // Pipeline (per CTA; tiles numbered gt across the items of the cluster, the
 // same in both CTAs; stage gt % kNS, S / P buffer gt % 3, exchange slot gt & 1):
 //   loaders  : wait kempty (P V of tile gt - kNS done) -> TMA, or cp.async +
@@ -477,10 +494,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_s = umma_idesc_bf16(kM, kNk, false);
       const uint32_t idesc_pv = umma_idesc_bf16(kM, 256, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK);
-      // descriptors differ only in the start address (low 14 bits, in 16-byte units)
-      const uint64_t dq0 = umma_desc_sw128(sQa, 16, 1024);
-      const uint64_t dk0 = umma_desc_sw128(sKa + s_blk0 * (kNk * 128), 16, 1024);
-      const uint64_t dv0 = umma_desc_sw128(sKa, kNk * 128, 1024);
       bool ok = mbar_wait(qbar, n_item & 1u, p.status);
       for (int it = 0; it <= ntiles + 1 && ok && !*sAbort; ++it) {
         if (it < ntiles) {
@@ -489,21 +502,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the tile is shared memory written by TMA or fenced cp.async / stores: the mbarrier
           // orders it; tensor memory reuse is ordered by the fence after the P waits below
           if (!(ok = mbar_wait(&kfull[st], (gt / kNS) & 1u, p.status))) break;
-          const uint64_t dk = dk0 + ((st * kStageBytes) >> 4);
           const uint32_t d = tmem + kColS + buf * kNk;
-          // 16 or 20 MMAs (issue-bound at N = 32, so one accumulator costs nothing)
-#pragma unroll 1
-          for (int j = 0; j < n_sblk; ++j) {
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t db = dk + ((j * (kNk * 128) + ks * 32) >> 4);
-              const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
-              if (j < n_qs)
-                umma_ss(d, dq0 + ((j * (kM * 128) + ks * 32) >> 4), db, idesc_s, acc);
-              else
-                umma_ts(d, tmem + kColQ + (j - n_qs) * 32 + ks * 8, db, idesc_s, acc);
-            }
-          }
+          const uint32_t kb = sKa + st * kStageBytes + s_blk0 * (kNk * 128);
+          // 20 (rank 0) or 16 (rank 1) MMAs into one accumulator
+          if (rank == 0)
+            issue_s<5, 2>(d, sQa, tmem + kColQ, kb, idesc_s);
+          else
+            issue_s<4, 1>(d, sQa, tmem + kColQ, kb, idesc_s);
           umma_commit(&sfull[buf]);
         }
         if (it >= 2) {
@@ -511,11 +516,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int pb = gp % kNSP, sp = gp % kNS;
           if (!(ok = mbar_wait(&pfull[pb], (gp / kNSP) & 1u, p.status))) break;
           tc_fence_after();
-          const uint64_t dv = dv0 + ((sp * kStageBytes) >> 4);  // blocks 0..3 of the stage: this CTA's V
+          const uint32_t vb = sKa + sp * kStageBytes;  // blocks 0..3 of the stage: this CTA's V
 #pragma unroll
           for (int k2 = 0; k2 < 2; ++k2)
-            umma_ts(tmem + kColO, tmem + kColP + pb * 16 + k2 * 8, dv + ((k2 * 16 * 128) >> 4), idesc_pv,
-                    (it > 2 || k2 > 0) ? 1u : 0u);
+            umma_ts(tmem + kColO, tmem + kColP + pb * 16 + k2 * 8,
+                    umma_desc_sw128(vb + k2 * 16 * 128, kNk * 128, 1024), idesc_pv, (it > 2 || k2 > 0) ? 1u : 0u);
           umma_commit(&kempty[sp]);
           umma_commit(&obar[pb]);
         }
