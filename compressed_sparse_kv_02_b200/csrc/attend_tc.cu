@@ -536,13 +536,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t rempty_peer = peer_addr(rempty, peer);
       const int rr = tid;  // head row
       float m_used = -INFINITY, l_run = 0.f;
-      // Loop control stays uniform over the 128 threads (they meet at named
-      // barriers inside produce): it changes only through the flag read after
-      // produce's second barrier. A failed wait elsewhere raises the abort flag
-      // and lets the iteration finish on whatever data is there.
+      // Loop control is per warp (the four warps never meet at a barrier inside the loop); a
+      // failed wait raises the abort flag, and the other warps stop at their next bounded wait.
       bool ok = true;
       float part[32];
-      volatile int* sSendOk = sLdOk + 2;  // [1] published by thread 0 inside produce
       // own partial of tile gt into part[], and one bulk copy of it into the other CTA's slot gt & 1
       auto produce = [&](uint32_t gt) -> bool {
         const int buf = gt % kNSP, slot = gt & 1;
@@ -553,23 +550,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
 #pragma unroll
         for (int j = 0; j < 32; ++j) part[j] = __uint_as_float(s0[j]);
-        // slot gt & 1 of the send buffers here and of the receive slots there held
-        // tile gt - 2: both are free once the other CTA has read that tile
-        if (tid == 0) *sSendOk = !*sAbort && (gt < 2 || mbar_wait(&rempty[slot], ((gt >> 1) - 1) & 1u, p.status));
-        named_sync(1, kM);
-        const bool sent = *sSendOk != 0;
-        uint8_t* sbuf = sSend + slot * kRecvBytes;
+        // slot gt & 1 of the send buffers here and of the receive slots there held tile gt - 2:
+        // both are free once the other CTA has read that tile. Each warp sends its own 32 rows
+        // (4 KB) by its own bulk copy, so the warps need not meet.
+        bool sent = !*sAbort;
+        if (lane == 0 && sent && gt >= 2) sent = mbar_wait(&rempty[slot], ((gt >> 1) - 1) & 1u, p.status);
+        sent = __shfl_sync(kFull, sent, 0);
         if (sent) {
-          uint8_t* row = sbuf + rr * 128;
+          uint8_t* row = sSend + slot * kRecvBytes + rr * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c)
             *reinterpret_cast<uint4*>(row + ((c ^ (rr & 7)) << 4)) =
                 make_uint4(__float_as_uint(part[4 * c]), __float_as_uint(part[4 * c + 1]),
                            __float_as_uint(part[4 * c + 2]), __float_as_uint(part[4 * c + 3]));
           fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0)
+            bulk_copy_to_peer(recv_peer + slot * kRecvBytes + warp * 4096, sSend + slot * kRecvBytes + warp * 4096,
+                              4096, rfull_peer + slot * 8);
         }
-        named_sync(1, kM);
-        if (sent && tid == 0) bulk_copy_to_peer(recv_peer + slot * kRecvBytes, sbuf, kRecvBytes, rfull_peer + slot * 8);
         return sent;
       };
       {  // this thread's head row of the tensor-memory Q blocks (bf16 pairs, low half first)
