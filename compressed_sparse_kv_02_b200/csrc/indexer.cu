@@ -43,6 +43,7 @@ constexpr int kSelThreads = 1024;
 constexpr int kSliceCap = 32768;   // scores per CTA of the selection kernel
 constexpr int kMaxCluster = 16;   // CTAs per query in the selection kernel (above 8: non-portable)
 constexpr int kHistBins = 2048;   // bins of the score-key histogram the TMA scan leaves for the selection
+constexpr int kGroupScanMinQueries = 256;  // from this many queries per call the grouped scan is used
 
 __device__ __forceinline__ int64_t query_visible(const IndexParams& p, int b) {
   const int64_t t = p.q_pos[b];
@@ -556,6 +557,245 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------- grouped TMA scan
+// For calls with many queries (a prefill chunk): consecutive queries of one
+// sequence form groups of GQ = 32 / HI (8 queries of 4 indexer heads, or 4 of
+// 8), and every 64-key unit is scored against the whole group at once, the
+// group's queries x heads filling the mma's N = 32. Keys are read once per
+// group instead of once per query. A group starts at every GQ-th query and
+// wherever the sequence changes, so it never mixes sequences. The scores are
+// the same as the per-query scan's; the digit histogram is left to the select.
+template <int NCH, int HI>
+__global__ void __launch_bounds__(kTmaThreads, 1)
+    index_scan_group_kernel(const __grid_constant__ CUtensorMap tmap, IndexParams p) {
+  using Sh = TmaScanShape<NCH>;
+  constexpr int NSTAGE = Sh::NSTAGE;
+  constexpr int NGROUP = kTmaConsumerWarps / 4;
+  constexpr int GQ = 32 / HI;  // queries per group
+  constexpr int NTH = 4;       // n-tiles of 8 columns: GQ x HI = 32
+  static_assert(HI == 4 || HI == 8, "group shapes");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(tiles + kTmaRingBytes);
+  uint64_t* empty = full + NSTAGE;
+  int* s_valid = reinterpret_cast<int*>(empty + NSTAGE);
+  int* e_start = s_valid + NSTAGE;   // [n_q + 1] first query of each group
+  int* e_pref = e_start + p.n_q + 1;  // [n_q + 1] 64-key units before each group
+  __shared__ int s_wsum[32];
+  __shared__ int s_nent;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  grid_dependency_wait();
+  grid_dependents_launch();
+  {  // group starts
+    int run = 0;
+    for (int base = 0; base < p.n_q; base += kTmaThreads) {
+      const int b = base + tid;
+      int f = 0;
+      if (b < p.n_q) f = (b % GQ == 0) || p.q_seq[b] != p.q_seq[b - 1];
+      int tot;
+      const int ex = block_exclusive_scan<kTmaThreads>(f, s_wsum, tot);
+      if (f) e_start[run + ex] = b;
+      run += tot;
+    }
+    if (tid == 0) {
+      e_start[run] = p.n_q;
+      s_nent = run;
+    }
+    __syncthreads();
+  }
+  const int n_ent = s_nent;
+  {  // units per group: the most visible entries of its queries
+    int run = 0;
+    for (int base = 0; base < n_ent; base += kTmaThreads) {
+      const int e = base + tid;
+      int u = 0;
+      if (e < n_ent) {
+        int64_t nv = 0;
+        for (int b = e_start[e]; b < e_start[e + 1]; ++b) {
+          const int64_t v = query_visible(p, b);
+          nv = v > nv ? v : nv;
+        }
+        u = static_cast<int>((nv + kUnitKeys - 1) / kUnitKeys);
+      }
+      int tot;
+      const int ex = block_exclusive_scan<kTmaThreads>(u, s_wsum, tot);
+      if (e < n_ent) e_pref[e] = run + ex;
+      run += tot;
+    }
+    if (tid == 0) e_pref[n_ent] = run;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 4);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (blockIdx.x == 0)
+    for (int b = tid; b < p.n_q; b += kTmaThreads)
+      if (query_visible(p, b) < 0) report(p.status, CSKV_ERR_INVALID_ARG);
+
+  const int64_t total = e_pref[n_ent];
+  const int64_t u_begin = total * blockIdx.x / gridDim.x;
+  const int64_t n_units = total * (blockIdx.x + 1) / gridDim.x - u_begin;
+  auto locate = [&](int64_t u, int& e, int64_t& j0) {
+    int lo = 0, hi = n_ent - 1;  // last e with e_pref[e] <= u
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (e_pref[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    e = lo;
+    j0 = (u - e_pref[lo]) * kUnitKeys;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (as in the per-query scan)
+    if (lane == 0) prefetch_tensormap(&tmap);
+    int64_t issued = 0;
+    bool ok = true;
+    for (int64_t i0 = 0; i0 < n_units && ok; i0 += 32) {
+      int row0 = -1;
+      if (i0 + lane < n_units) {
+        int e;
+        int64_t j0;
+        locate(u_begin + i0 + lane, e, j0);
+        const int seq = p.q_seq[e_start[e]];
+        const int64_t pi = j0 / p.page_size;
+        int32_t page = -1;
+        if (seq >= 0 && seq < p.n_seqs_layer && pi < p.max_pages_per_seq)
+          page = p.page_table[(int64_t)seq * p.max_pages_per_seq + pi];
+        if (page >= 0 && page < p.n_pages) row0 = static_cast<int>((int64_t)page * p.page_size + (j0 % p.page_size));
+      }
+      const int nb = static_cast<int>(n_units - i0 < 32 ? n_units - i0 : 32);
+      for (int k = 0; k < nb; ++k) {
+        const int r0 = __shfl_sync(kFull, row0, k);
+        if (lane == 0) {
+          const int64_t i = i0 + k;
+          const int s = static_cast<int>(i % NSTAGE);
+          const uint32_t round = static_cast<uint32_t>(i / NSTAGE);
+          if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, p.status)) {
+            ok = false;
+          } else {
+            if (r0 >= 0) {
+              s_valid[s] = 1;
+              mbar_arrive_expect_tx(&full[s], Sh::STAGE_BYTES);
+#pragma unroll
+              for (int box = 0; box < Sh::ROWB / 128; ++box)
+                tma_load_2d(tiles + (size_t)s * Sh::STAGE_BYTES + box * (kUnitKeys * 128), &tmap, box * 64, r0,
+                            &full[s]);
+            } else {
+              report(p.status, CSKV_ERR_OUT_OF_RANGE);
+              s_valid[s] = 0;
+              mbar_arrive(&full[s]);
+            }
+            issued = i + 1;
+          }
+        }
+        ok = __shfl_sync(kFull, ok, 0);
+        if (!ok) break;
+      }
+    }
+    if (lane == 0)
+      for (int64_t r = issued > NSTAGE ? issued - NSTAGE : 0; r < issued; ++r)
+        mbar_wait(&full[r % NSTAGE], static_cast<uint32_t>((r / NSTAGE) & 1), p.status);
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int cw = warp - 1, group = cw >> 2, sub = cw & 3;
+  const int g = lane >> 2, c = lane & 3;
+  const int pg = (g >> 1) + 4 * (g & 1);  // physical row of fragment row g within its 8-row half
+  uint4 qf[NTH][NCH];
+  float wv[NTH][2];
+  // visible entries of the query whose scores this lane writes in n-tile nt (0 past the group's
+  // end; < 2^31 by the host checks)
+  int nvw[NTH];
+  int cur_e = -1, gs = 0;
+  for (int64_t i = group; i < n_units; i += NGROUP) {
+    const int s = static_cast<int>(i % NSTAGE);
+    const uint32_t round = static_cast<uint32_t>(i / NSTAGE);
+    if (!mbar_wait(&full[s], round & 1u, p.status)) break;
+    int e;
+    int64_t j0;
+    locate(u_begin + i, e, j0);
+    if (e != cur_e) {
+      cur_e = e;
+      gs = e_start[e];
+      const int gn = e_start[e + 1] - gs;
+#pragma unroll
+      for (int nt = 0; nt < NTH; ++nt) {
+        const int m = HI == 8 ? nt : 2 * nt + (c >> 1);
+        const int64_t v = m < gn ? query_visible(p, gs + m) : 0;
+        nvw[nt] = v > 0 ? static_cast<int>(v) : 0;
+      }
+#pragma unroll
+      for (int nt = 0; nt < NTH; ++nt) {
+        const int n = 8 * nt + g;  // this lane's B column
+        const int m = n / HI, h = n % HI;
+        const uint16_t* qr = static_cast<const uint16_t*>(p.q_idx) + ((int64_t)(gs + m) * p.n_heads_idx + h) * p.d_idx;
+#pragma unroll
+        for (int jj = 0; jj < NCH; ++jj)
+          qf[nt][jj] = m < gn ? ldg16(qr + (c + 4 * jj) * 8) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int ee = 0; ee < 2; ++ee) {
+          const int n2 = 8 * nt + 2 * c + ee;
+          const int m2 = n2 / HI, h2 = n2 % HI;
+          wv[nt][ee] = m2 < gn ? p.w[(int64_t)(gs + m2) * p.n_heads_idx + h2] : 0.f;
+        }
+      }
+    }
+    const int64_t j = j0 + 16 * sub;  // this warp's 16 keys
+    float acc[NTH][4];  // one accumulation chain (the four n-tiles already interleave)
+#pragma unroll
+    for (int nt = 0; nt < NTH; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+    const bool valid = s_valid[s] != 0;
+    if (valid) {
+      const uint8_t* tb = tiles + (size_t)s * Sh::STAGE_BYTES;
+      const int r0 = 16 * sub + pg;  // rows r0 and r0 + 8 (same swizzle phase)
+#pragma unroll
+      for (int jj = 0; jj < NCH; ++jj) {
+        const int q = c + 4 * jj;
+        const int off = (q >> 3) * (kUnitKeys * 128) + (((q & 7) ^ pg) << 4);
+        const uint4 ka = lds16(tb + off + r0 * 128);
+        const uint4 kb = lds16(tb + off + (r0 + 8) * 128);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t a[4] = {u4_at(ka, 2 * h), u4_at(kb, 2 * h), u4_at(ka, 2 * h + 1), u4_at(kb, 2 * h + 1)};
+#pragma unroll
+          for (int nt = 0; nt < NTH; ++nt) mma_bf16(acc[nt], a, u4_at(qf[nt][jj], 2 * h), u4_at(qf[nt][jj], 2 * h + 1));
+        }
+      }
+    }
+    // per n-tile: rows (keys) j + pg and j + pg + 8, columns 2c, 2c+1 of the tile
+#pragma unroll
+    for (int nt = 0; nt < NTH; ++nt) {
+      float s0 = -INFINITY, s1 = -INFINITY;
+      if (valid) {
+        s0 = wv[nt][0] * fmaxf(acc[nt][0], 0.f) + wv[nt][1] * fmaxf(acc[nt][1], 0.f);
+        s1 = wv[nt][0] * fmaxf(acc[nt][2], 0.f) + wv[nt][1] * fmaxf(acc[nt][3], 0.f);
+        // a query's heads are HI consecutive columns: 2 lanes (HI = 4) or 4 lanes (HI = 8)
+        s0 += __shfl_xor_sync(kFull, s0, 1);
+        s1 += __shfl_xor_sync(kFull, s1, 1);
+        if (HI == 8) {
+          s0 += __shfl_xor_sync(kFull, s0, 2);
+          s1 += __shfl_xor_sync(kFull, s1, 2);
+        }
+      }
+      const bool writer = HI == 8 ? c == 0 : (c & 1) == 0;
+      const int m = HI == 8 ? nt : 2 * nt + (c >> 1);
+      if (writer) {
+        const int64_t nv = nvw[nt];
+        float* out = p.scores + (int64_t)(gs + m) * p.vis_stride;
+        if (j + pg < nv) out[j + pg] = s0;
+        if (j + pg + 8 < nv) out[j + pg + 8] = s1;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+}
+
 // ---------------------------------------------------------------- top-k
 // Radix select on 32-bit order-preserving keys with three digits:
 // A = bits 31..21 (2048 bins), B = bits 20..10 (2048 bins), C = bits 9..0
@@ -1010,6 +1250,27 @@ cudaError_t launch_scan_tma(IndexParams& p, int n_sm, cudaStream_t st) {
   return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(kTmaThreads), smem, st, map, p);
 }
 
+template <int NCH, int HI>
+cudaError_t launch_scan_group(IndexParams& p, int n_sm, cudaStream_t st) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.d_idx), static_cast<cuuint64_t>(p.n_pages) * p.page_size};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.d_idx) * 2};
+  const cuuint32_t box[2] = {64, kUnitKeys};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p.idx_pool), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  auto kern = index_scan_group_kernel<NCH, HI>;
+  const size_t smem = 1024 + (size_t)kTmaRingBytes + 2 * TmaScanShape<NCH>::NSTAGE * sizeof(uint64_t) +
+                      TmaScanShape<NCH>::NSTAGE * sizeof(int) + 2 * sizeof(int) * (size_t)(p.n_q + 1);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(static_cast<unsigned>(n_sm)), dim3(kTmaThreads), smem, st, map, p);
+}
+
 }  // namespace
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link)
@@ -1043,7 +1304,15 @@ cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st) {
   const bool tma_ok = !fp4 && p.page_size % kUnitKeys == 0 && (p.d_idx == 64 || p.d_idx == 128) && nth <= 2 &&
                       (reinterpret_cast<uintptr_t>(p.idx_pool) & 15u) == 0 &&
                       (int64_t)p.n_pages * p.page_size < (int64_t(1) << 31);
-  if (nv_max > 0 && tma_ok) {
+  // many queries in one call (a prefill chunk): the grouped scan reads each key once per group
+  const bool grouped = tma_ok && p.n_q >= kGroupScanMinQueries && (p.n_heads_idx == 4 || p.n_heads_idx == 8);
+  if (nv_max > 0 && grouped) {
+    if (p.d_idx == 64 && p.n_heads_idx == 4) e = launch_scan_group<2, 4>(p, n_sm, st);
+    else if (p.d_idx == 64) e = launch_scan_group<2, 8>(p, n_sm, st);
+    else if (p.n_heads_idx == 4) e = launch_scan_group<4, 4>(p, n_sm, st);
+    else e = launch_scan_group<4, 8>(p, n_sm, st);
+    if (e != cudaSuccess) return e;
+  } else if (nv_max > 0 && tma_ok) {
     p.hist = reinterpret_cast<uint32_t*>(p.scores + (size_t)p.n_q * p.vis_stride);
     e = cudaMemsetAsync(p.hist, 0, sizeof(uint32_t) * kHistBins * (size_t)p.n_q, st);
     if (e != cudaSuccess) return e;

@@ -156,3 +156,45 @@ def test_workspace_too_small_is_rejected(ck):
     with pytest.raises(ck.CskvError) as e:
         ck.csa_index_score_topk(L, seq, pos, positions[0], q_idx, w, k, out_idx, out_cnt, workspace=ws)
     assert e.value.code == ck.ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("hi,di", [(4, 64), (8, 128)])
+def test_many_queries_grouped_scan(ck, orc, hi, di):
+    # 300 queries (the grouped scan: consecutive queries of one sequence share key tiles) from three
+    # sequences in runs of uneven length, at positions that vary inside a run: groups must split where
+    # the sequence changes and mask each query to its own visible entries
+    k = 128
+    g = torch.Generator().manual_seed(77 + hi)
+    n_seq, n_e = 3, 3000
+    L = make_layer(ck.LAYER_CSA, 4, 128, 128, n_seq, n_e, d_idx=di, seed=hi)
+    for s in range(n_seq):
+        L.write_entries(s, 0, idx=torch.randn(n_e, di, generator=g).to(torch.bfloat16).cuda())
+    runs = [(0, 37), (1, 101), (2, 5), (0, 90), (2, 67)]
+    seqs, positions = [], []
+    for s, n in runs:
+        base = int(torch.randint(200, 4 * n_e - 200, (1,), generator=g))
+        for i in range(n):
+            seqs.append(s)
+            positions.append(min(4 * n_e + 127 - 1, base + 3 * i))
+    B = len(seqs)
+    assert B >= 256
+    q_idx = torch.randn(B, hi, di, generator=g).to(torch.bfloat16).cuda()
+    w = torch.rand(B, hi, generator=g).cuda()
+    seq = torch.tensor(seqs, dtype=torch.int32, device="cuda")
+    pos = torch.tensor(positions, dtype=torch.int64, device="cuda")
+    out_idx = torch.full((B, k), -7, dtype=torch.int32, device="cuda")
+    out_cnt = torch.full((B,), -7, dtype=torch.int32, device="cuda")
+    out_sc = torch.zeros(B, k, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ck.csa_index_score_topk(L, seq, pos, max(positions), q_idx, w, k, out_idx, out_cnt, out_sc, status=status)
+    torch.cuda.synchronize()
+    assert ck.cskv_get_status(status) == ck.OK
+    idx, cnt, scs = out_idx.cpu().numpy(), out_cnt.cpu().numpy(), out_sc.cpu().numpy()
+    ents = [layer_entries(L, s, orc.visible_entries(4 * n_e + 127, 4, 128))["idx"] for s in range(n_seq)]
+    for b in range(0, B, 7):
+        t, s = positions[b], seqs[b]
+        nv = orc.visible_entries(t, 4, 128)
+        sc = orc.index_scores(stored_bf16(q_idx[b]), w[b].cpu().double().numpy(), ents[s].rows_subset(0, nv), nv)
+        check_topk(idx[b], int(cnt[b]), sc, k)
+        chosen = idx[b][:int(cnt[b])]
+        assert np.allclose(scs[b][:len(chosen)], sc[chosen], rtol=1e-3, atol=1e-3 * max(1.0, np.abs(sc).max()))
