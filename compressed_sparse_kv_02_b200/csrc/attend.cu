@@ -531,6 +531,7 @@ cudaError_t launch_attend(AttendParams& p, void* ws, int n_sm, cudaStream_t st) 
   p.part_o = static_cast<float*>(ws);
   p.part_lse = p.part_o + rows * p.d_v;
   if (p.n_q == 0) return cudaSuccess;
+  if (attend_pair_supported(p, n_sm)) return launch_attend_pair(p, n_sm, st);
   if (tc) return launch_attend_tc(p, n_sm, st);
   const Plan pl = plan_for(p.d_qk, p.d_v, p.n_heads);
   const bool fp8 = p.kv_dtype == CSKV_FP8_E4M3;

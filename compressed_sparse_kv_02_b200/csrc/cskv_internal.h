@@ -140,5 +140,9 @@ cudaError_t launch_attend_merge(AttendParams& p, cudaStream_t st);
 bool attend_tc_supported(int d_qk, int d_v, int n_heads, int kv_dtype, int n_q);
 void attend_tc_plan(AttendParams& p, int n_sm);
 cudaError_t launch_attend_tc(AttendParams& p, int n_sm, cudaStream_t st);
+// tensor-core attention for calls with many queries on the 128-wide latent with 64 heads:
+// query pairs, whole key lists, bf16 output written directly
+bool attend_pair_supported(const AttendParams& p, int n_sm);
+cudaError_t launch_attend_pair(AttendParams& p, int n_sm, cudaStream_t st);
 
 }  // namespace cskv

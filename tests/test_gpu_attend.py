@@ -23,8 +23,9 @@ def ck(cskv_built):
     return ck
 
 
-def _fill(ck, L, B, n_e, g, sharp, fp8=False):
-    std = 1.0 if sharp else 1.0 / math.sqrt(L.d_qk)
+def _fill(ck, L, B, n_e, g, sharp, fp8=False, std=None):
+    if std is None:
+        std = 1.0 if sharp else 1.0 / math.sqrt(L.d_qk)
     for b in range(B):
         e = torch.randn(n_e, L.d_qk, generator=g) * std
         if fp8:
@@ -171,3 +172,91 @@ def test_invalid_selection_is_reported(ck, orc):
     keys = np.vstack([orc.decode(win), orc.decode(ent)[[0, 3]]])
     o, _ = orc.attend(stored_bf16(q[0]), orc.f64(keys), d, 1.0 / math.sqrt(d))
     assert_close(out[0].float().cpu().numpy(), o, ATOL_BF16, REL_BF16, "masked")
+
+
+def _many(ck, orc, kind, n_q, n_seq, max_t, k=512, seed=0, sharp=False, short_every=0, bad_query=None):
+    """n_q queries (64 heads, d = 128) over n_seq sequences: enough queries for the query-pair
+    tensor-core kernel (it takes calls with at least four queries per SM). Positions are random
+    with the edge cases first; q_seq cycles through the sequences; a sample is checked.
+
+    The sharp variant draws keys with std 0.4 and q x sqrt(d): logits of std ~4.5 (a peaked
+    softmax), outputs below 2 in magnitude. Above 2.56 half a bf16 step of the output alone
+    exceeds the 1e-2 bound, and with unit-variance values 8,192 outputs per query x 24 sampled
+    queries reach 4.5 sigma."""
+    d, H = 128, 64
+    m = 4 if kind == "csa" else 128
+    n_e = max_t // m + 2
+    L = make_layer(ck.LAYER_CSA if kind == "csa" else ck.LAYER_HCA, m, d, d, n_seq, n_e,
+                   d_idx=64 if kind == "csa" else 0, seed=seed)
+    g = torch.Generator().manual_seed(3000 + seed)
+    _fill(ck, L, n_seq, n_e, g, sharp, std=0.4 if sharp else None)
+    rng = np.random.default_rng(seed)
+    pos = rng.integers(0, max_t + 1, n_q)
+    pos[:6] = [0, 5, 126, 127, 128, 131]
+    pos[-1] = max_t
+    if bad_query is not None:
+        pos[bad_query] = max_t - 2
+    qseq = np.arange(n_q) % n_seq
+    q = (torch.randn(n_q, H, d, generator=g) * (math.sqrt(d) if sharp else 1.0)).to(torch.bfloat16).cuda()
+    out = torch.zeros(n_q, H, d, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(n_q, H, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    seq_t = torch.from_numpy(qseq.astype(np.int32)).cuda()
+    pos_t = torch.from_numpy(pos.astype(np.int64)).cuda()
+    sel = cnt = None
+    if kind == "csa":
+        sel = np.full((n_q, k), -1, np.int32)
+        cnt = np.zeros(n_q, np.int32)
+        for i, t in enumerate(pos):
+            nv = orc.visible_entries(int(t), m, 128)
+            c = min(k, nv)
+            if short_every and i % short_every == 1:
+                c = min(c, 37)
+            if c:
+                sel[i, :c] = np.sort(rng.choice(nv, c, replace=False))
+            cnt[i] = c
+        if bad_query is not None:  # one index past the visible entries: reported and masked
+            i = bad_query
+            nv = orc.visible_entries(int(pos[i]), m, 128)
+            sel[i, 1] = nv + 3
+        ck.csa_attend(L, seq_t, pos_t, int(max_t), q, torch.from_numpy(sel).cuda(), torch.from_numpy(cnt).cuda(),
+                      out, lse, status=status)
+    else:
+        ck.hca_attend(L, seq_t, pos_t, int(max_t), q, out, lse, status=status)
+    want = ck.ERR_OUT_OF_RANGE if bad_query is not None else ck.OK
+    assert ck.cskv_get_status(status) == want
+    scale = 1.0 / math.sqrt(d)
+    got_o = out.float().cpu().numpy()
+    got_l = lse.cpu().numpy()
+    sample = sorted(set(list(range(6)) + [n_q // 2, n_q // 2 + 1, n_q - 2, n_q - 1] +
+                        list(rng.choice(n_q, 14, replace=False)) + ([bad_query] if bad_query is not None else [])))
+    for i in sample:
+        t, b = int(pos[i]), int(qseq[i])
+        nv = orc.visible_entries(t, m, 128)
+        win = ring_window(L, b, t)
+        ent = layer_entries(L, b, max(nv, 1))["kv"]
+        qb = stored_bf16(q[i])
+        if kind == "csa":
+            ids = sel[i, :cnt[i]]
+            ids = ids[(ids >= 0) & (ids < nv)]
+            keys = np.vstack([orc.decode(win), orc.decode(ent)[ids]]) if len(ids) else orc.decode(win)
+            o, l = orc.attend(qb, orc.f64(keys), d, scale)
+        else:
+            o, l = orc.hca_query(t, m, 128, qb, win, ent if nv else ent.rows_subset(0, 0), d, scale)
+        assert_close(got_o[i], o, ATOL_BF16, REL_BF16, "%s many i=%d t=%d" % (kind, i, t))
+        assert np.allclose(got_l[i], l, rtol=0, atol=2e-3), "lse i=%d" % i
+
+
+def test_many_queries_csa(ck, orc):
+    # 601 queries (the last pair holds one), top-512 with some short selections: 1-5 key tiles
+    _many(ck, orc, "csa", 601, 3, 127 + 4 * 5000, k=512, seed=21, short_every=7)
+
+
+def test_many_queries_hca(ck, orc):
+    # up to 727 keys (6 tiles) per query; peaked softmax (the lazy O rescale)
+    _many(ck, orc, "hca", 601, 3, 128 * 600, seed=22)
+    _many(ck, orc, "hca", 640, 2, 128 * 200 + 17, seed=23, sharp=True)
+
+
+def test_many_queries_invalid_index_is_masked(ck, orc):
+    _many(ck, orc, "csa", 600, 2, 127 + 4 * 800, k=128, seed=24, bad_query=301)
