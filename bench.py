@@ -292,6 +292,27 @@ def run_prefill(args, rank, world):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev, world)
     n_blocks = -(-PREFILL_CHUNK // model.q_block)
+
+    # one more pass, untimed, with events around every call: where the pass's time goes
+    from compressed_sparse_kv_02_b200 import _binding as Bn
+    st_h = Bn._stream(stream)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in model._calls]
+    with torch.cuda.stream(stream):
+        for c, (a, b) in zip(model._calls, ev):
+            a.record(stream)
+            c(st_h)
+            b.record(stream)
+    torch.cuda.synchronize()
+    op_ms = {}
+    for c, (a, b) in zip(model._calls, ev):
+        op_ms[c.where] = op_ms.get(c.where, 0.0) + a.elapsed_time(b)
+    attn_ms = op_ms.get("csa_attend", 0.0) + op_ms.get("hca_attend", 0.0)
+    # launches per pass: 4 ring appends + 2 chunk compressions, and per query block the indexer's scan and
+    # selection plus one launch per attention call (the query-pair kernel takes calls of at least four
+    # queries per SM on the 128-wide latent with 64 heads; the split kernel adds a merge launch)
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    pair = cfg.heads == 64 and cfg.d_qk == 128 and cfg.d_v == 128 and model.q_block >= 4 * n_sm
+    per_block = 2 + (2 if pair else 4)
     out = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -329,7 +350,10 @@ def run_prefill(args, rank, world):
         },
         "e2e": {"value": round(whole_job_rate(PREFILL_CHUNK, world, e2e_ms), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": (6 + 6 * n_blocks) * args.steps,
+        "gpu_launches": (6 + per_block * n_blocks) * args.steps,
+        "op_ms_untimed_breakdown": {k_: round(v_, 3) for k_, v_ in op_ms.items()},
+        "attention_tflops_untimed": round((fl["csa_attend"] + fl["hca_attend"]) / (attn_ms * 1e-3) / 1e12, 1)
+        if attn_ms > 0 else None,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = prefill_cpu_baseline(model, cfg, budget_s=args.cpu_budget)

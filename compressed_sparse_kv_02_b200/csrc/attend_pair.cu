@@ -13,20 +13,21 @@
 // second query's tile sits at lane offset 16, so the two queries' S (and O)
 // share the 128 lanes and one softmax warpgroup serves both: thread (warp w,
 // lane l) owns head 16 w + (l & 15) of query l >> 4.
-//   loaders (warps 5-8): per tile, the source rows of 128 keys of each query,
-//     then cp.async of the 2 x 128 rows (16 threads per 256-byte row) into a
-//     128-byte-swizzled stage; Q of the pair by TMA;
-//   MMA (warp 4, one thread): S(t) = Q K^T (2 x 8 MMAs, M = 64, N = 128, K = 16)
-//     into S buffer t & 1; then O += P(t - 1) V (2 x 8 MMAs, N = d_v = 128, V read
+//   loaders (warps 5-8): per tile, the source rows of 64 keys of each query,
+//     then cp.async of the 2 x 64 rows (16 threads per 256-byte row) into a
+//     128-byte-swizzled stage (four stages: the loaders run up to three tiles
+//     ahead, so the hand-offs of consecutive tiles overlap); Q of the pair by TMA;
+//   MMA (warp 4, one thread): S(t) = Q K^T (2 x 8 MMAs, M = 64, N = 64, K = 16)
+//     into S buffer t & 1; then O += P(t - 1) V (2 x 4 MMAs, N = d_v = 128, V read
 //     MN-major from the same stage: V is the first d_v channels of each key);
 //   softmax (warps 0-3): max pass over S(t) in tensor memory, lazy O rescale,
 //     exp pass writing bf16 P(t) into shared buffer t & 1 (the A operand).
 // O is rescaled only when a row's running max rises by more than 2^8, so most
 // tiles skip it (the probabilities stay below 256 in bf16).
 //
-// Shared memory (1024-aligned): Q 32 KB | key stages 2 x 64 KB | P 2 x 32 KB |
-// source-row codes 1 KB | barriers | valid-key bits. Tensor memory: O 128 |
-// S 2 x 128 columns. A key without a valid source row (an index outside the
+// Shared memory (1024-aligned): Q 32 KB | key stages 4 x 32 KB | P 2 x 16 KB |
+// source-row codes | barriers | valid-key bits. Tensor memory: O 128 | S 2 x 64
+// columns. A key without a valid source row (an index outside the
 // visible entries) is masked out of the softmax and reported.
 #include "cskv_device.cuh"
 #include "cskv_internal.h"
@@ -36,19 +37,20 @@ namespace {
 
 constexpr int kD = 128;             // d_qk = d_v
 constexpr int kH = 64;              // heads of one query (the M of its tile)
-constexpr int kNk = 128;            // keys per tile and query
-constexpr int kNS = 2;              // key stages
-constexpr int kSlotBytes = kNk * kD * 2;        // 32768: one query's key tile (two 64-channel halves)
-constexpr int kHalfBytes = kNk * 128;           // 16384: one 64-channel half of it
-constexpr int kStageBytes = 2 * kSlotBytes;     // 65536
+constexpr int kNk = 64;             // keys per tile and query
+constexpr int kNS = 4;              // key stages: the loaders run up to three tiles ahead
+constexpr int kSlotBytes = kNk * kD * 2;        // 16384: one query's key tile (two 64-channel halves)
+constexpr int kHalfBytes = kNk * 128;           // 8192: one 64-channel half of it
+constexpr int kStageBytes = 2 * kSlotBytes;     // 32768
 constexpr int kQBytes = 2 * kH * kD * 2;        // 32768: Q of both queries
-constexpr int kPBytes = 2 * kH * kNk * 2;       // 32768: P of both queries (one buffer)
+constexpr int kPBytes = 2 * kH * kNk * 2;       // 16384: P of both queries (one buffer)
+constexpr int kRows = 2 * kNk;                  // key rows of a tile (both queries)
 constexpr int kThreads = 288;       // warps 0-3 softmax, warp 4 MMA, warps 5-8 loads
 constexpr int kMmaThread = 128;
 constexpr int kLoadThread0 = 160;
 constexpr int kLoaders = kThreads - kLoadThread0;  // 128
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0, kColS = 128;       // O | S buffer 0 | S buffer 1
+constexpr uint32_t kColO = 0, kColS = 128;       // O | S buffer 0 | S buffer 1 (64 columns each)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;        // log2 units
@@ -57,12 +59,12 @@ struct Smem {
   static constexpr int Q = 0;
   static constexpr int K = Q + kQBytes;
   static constexpr int P = K + kNS * kStageBytes;
-  static constexpr int ROWS = P + 2 * kPBytes;    // 256 source-row codes of the tile being issued
-  static constexpr int BAR = ROWS + 256 * 4;
-  static constexpr int TMEM = BAR + 13 * 8;
+  static constexpr int ROWS = P + 2 * kPBytes;    // source-row codes of the tile being issued
+  static constexpr int BAR = ROWS + kRows * 4;
+  static constexpr int TMEM = BAR + (2 * kNS + 9) * 8;
   static constexpr int FLAGS = TMEM + 4;
-  static constexpr int MASK = FLAGS + 8;          // valid-key bits: [stage][query][4 words]
-  static constexpr int END = MASK + kNS * 2 * 4 * 4;
+  static constexpr int MASK = FLAGS + 8;          // valid-key bits: [stage][query][2 words]
+  static constexpr int END = MASK + kNS * 2 * 2 * 4;
   static constexpr size_t bytes() { return 1024 + END; }
 };
 static_assert(Smem::bytes() <= 232448, "shared memory budget");
@@ -130,7 +132,7 @@ __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
 }
 
-// S of one query: 8 MMAs (K = 16 channels each) over the two 64-channel halves
+// S of one query: 8 MMAs (K = 16 channels each) over the two 64-channel halves (N = 64 keys)
 __device__ __forceinline__ void issue_s(uint32_t d, uint32_t q, uint32_t k, uint32_t idesc) {
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks) {
@@ -139,18 +141,18 @@ __device__ __forceinline__ void issue_s(uint32_t d, uint32_t q, uint32_t k, uint
             umma_desc_sw128(k + (ks >> 2) * kHalfBytes + off, 16, 1024), idesc, ks > 0 ? 1u : 0u);
   }
 }
-// O += P V of one query: 8 MMAs (K = 16 keys each); V MN-major (its two 64-channel halves
-// kHalfBytes apart, 8-key groups 1024 bytes apart)
+// O += P V of one query: 4 MMAs (K = 16 keys each; P is one 64-key swizzle atom); V MN-major
+// (its two 64-channel halves kHalfBytes apart, 8-key groups 1024 bytes apart)
 __device__ __forceinline__ void issue_pv(uint32_t d, uint32_t pm, uint32_t v, uint32_t idesc, bool acc) {
 #pragma unroll
-  for (int ks = 0; ks < 8; ++ks)
-    umma_ss(d, umma_desc_sw128(pm + (ks >> 2) * (kH * 128) + (ks & 3) * 32, 16, 1024),
+  for (int ks = 0; ks < 4; ++ks)
+    umma_ss(d, umma_desc_sw128(pm + ks * 32, 16, 1024),
             umma_desc_sw128(v + ks * 16 * 128, kHalfBytes, 1024), idesc, (acc || ks > 0) ? 1u : 0u);
 }
 
-// Pipeline (tiles numbered gt across the CTA's items; stage gt % 2, S buffer gt & 1,
+// Pipeline (tiles numbered gt across the CTA's items; stage gt % 4, S buffer gt & 1,
 // P buffer gt & 1):
-//   loaders : wait kempty[stage] (P V of tile gt - 2 done) -> cp.async -> kfull[stage]
+//   loaders : wait kempty[stage] (P V of tile gt - 4 done) -> cp.async -> kfull[stage]
 //   MMA     : wait kfull -> S(gt) -> commit sfull[gt & 1] (and qempty after an item's last S);
 //             wait pfull[(gt - 1) & 1] -> P V(gt - 1) -> commit kempty, obar[(gt - 1) & 1]
 //   softmax : wait sfull, kfull (valid-key bits) -> row max -> wait obar (P V of tile gt - 2
@@ -165,14 +167,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sP = sm + Smem::P;
   uint32_t* sRow = reinterpret_cast<uint32_t*>(sm + Smem::ROWS);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Smem::BAR);
-  uint64_t* kfull = bars;           // [2] loaders -> MMA
-  uint64_t* kempty = bars + 2;      // [2] MMA -> loaders (commit after the tile's P V)
-  uint64_t* sfull = bars + 4;       // [2] MMA -> softmax
-  uint64_t* pfull = bars + 6;       // [2] softmax -> MMA (128 arrivals)
-  uint64_t* obar = bars + 8;        // [2] MMA -> softmax (P V of that P buffer done)
-  uint64_t* qfull = bars + 10;      //     Q of the item landed (TMA)
-  uint64_t* qempty = bars + 11;     //     the item's S products are done with Q
-  uint64_t* dbar = bars + 12;       //     the item's last P V is done
+  uint64_t* kfull = bars;               // [kNS] loaders -> MMA and softmax
+  uint64_t* kempty = bars + kNS;        // [kNS] MMA -> loaders (commit after the tile's P V)
+  uint64_t* sfull = bars + 2 * kNS;     // [2] MMA -> softmax
+  uint64_t* pfull = sfull + 2;          // [2] softmax -> MMA (128 arrivals)
+  uint64_t* obar = pfull + 2;           // [2] MMA -> softmax (P V of that P buffer done)
+  uint64_t* qfull = obar + 2;           //     Q of the item landed (TMA)
+  uint64_t* qempty = qfull + 1;         //     the item's S products are done with Q
+  uint64_t* dbar = qempty + 1;          //     the item's last P V is done
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + Smem::TMEM);
   volatile int* sAbort = reinterpret_cast<int*>(sm + Smem::FLAGS);
   volatile int* sLdOk = sAbort + 1;
@@ -180,9 +182,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kNS; ++i) {
       mbar_init(&kfull[i], 1);
       mbar_init(&kempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&sfull[i], 1);
       mbar_init(&pfull[i], 128);
       mbar_init(&obar[i], 1);
@@ -244,29 +248,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           *sAbort = 1;
         }
       }
-      // this thread's part of every tile: chunk (lt & 15) of rows (lt >> 4) + 8 q. A tile is
-      // signalled as soon as its copy has landed (two stages leave no room to hold it back); the
-      // next tile's source rows are looked up while the copy is in flight.
+      // this thread's part of every tile: the source row of key (lt & 63) of query lt >> 6, and
+      // chunk (lt & 15) of rows (lt >> 4) + 8 q. A tile is signalled as soon as its copy has
+      // landed; the next tile's source rows are looked up after that, while the loaders wait
+      // for its stage.
       const int chunk = lt & 15, half = chunk >> 3, c8 = chunk & 7;
-      auto codes = [&](int it, uint32_t& c0, uint32_t& c1) {
-        const int u = it * kNk + lt;
-        c0 = 0;
-        c1 = 0;
-        if (u < n0) {
-          c0 = key_code(p, b0, s0, k0, u);
-          if (!c0) report(p.status, CSKV_ERR_OUT_OF_RANGE);
+      const int my_slot = lt >> 6, my_key = lt & (kNk - 1);
+      auto code_of = [&](int it) -> uint32_t {
+        const int u = it * kNk + my_key;
+        uint32_t c = 0;
+        if (u < (my_slot ? n1 : n0)) {
+          c = my_slot ? key_code(p, b1, s1, k1, u) : key_code(p, b0, s0, k0, u);
+          if (!c) report(p.status, CSKV_ERR_OUT_OF_RANGE);
         }
-        if (u < n1) {
-          c1 = key_code(p, b1, s1, k1, u);
-          if (!c1) report(p.status, CSKV_ERR_OUT_OF_RANGE);
-        }
+        return c;
       };
-      uint32_t nc0 = 0, nc1 = 0;
-      if (ntiles > 0) codes(0, nc0, nc1);
+      uint32_t nc = ntiles > 0 ? code_of(0) : 0u;
       for (int it = 0; it < ntiles; ++it) {
         const uint32_t gt = g + it;
         const int st = gt % kNS;
-        const uint32_t c0 = nc0, c1 = nc1;
+        const uint32_t c = nc;
         if (lt == 0)
           *sLdOk = !*sAbort && (gt < (uint32_t)kNS || mbar_wait(&kempty[st], ((gt / kNS) - 1) & 1u, p.status));
         named_sync(3, kLoaders);  // sLdOk is set (and the last tile's issue has read sRow)
@@ -274,32 +275,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           *sAbort = 1;
           break;
         }
-        sRow[lt] = c0;
-        sRow[lt + 128] = c1;
-        {  // valid-key bits of the tile (the softmax reads them after kfull[st])
-          const unsigned m0 = __ballot_sync(kFull, c0 != 0), m1 = __ballot_sync(kFull, c1 != 0);
-          if ((lt & 31) == 0) {
-            sMask[st * 8 + (lt >> 5)] = m0;
-            sMask[st * 8 + 4 + (lt >> 5)] = m1;
-          }
+        sRow[lt] = c;
+        {  // valid-key bits of the tile (the softmax reads them after kfull[st]): warp w of the
+           // loaders holds keys 32 (w & 1) .. + 31 of query w >> 1
+          const unsigned mw = __ballot_sync(kFull, c != 0);
+          if ((lt & 31) == 0) sMask[st * 4 + (lt >> 5)] = mw;
         }
         named_sync(3, kLoaders);
         uint8_t* dst = sK + st * kStageBytes + half * kHalfBytes;
-#pragma unroll 8
-        for (int q = 0; q < 32; ++q) {
-          const int row = (lt >> 4) + 8 * q;  // query q >> 4, key row & 127
-          const int key = row & 127;
+#pragma unroll 4
+        for (int q = 0; q < kRows / 8; ++q) {
+          const int row = (lt >> 4) + 8 * q;  // query row / kNk, key row % kNk
+          const int key = row & (kNk - 1);
           const uint16_t* src = code_row(p, sRow[row]);
-          cp_async16(dst + (q >> 4) * kSlotBytes + key * 128 + ((c8 ^ (key & 7)) << 4),
+          cp_async16(dst + (row / kNk) * kSlotBytes + key * 128 + ((c8 ^ (key & 7)) << 4),
                      src ? static_cast<const void*>(src + half * 64 + c8 * 8) : static_cast<const void*>(p.q),
                      src ? 16 : 0);
         }
         cp_async_commit();
-        if (it + 1 < ntiles) codes(it + 1, nc0, nc1);
         cp_async_wait<0>();
         fence_proxy_async_smem();
         named_sync(3, kLoaders);
         if (lt == 0) mbar_arrive(&kfull[st]);
+        if (it + 1 < ntiles) nc = code_of(it + 1);
       }
     } else if (tid == kMmaThread) {
       // ---------------------------------------------------------------- MMA issue
@@ -362,17 +360,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t* valid = sMask + (gt % kNS) * 8 + slot * 4;
+        const uint32_t* valid = sMask + (gt % kNS) * 4 + slot * 2;
         float mt = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t s[32];
-          tmem_ld32(sb + c * 32, s);
-          const uint32_t vw = valid[c];
+        {  // both 32-key halves of the tile, one wait
+          uint32_t s[32], s2[32];
+          tmem_ld32(sb, s);
+          tmem_ld32(sb + 32, s2);
+          const uint32_t vw = valid[0], vw2 = valid[1];
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
+          for (int j = 0; j < 32; ++j) {
             if ((vw >> j) & 1u) mt = fmaxf(mt, __uint_as_float(s[j]) * sl2);
+            if ((vw2 >> j) & 1u) mt = fmaxf(mt, __uint_as_float(s2[j]) * sl2);
+          }
         }
         float corr = 1.f;
         bool rescale = false;
@@ -411,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint8_t* pbuf = prow + (gt & 1u) * kPBytes;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < kNk / 32; ++c) {
           uint32_t s[32];
           tmem_ld32(sb + c * 32, s);
           const uint32_t vw = valid[c];
@@ -424,11 +424,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             l_run += e0 + e1;
             pp[j] = pack_bf16(e0, e1);
           }
-          // keys 32 c .. 32 c + 31: 64-key atom c >> 1, 16-byte chunks 4 (c & 1) .. + 3
-          uint8_t* dst = pbuf + (c >> 1) * (kH * 128);
+          // keys 32 c .. 32 c + 31: 16-byte chunks 4 c .. 4 c + 3 of the row (one 64-key atom)
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<uint4*>(dst + ((((c & 1) * 4 + i) ^ sw) << 4)) =
+            *reinterpret_cast<uint4*>(pbuf + (((c * 4 + i) ^ sw) << 4)) =
                 make_uint4(pp[4 * i], pp[4 * i + 1], pp[4 * i + 2], pp[4 * i + 3]);
         }
         fence_proxy_async_smem();
