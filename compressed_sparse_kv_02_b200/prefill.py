@@ -174,3 +174,29 @@ class PrefillModel:
             fc += (n_w + min(cfg.k, nv)) * per_key
             fh += (n_w + nv_h) * per_key
         return {"index": fi, "csa_attend": fc, "hca_attend": fh, "total": fi + fc + fh}
+
+
+def main(argv=None) -> int:
+    """Run `passes` prefill passes of one chunk (the benchmark's shapes: 64 heads, d = 128, indexer 4 x 64,
+    top-512) and check the status word; used to profile one block of the prefill on its own."""
+    import argparse
+    ap = argparse.ArgumentParser(description=main.__doc__)
+    ap.add_argument("--cached", type=int, default=65536)
+    ap.add_argument("--chunk", type=int, default=4096)
+    ap.add_argument("--q-block", type=int, default=4096)
+    ap.add_argument("--passes", type=int, default=2)
+    a = ap.parse_args(argv)
+    cfg = synth.Config("prefill_block", 1, a.cached + a.chunk, 64, 128, 128, 4, 64, 512, seed=3)
+    model = PrefillModel(cfg, cached=a.cached, chunk=a.chunk, q_block=a.q_block)
+    model.fill_synthetic()
+    for _ in range(a.passes):
+        model.step()
+    torch.cuda.synchronize()
+    st = model.check_status()
+    print("prefill passes: %d, status %s, device memory %.2f GB"
+          % (a.passes, B.status_string(st), torch.cuda.max_memory_allocated() / 1e9))
+    return 0 if st == B.OK else 1
+
+
+if __name__ == "__main__":
+    raise SystemExit(main())
