@@ -229,6 +229,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int s0 = p.q_seq[b0], s1 = b1 >= 0 ? p.q_seq[b1] : 0;
     const bool ok0 = s0 >= 0 && s0 < p.n_seqs_layer, ok1 = b1 >= 0 && s1 >= 0 && s1 < p.n_seqs_layer;
     const int n0 = ok0 ? k0.n : 0, n1 = ok1 ? k1.n : 0;
+    // a sequence id outside the layer: the query's keys are all masked (zero output), as in the
+    // other attention kernels, and the status word says why
+    if (tid == 0 && ((!ok0 && k0.n > 0) || (b1 >= 0 && !ok1 && k1.n > 0))) report(p.status, CSKV_ERR_OUT_OF_RANGE);
     const int nmax = n0 > n1 ? n0 : n1;
     const int ntiles = (nmax + kNk - 1) / kNk;
 
