@@ -176,16 +176,28 @@ def workload_text(cfg, nq, model):
     return "%s decode: B=%d, t=%d, H=%d, d=%d" % (cfg.name, nq, cfg.ctx - 1, cfg.heads, cfg.d_qk)
 
 
-# DRAM bytes (read + write) of the indexer op per query, from one ncu capture of
-# the scan and select kernels on the Pro workload at batch 2, scaled by queries
-# (profiles/decode_pro_b2_kernels_full.md); None for other workloads or once
-# those kernels change.
-INDEX_OP_DRAM_BYTES_PER_QUERY = {"pro": (134.301440e6 + 4.370944e6 + 2.179840e6) / 2}
+# DRAM bytes (read + write) of the indexer op per query, from one ncu capture of its
+# kernels on a batch-2 run of the workload, scaled by queries. Each figure is tied to
+# the digest of the kernel sources it was captured from; once those sources change
+# the figure no longer describes the build and `traffic` is reported as null.
+INDEX_OP_SOURCES = ("compressed_sparse_kv_02_b200/csrc/indexer.cu", "compressed_sparse_kv_02_b200/csrc/cskv_device.cuh")
+INDEX_OP_DRAM = {}  # workload -> (source digest, DRAM bytes per query)
+
+
+def sources_digest(paths=INDEX_OP_SOURCES):
+    import hashlib
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def index_op_traffic(cfg, nq):
-    per_q = INDEX_OP_DRAM_BYTES_PER_QUERY.get(cfg.name)
-    return None if per_q is None else round(per_q * nq)
+    rec = INDEX_OP_DRAM.get(cfg.name)
+    if rec is None or rec[0] != sources_digest():
+        return None
+    return round(rec[1] * nq)
 
 
 # ----------------------------------------------------------------- ranks
@@ -594,11 +606,22 @@ def run_ours(args, rank, world):
 
 
 # ----------------------------------------------------------------- the oracle on host cores
+def _window_rows(layer, new_x, b, t):
+    """Raw window rows of positions t-n_win+1 .. t in position order, from the synthesised state: the
+    ring slots of positions t-n_win+1 .. t-1 (written by the synthesis, never by a decode step, which only
+    writes the slot of t) and the decode token's own row."""
+    from gpu_helpers import stored_bf16
+    ws = max(0, t - layer.n_win + 1)
+    slots = [p % layer.n_win for p in range(ws, t)]
+    rows = torch.cat([layer.ring_x[b][slots], new_x[b].reshape(1, -1).to(layer.ring_x.dtype)], 0)
+    return stored_bf16(rows)
+
+
 def _oracle_inputs(model, cfg, b):
-    """Host copies (oracle storage views) of sequence b's caches and query, read from the device."""
+    """Host copies (oracle storage views) of sequence b's synthesised caches and query."""
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     import oracle
-    from gpu_helpers import layer_entries, ring_window, stored_bf16, stored_fp4
+    from gpu_helpers import layer_entries, stored_bf16, stored_fp4
     t = model.ctx_lens[b] - 1
     csa, hca = model.layers[0], model.layers[1]
     nv = oracle.visible_entries(t, cfg.m_csa, cfg.n_win)
@@ -607,9 +630,9 @@ def _oracle_inputs(model, cfg, b):
     inp = model.inputs[0]
     qi = (stored_bf16(inp["q_idx"][b]) if cfg.idx_dtype == "bf16" else
           stored_fp4(inp["q_idx"][b], inp["q_idx_scale"][b]))
-    return dict(t=t, win=ring_window(csa, b, t), kv=ent["kv"], ki=ent["idx"], q=stored_bf16(inp["q_csa"][b]),
-                qi=qi, w=inp["w"][b].double().cpu().numpy(),
-                win_h=ring_window(hca, b, t), kv_h=layer_entries(hca, b, nv_h)["kv"],
+    return dict(t=t, win=_window_rows(csa, inp["csa_x"], b, t), kv=ent["kv"], ki=ent["idx"],
+                q=stored_bf16(inp["q_csa"][b]), qi=qi, w=inp["w"][b].double().cpu().numpy(),
+                win_h=_window_rows(hca, inp["hca_x"], b, t), kv_h=layer_entries(hca, b, nv_h)["kv"],
                 q_h=stored_bf16(inp["q_hca"][b]))
 
 
@@ -641,15 +664,15 @@ def cpu_baseline(model, cfg, budget_s=20.0):
 
 
 def run_reference(args, rank, world):
-    """The oracle as the reference arm: K steps, each a bounded sample of the decode workload."""
-    import compressed_sparse_kv_02_b200  # noqa: F401  (the caches are synthesised on the GPU)
-    from compressed_sparse_kv_02_b200 import decode, synth
+    """The oracle as the reference arm: K steps, each a bounded sample of the decode workload. The caches,
+    rings and queries are synthesised on the GPU by torch's generators (no decode step runs: the oracle
+    reads the synthesised state, with the decode token's own row as the newest window row)."""
+    from compressed_sparse_kv_02_b200 import synth
     import oracle
     oracle.build()
     cfg = synth.CONFIGS[args.config]
     model = workload_model(cfg)
     model.fill_synthetic()
-    model.step()
     torch.cuda.synchronize()
     cores = os.cpu_count() or 1
     oracle.set_threads(cores)

@@ -12,5 +12,5 @@ from ._binding import (  # noqa: F401
     csa_compress_kv, hca_compress_kv, cskv_cache_append,
     csa_index_ws_bytes, csa_index_score_topk, csa_index_score_topk_static,
     cskv_attend_ws_bytes, csa_attend, hca_attend,
-    cskv_get_status, cskv_version,
+    cskv_get_status, cskv_selftest_wait, cskv_version,
 )

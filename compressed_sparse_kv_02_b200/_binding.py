@@ -101,6 +101,7 @@ SYMBOLS = {
     "csa_attend": (_I32, [ctypes.POINTER(AttendArgs), _P, ctypes.c_size_t, _P]),
     "hca_attend": (_I32, [ctypes.POINTER(AttendArgs), _P, ctypes.c_size_t, _P]),
     "cskv_get_status": (_I32, [_P, _P, ctypes.POINTER(_I32)]),
+    "cskv_selftest_wait": (_I32, [_I32, ctypes.c_uint32, _P, _P]),
     "cskv_status_string": (ctypes.c_char_p, [_I32]),
     "cskv_version": (_I32, []),
 }
@@ -474,6 +475,14 @@ def cskv_get_status(status: torch.Tensor, stream=None) -> int:
     h = ctypes.c_int32()
     _check(lib().cskv_get_status(_ptr(status), _stream(stream), ctypes.byref(h)), "cskv_get_status")
     return h.value
+
+
+def cskv_selftest_wait(arrive: bool, spin_limit: int, status: torch.Tensor, stream=None):
+    """Launch the library's bounded-wait check: one warp waits on an mbarrier for at most spin_limit
+    polls; with arrive=False nothing arrives and the wait reports CSKV_ERR_TIMEOUT in `status`."""
+    _need(status, "status", torch.int32)
+    _check(lib().cskv_selftest_wait(1 if arrive else 0, int(spin_limit), _ptr(status), _stream(stream)),
+           "cskv_selftest_wait")
 
 
 def cskv_version() -> int:

@@ -349,6 +349,11 @@ cskv_status cskv_get_status(int32_t* d_status, void* stream, int32_t* status) {
   return CSKV_OK;
 }
 
+cskv_status cskv_selftest_wait(int32_t arrive, uint32_t spin_limit, int32_t* d_status, void* stream) {
+  if (!d_status || spin_limit == 0) return CSKV_ERR_INVALID_ARG;
+  return from_cuda(cskv::launch_wait_selftest(arrive != 0, spin_limit, d_status, static_cast<cudaStream_t>(stream)));
+}
+
 const char* cskv_status_string(cskv_status s) {
   switch (s) {
     case CSKV_OK: return "ok";

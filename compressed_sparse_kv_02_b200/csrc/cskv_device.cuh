@@ -170,12 +170,16 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, 
       : "memory");
 }
 
-// Wait for the phase of parity `parity` to complete; false after the spin limit.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
+// Wait for the phase of parity `parity` to complete; false after `limit` polls,
+// with CSKV_ERR_TIMEOUT in the status word.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, int32_t* status, uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   report(status, CSKV_ERR_TIMEOUT);
   return false;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+  return mbar_wait_limit(bar, parity, status, kSpinLimit);
 }
 // 2D tiled TMA load (no multicast) of box {x, y} into shared memory; completes
 // `bytes` of transaction on `bar`.

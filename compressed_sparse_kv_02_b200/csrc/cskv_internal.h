@@ -145,4 +145,7 @@ cudaError_t launch_attend_tc(AttendParams& p, int n_sm, cudaStream_t st);
 bool attend_pair_supported(const AttendParams& p, int n_sm);
 cudaError_t launch_attend_pair(AttendParams& p, int n_sm, cudaStream_t st);
 
+// the bounded-wait check (selftest.cu)
+cudaError_t launch_wait_selftest(int arrive, uint32_t spin_limit, int32_t* status, cudaStream_t st);
+
 }  // namespace cskv

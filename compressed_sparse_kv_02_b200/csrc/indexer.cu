@@ -888,10 +888,10 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
   __shared__ uint32_t s_hA[kBinsA], s_hB[kBinsB], s_hC[kBinsC];
   __shared__ int s_w[32];
   __shared__ uint32_t s_res[3];
-  __shared__ int s_cnt[2];
+  __shared__ int s_cnt[3];
   __shared__ int s_ncand;
   __shared__ __align__(8) uint64_t s_bar;
-  __shared__ int s_peer[2 * kMaxCluster];
+  __shared__ int s_peer[3 * kMaxCluster];
   constexpr int NW = kSelThreads / 32;
   __shared__ int s_wgt[NW], s_weq[NW];
 
@@ -912,12 +912,12 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
   float* osc = p.out_scores ? p.out_scores + (int64_t)b * k : nullptr;
   const int64_t lo = (int64_t)rank * p.slice;
   const int64_t hi = lo + p.slice < nv ? lo + p.slice : nv;
-  const int len = hi > lo ? static_cast<int>(hi - lo) : 0;
+  int len = hi > lo ? static_cast<int>(hi - lo) : 0;
   grid_dependency_wait();  // the scores and the digit-A histogram come from the scan
   grid_dependents_launch();
   __syncthreads();
   // the slice's scores (whole 16-byte pieces) land by one bulk copy while digit A is found
-  const int n4 = nv > k ? len >> 2 : 0;
+  int n4 = nv > k ? len >> 2 : 0;
   if (tid == 0 && n4 > 0) {
     mbar_arrive_expect_tx(&s_bar, static_cast<uint32_t>(n4) * 16u);
     bulk_load(s_keys, sc + lo, static_cast<uint32_t>(n4) * 16u, &s_bar);
@@ -932,6 +932,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
     return;
   }
 
+  bool copy_ok = true;  // this CTA's slice landed
   // digit A from the scan's histogram, when there is one (identical in every CTA)
   uint32_t dA = 0u;
   int krem = k, nA = 0;
@@ -955,7 +956,12 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
     const bool gather_now = p.hist && nA <= kCandCap;
     const uint32_t pre = dA << 21;
     if (n4 > 0 && !mbar_wait(&s_bar, 0u, p.status)) {
-      // the copy never completed: leave the (undefined) slice as it is; the status word says why
+      // The copy did not complete within the wait limit (the status word says so): this CTA
+      // contributes no keys, the cluster still runs every barrier, and the query's result is
+      // withdrawn below (out_cnt = 0).
+      copy_ok = false;
+      n4 = 0;
+      len = 0;
     }
     uint4* k4 = reinterpret_cast<uint4*>(s_keys);
     for (int base = 0; base < n4; base += kSelThreads) {
@@ -1115,15 +1121,26 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
     }
     s_cnt[0] = tg;
     s_cnt[1] = te;
+    s_cnt[2] = copy_ok ? 0 : 1;
   }
   cluster.sync();
-  if (tid < 2 * CL) s_peer[tid] = *cluster.map_shared_rank(&s_cnt[tid & 1], tid >> 1);  // one remote read each
+  if (tid < 3 * CL) s_peer[tid] = *cluster.map_shared_rank(&s_cnt[tid % 3], tid / 3);  // one remote read each
   __syncthreads();
+  bool any_fail = false;
+  for (int r = 0; r < CL; ++r) any_fail |= s_peer[3 * r + 2] != 0;
+  if (any_fail) {
+    // a slice of this query is missing: no selection is reported for it
+    if (rank == 0 && tid == 0) p.out_cnt[b] = 0;
+    // a copy that gave up may still land: wait for it (bounded) before this CTA's memory is released
+    if (!copy_ok && tid == 0) mbar_wait(&s_bar, 0u, nullptr);
+    cluster.sync();  // peers may still read this CTA's shared memory
+    return;
+  }
   // ties are taken in index order: CTA r may take krem minus the ties of CTAs before it
   int eq_before = 0, sel_before = 0, take_eq = 0;
   for (int r = 0; r < CL; ++r) {
-    const int g_r = s_peer[2 * r];
-    const int e_r = s_peer[2 * r + 1];
+    const int g_r = s_peer[3 * r];
+    const int e_r = s_peer[3 * r + 1];
     int t_r = krem - eq_before;
     t_r = t_r < 0 ? 0 : (t_r > e_r ? e_r : t_r);
     if (r < rank) {

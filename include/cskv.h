@@ -255,12 +255,17 @@ cskv_status csa_index_score_topk(const cskv_index_args* args, void* workspace, s
  *   - Scratch: a file-scope device array of CSKV_STATIC_INDEX_SCRATCH_FLOATS
  *     fp32 values (16 MiB) inside libcskv.so. Every GPU that loads the
  *     library holds it until the process exits.
- *   - Limit: a call needs csa_index_ws_bytes() bytes of it; a larger request
+ *   - Limit: a call needs csa_index_ws_bytes() bytes of it, i.e. 4 bytes x
  *     (n_q x (the visible entries of max_pos rounded up to 64, plus 2048
- *     histogram counters)) returns CSKV_ERR_WORKSPACE and launches nothing.
+ *     histogram counters) + 64); a request above 16 MiB, that is with
+ *     n_q x (...) > CSKV_STATIC_INDEX_SCRATCH_FLOATS - 64, returns
+ *     CSKV_ERR_WORKSPACE and launches nothing.
  *   - Set-up: the first call on each device looks up the array's device
- *     address (cudaGetSymbolAddress) with that device current; make that
- *     first call before any stream capture.
+ *     address (cudaGetSymbolAddress) with that device current and keeps it
+ *     for the life of the process; make that first call before any stream
+ *     capture. The address belongs to the device's primary context: call
+ *     this entry point only with the primary context current (the runtime
+ *     API's default), and not after cudaDeviceReset() in the same process.
  *   - Sharing: every call uses the same array and leaves its contents
  *     behind. Nothing in it needs clearing (each call writes every score it
  *     reads and zeroes the counters it uses), but two calls that can run on the GPU at the same time -- on
@@ -316,6 +321,23 @@ cskv_status hca_attend(const cskv_attend_args* args, void* workspace, size_t ws_
 /* cskv_get_status -- copies the device status word to *status (host) and
  * clears it; synchronises the stream. */
 cskv_status cskv_get_status(int32_t* d_status, void* stream, int32_t* status);
+
+/*
+ * cskv_selftest_wait -- checks the bounded device wait behind every
+ * mbarrier hand-off of the library's kernels (producer -> consumer stages;
+ * no wait may spin forever, so a lost arrival ends the kernel with
+ * CSKV_ERR_TIMEOUT in the status word instead of hanging the GPU).
+ * Launches one warp that waits on an mbarrier for at most spin_limit polls.
+ *   arrive = 1: the barrier's one expected arrival is made first; the wait
+ *               succeeds and the status word is left alone.
+ *   arrive = 0: nothing arrives and no asynchronous copy is outstanding; the
+ *               wait gives up after spin_limit polls and writes
+ *               CSKV_ERR_TIMEOUT into *d_status (if it still holds 0).
+ * The kernels themselves use a fixed limit of 2^24 polls. Read the result
+ * with cskv_get_status(). Errors: CSKV_ERR_INVALID_ARG for a NULL status
+ * word or spin_limit = 0; CSKV_ERR_CUDA if the launch fails.
+ */
+cskv_status cskv_selftest_wait(int32_t arrive, uint32_t spin_limit, int32_t* d_status, void* stream);
 
 /* human-readable name of a status code (static string) */
 const char* cskv_status_string(cskv_status s);

@@ -112,3 +112,11 @@ def test_workspace_queries_are_host_only(cskv_built):
     assert n >= 8 * 262112 * 4
     with pytest.raises(ck.CskvError):
         ck.csa_index_ws_bytes(layer, n_q=8, n_heads_idx=8, max_pos=-1, k=1024)
+
+
+def test_wait_selftest_rejects_bad_arguments_on_host(cskv_built):
+    import compressed_sparse_kv_02_b200 as ck
+    L = ck.lib()
+    assert L.cskv_selftest_wait(0, 1000, None, None) == ck.ERR_INVALID_ARG  # no status word
+    st = ctypes.c_int32(0)  # never dereferenced: the limit check returns first
+    assert L.cskv_selftest_wait(0, 0, ctypes.addressof(st), None) == ck.ERR_INVALID_ARG
