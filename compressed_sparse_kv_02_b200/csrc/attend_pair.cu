@@ -17,7 +17,7 @@
 //     then cp.async of the 2 x 64 rows (16 threads per 256-byte row) into a
 //     128-byte-swizzled stage (four stages: the loaders run up to three tiles
 //     ahead, so the hand-offs of consecutive tiles overlap); Q of the pair by TMA;
-//   MMA (warp 4, one thread): S(t) = Q K^T (2 x 8 MMAs, M = 64, N = 64, K = 16)
+//   MMA (warp 4, lane 0 issues): S(t) = Q K^T (2 x 8 MMAs, M = 64, N = 64, K = 16)
 //     into S buffer t & 1; then O += P(t - 1) V (2 x 4 MMAs, N = d_v = 128, V read
 //     MN-major from the same stage: V is the first d_v channels of each key);
 //   softmax (warps 0-3): max pass over S(t) in tensor memory, lazy O rescale,
@@ -46,7 +46,6 @@ constexpr int kQBytes = 2 * kH * kD * 2;        // 32768: Q of both queries
 constexpr int kPBytes = 2 * kH * kNk * 2;       // 16384: P of both queries (one buffer)
 constexpr int kRows = 2 * kNk;                  // key rows of a tile (both queries)
 constexpr int kThreads = 288;       // warps 0-3 softmax, warp 4 MMA, warps 5-8 loads
-constexpr int kMmaThread = 128;
 constexpr int kLoadThread0 = 160;
 constexpr int kLoaders = kThreads - kLoadThread0;  // 128
 constexpr uint32_t kTmemCols = 512;
@@ -237,19 +236,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid >= kLoadThread0) {
       // ---------------------------------------------------------------- loaders
-      const int lt = tid - kLoadThread0;
-      if (lt == 0) {  // Q of both queries once the last item's S products are done with the buffer
-        bool okq = n_item == 0 || mbar_wait(qempty, (n_item - 1) & 1u, p.status);
-        if (okq) {
-          mbar_arrive_expect_tx(qfull, kQBytes);
-          const int qb1 = b1 >= 0 ? b1 : b0;  // a lone last query: its slot repeats it (never read out)
-          for (int h = 0; h < 2; ++h) {
-            tma_load_2d(sQ + h * (kH * 128), &tm_q, h * 64, b0 * kH, qfull);
-            tma_load_2d(sQ + kQBytes / 2 + h * (kH * 128), &tm_q, h * 64, qb1 * kH, qfull);
+      const int lt = tid - kLoadThread0, lw = lt >> 5, ll = lt & 31;
+      // The first loader warp takes the loaders' waits together (no lane of it waits on an
+      // mbarrier while the others sit at a barrier); lane 0 issues.
+      if (lw == 0) {  // Q of both queries once the last item's S products are done with the buffer
+        const bool okq = __all_sync(kFull, n_item == 0 || mbar_wait(qempty, (n_item - 1) & 1u, p.status));
+        if (ll == 0) {
+          if (okq) {
+            mbar_arrive_expect_tx(qfull, kQBytes);
+            const int qb1 = b1 >= 0 ? b1 : b0;  // a lone last query: its slot repeats it (never read out)
+            for (int h = 0; h < 2; ++h) {
+              tma_load_2d(sQ + h * (kH * 128), &tm_q, h * 64, b0 * kH, qfull);
+              tma_load_2d(sQ + kQBytes / 2 + h * (kH * 128), &tm_q, h * 64, qb1 * kH, qfull);
+            }
+          } else {
+            *sAbort = 1;
           }
-        } else {
-          *sAbort = 1;
         }
+        __syncwarp();
       }
       // this thread's part of every tile: the source row of key (lt & 63) of query lt >> 6, and
       // chunk (lt & 15) of rows (lt >> 4) + 8 q. A tile is signalled as soon as its copy has
@@ -271,8 +275,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t gt = g + it;
         const int st = gt % kNS;
         const uint32_t c = nc;
-        if (lt == 0)
-          *sLdOk = !*sAbort && (gt < (uint32_t)kNS || mbar_wait(&kempty[st], ((gt / kNS) - 1) & 1u, p.status));
+        if (lw == 0) {
+          bool okw = __shfl_sync(kFull, *sAbort, 0) == 0;
+          if (okw && gt >= (uint32_t)kNS)
+            okw = __all_sync(kFull, mbar_wait(&kempty[st], ((gt / kNS) - 1) & 1u, p.status));
+          if (ll == 0) *sLdOk = okw;
+        }
         named_sync(3, kLoaders);  // sLdOk is set (and the last tile's issue has read sRow)
         if (!*sLdOk) {
           *sAbort = 1;
@@ -302,41 +310,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lt == 0) mbar_arrive(&kfull[st]);
         if (it + 1 < ntiles) nc = code_of(it + 1);
       }
-    } else if (tid == kMmaThread) {
+    } else if (warp == 4) {
       // ---------------------------------------------------------------- MMA issue
+      // The whole warp takes every wait (it never diverges around a barrier); lane 0 issues the
+      // MMAs and their commits.
+      const bool issuer = lane == 0;
       const uint32_t idesc_s = umma_idesc_bf16(kH, kNk, false);
       const uint32_t idesc_pv = umma_idesc_bf16(kH, kD, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sPa = smem_u32(sP);
-      bool ok = mbar_wait(qfull, n_item & 1u, p.status);
+      bool ok = __all_sync(kFull, mbar_wait(qfull, n_item & 1u, p.status));
       tc_fence_after();
-      for (int it = 0; it <= ntiles && ok && !*sAbort; ++it) {
+      for (int it = 0; it <= ntiles && ok; ++it) {
+        if (__shfl_sync(kFull, *sAbort, 0)) break;
         if (it < ntiles) {
           const uint32_t gt = g + it;
           const int st = gt % kNS;
-          if (!(ok = mbar_wait(&kfull[st], (gt / kNS) & 1u, p.status))) break;
+          if (!(ok = __all_sync(kFull, mbar_wait(&kfull[st], (gt / kNS) & 1u, p.status)))) break;
           tc_fence_after();
-          const uint32_t d = tmem + kColS + (gt & 1u) * kNk;
-          const uint32_t kb = sKa + st * kStageBytes;
-          issue_s(d, sQa, kb, idesc_s);
-          issue_s(d + (16u << 16), sQa + kQBytes / 2, kb + kSlotBytes, idesc_s);
-          umma_commit(&sfull[gt & 1u]);
-          if (it == ntiles - 1) umma_commit(qempty);
+          if (issuer) {
+            const uint32_t d = tmem + kColS + (gt & 1u) * kNk;
+            const uint32_t kb = sKa + st * kStageBytes;
+            issue_s(d, sQa, kb, idesc_s);
+            issue_s(d + (16u << 16), sQa + kQBytes / 2, kb + kSlotBytes, idesc_s);
+            umma_commit(&sfull[gt & 1u]);
+            if (it == ntiles - 1) umma_commit(qempty);
+          }
+          __syncwarp();
         }
         if (it >= 1) {
           const uint32_t gp = g + it - 1;
           const int pb = gp & 1u, sp = gp % kNS;
-          if (!(ok = mbar_wait(&pfull[pb], (gp >> 1) & 1u, p.status))) break;
+          if (!(ok = __all_sync(kFull, mbar_wait(&pfull[pb], (gp >> 1) & 1u, p.status)))) break;
           tc_fence_after();
-          const uint32_t vb = sKa + sp * kStageBytes, pm = sPa + pb * kPBytes;
-          issue_pv(tmem + kColO, pm, vb, idesc_pv, it > 1);
-          issue_pv(tmem + kColO + (16u << 16), pm + kPBytes / 2, vb + kSlotBytes, idesc_pv, it > 1);
-          umma_commit(&kempty[sp]);
-          umma_commit(&obar[pb]);
+          if (issuer) {
+            const uint32_t vb = sKa + sp * kStageBytes, pm = sPa + pb * kPBytes;
+            issue_pv(tmem + kColO, pm, vb, idesc_pv, it > 1);
+            issue_pv(tmem + kColO + (16u << 16), pm + kPBytes / 2, vb + kSlotBytes, idesc_pv, it > 1);
+            umma_commit(&kempty[sp]);
+            umma_commit(&obar[pb]);
+          }
+          __syncwarp();
         }
       }
-      if (ntiles == 0) umma_commit(qempty);
-      umma_commit(dbar);  // one completion per item, also after an abort
-      if (!ok) *sAbort = 1;
+      if (issuer) {
+        if (ntiles == 0) umma_commit(qempty);
+        umma_commit(dbar);  // one completion per item, also after an abort
+        if (!ok) *sAbort = 1;
+      }
+      __syncwarp();
     } else if (warp < 4) {
       // ---------------------------------------------------------------- softmax (one head row per thread)
       const int slot = lane >> 4, h = warp * 16 + (lane & 15);
@@ -471,12 +492,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     g += ntiles;
   }
-  // after an abort, give tensor-core work and copies in flight a bounded chance to land
-  if (tid == kMmaThread && *sAbort) {
-    umma_commit(dbar);
+  // after an abort, give tensor-core work and copies in flight a bounded chance to land (each
+  // warp decides on lane 0's reading of the flag, so it stays converged)
+  if (warp == 4 && __shfl_sync(kFull, *sAbort, 0)) {
+    if (lane == 0) umma_commit(dbar);
+    __syncwarp();
     mbar_wait(dbar, n_item & 1u, nullptr);
   }
-  if (tid == kLoadThread0 && *sAbort) mbar_wait(qfull, n_item & 1u, nullptr);
+  if (warp == kLoadThread0 / 32 && __shfl_sync(kFull, *sAbort, 0)) mbar_wait(qfull, n_item & 1u, nullptr);
   cp_async_wait<0>();
   tc_fence_before();
   __syncthreads();
