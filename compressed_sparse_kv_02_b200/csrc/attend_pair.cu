@@ -385,18 +385,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t* valid = sMask + (gt % kNS) * 4 + slot * 2;
-        float mt = -INFINITY;
-        {  // both 32-key halves of the tile, one wait
-          uint32_t s[32], s2[32];
-          tmem_ld32(sb, s);
-          tmem_ld32(sb + 32, s2);
-          const uint32_t vw = valid[0], vw2 = valid[1];
+        // the tile's 64 logits of this row (two loads, one wait); the row max in four chains
+        const uint64_t vm = static_cast<uint64_t>(valid[0]) | (static_cast<uint64_t>(valid[1]) << 32);
+        float mt;
+        {
+          uint32_t s[kNk];
+          tmem_ld32(sb, *reinterpret_cast<uint32_t(*)[32]>(s));
+          tmem_ld32(sb + 32, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
           tmem_ld_wait();
+          float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if ((vw >> j) & 1u) mt = fmaxf(mt, __uint_as_float(s[j]) * sl2);
-            if ((vw2 >> j) & 1u) mt = fmaxf(mt, __uint_as_float(s2[j]) * sl2);
+          for (int j = 0; j < kNk; j += 4) {
+            if ((vm >> j) & 1u) m0 = fmaxf(m0, __uint_as_float(s[j]) * sl2);
+            if ((vm >> (j + 1)) & 1u) m1 = fmaxf(m1, __uint_as_float(s[j + 1]) * sl2);
+            if ((vm >> (j + 2)) & 1u) m2 = fmaxf(m2, __uint_as_float(s[j + 2]) * sl2);
+            if ((vm >> (j + 3)) & 1u) m3 = fmaxf(m3, __uint_as_float(s[j + 3]) * sl2);
           }
+          mt = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
         }
         float corr = 1.f;
         bool rescale = false;
@@ -434,24 +439,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st_wait();
         }
         uint8_t* pbuf = prow + (gt & 1u) * kPBytes;
-#pragma unroll 1
-        for (int c = 0; c < kNk / 32; ++c) {
-          uint32_t s[32];
-          tmem_ld32(sb + c * 32, s);
-          const uint32_t vw = valid[c];
+        {  // the logits again (two loads, one wait), their exponentials, the row sum in two chains
+          uint32_t s[kNk];
+          tmem_ld32(sb, *reinterpret_cast<uint32_t(*)[32]>(s));
+          tmem_ld32(sb + 32, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
           tmem_ld_wait();
-          uint32_t pp[16];
+          float l0 = 0.f, l1 = 0.f;
+          uint32_t pp[kNk / 2];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float e0 = (vw >> (2 * j)) & 1u ? exp2f(__uint_as_float(s[2 * j]) * sl2 - msub) : 0.f;
-            const float e1 = (vw >> (2 * j + 1)) & 1u ? exp2f(__uint_as_float(s[2 * j + 1]) * sl2 - msub) : 0.f;
-            l_run += e0 + e1;
+          for (int j = 0; j < kNk / 2; ++j) {
+            const float e0 = (vm >> (2 * j)) & 1u ? exp2f(__uint_as_float(s[2 * j]) * sl2 - msub) : 0.f;
+            const float e1 = (vm >> (2 * j + 1)) & 1u ? exp2f(__uint_as_float(s[2 * j + 1]) * sl2 - msub) : 0.f;
+            l0 += e0;
+            l1 += e1;
             pp[j] = pack_bf16(e0, e1);
           }
-          // keys 32 c .. 32 c + 31: 16-byte chunks 4 c .. 4 c + 3 of the row (one 64-key atom)
+          l_run += l0 + l1;
+          // keys 8 i .. 8 i + 7: 16-byte chunk i of the row (one 64-key atom)
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<uint4*>(pbuf + (((c * 4 + i) ^ sw) << 4)) =
+          for (int i = 0; i < kNk / 8; ++i)
+            *reinterpret_cast<uint4*>(pbuf + ((i ^ sw) << 4)) =
                 make_uint4(pp[4 * i], pp[4 * i + 1], pp[4 * i + 2], pp[4 * i + 3]);
         }
         fence_proxy_async_smem();
