@@ -231,7 +231,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     // a sequence id outside the layer: the query's keys are all masked (zero output), as in the
     // other attention kernels, and the status word says why
     if (tid == 0 && ((!ok0 && k0.n > 0) || (b1 >= 0 && !ok1 && k1.n > 0))) report(p.status, CSKV_ERR_OUT_OF_RANGE);
-    const int nmax = n0 > n1 ? n0 : n1;
+    // HCA rows of a prefill chunk: consecutive positions t, t + 1 of one sequence see the same
+    // entries up to the last one of t + 1 and windows that differ by one row, so the pair shares
+    // one key list (window rows ws(t) .. t + 1, then the entries of t + 1) and every tile is loaded
+    // once for both; the valid-key bits tell each query which of the keys it sees.
+    const bool shared = !p.is_csa && p.x_chunk && ok0 && ok1 && s0 == s1 && k0.n > 0 && k1.n > 0 &&
+                        k1.t == k0.t + 1;
+    Keys ksh;  // the shared list (window start of t, last position t + 1)
+    ksh.t = k1.t;
+    ksh.ws = k0.ws;
+    ksh.n_w = static_cast<int>(k1.t - k0.ws + 1);
+    ksh.n = ksh.n_w + (k1.n - k1.n_w);
+    const int nmax = shared ? ksh.n : (n0 > n1 ? n0 : n1);
     const int ntiles = (nmax + kNk - 1) / kNk;
 
     if (tid >= kLoadThread0) {
@@ -262,8 +273,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int chunk = lt & 15, half = chunk >> 3, c8 = chunk & 7;
       const int my_slot = lt >> 6, my_key = lt & (kNk - 1);
       auto code_of = [&](int it) -> uint32_t {
-        const int u = it * kNk + my_key;
         uint32_t c = 0;
+        if (shared) {  // threads 0 .. kNk - 1: key lt of the shared list
+          const int u = it * kNk + lt;
+          if (lt < kNk && u < ksh.n) {
+            c = key_code(p, b1, s1, ksh, u);
+            if (!c) report(p.status, CSKV_ERR_OUT_OF_RANGE);
+          }
+          return c;
+        }
+        const int u = it * kNk + my_key;
         if (u < (my_slot ? n1 : n0)) {
           c = my_slot ? key_code(p, b1, s1, k1, u) : key_code(p, b0, s0, k0, u);
           if (!c) report(p.status, CSKV_ERR_OUT_OF_RANGE);
@@ -287,15 +306,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         sRow[lt] = c;
-        {  // valid-key bits of the tile (the softmax reads them after kfull[st]): warp w of the
-           // loaders holds keys 32 (w & 1) .. + 31 of query w >> 1
+        if (shared) {  // loader warps 0 and 1 hold keys 32 w .. + 31 of the shared list
+          const int u = it * kNk + lt;
+          const bool win = u < ksh.n_w;
+          // t sees the window rows up to t (all but the last) and its own entries; t + 1 the rows
+          // from its window start and every entry of the list
+          const bool v0 = c != 0 && (win ? u < ksh.n_w - 1 : u - ksh.n_w < k0.n - k0.n_w);
+          const bool v1 = c != 0 && (!win || k0.ws + u >= k1.ws);
+          const unsigned m0 = __ballot_sync(kFull, v0), m1 = __ballot_sync(kFull, v1);
+          if (ll == 0 && lw < 2) {
+            sMask[st * 4 + lw] = m0;
+            sMask[st * 4 + 2 + lw] = m1;
+          }
+        } else {  // valid-key bits of the tile (the softmax reads them after kfull[st]): warp w of
+                  // the loaders holds keys 32 (w & 1) .. + 31 of query w >> 1
           const unsigned mw = __ballot_sync(kFull, c != 0);
           if ((lt & 31) == 0) sMask[st * 4 + (lt >> 5)] = mw;
         }
         named_sync(3, kLoaders);
         uint8_t* dst = sK + st * kStageBytes + half * kHalfBytes;
+        const int n_q8 = shared ? kNk / 8 : kRows / 8;  // 8-row steps: one list or two
 #pragma unroll 4
-        for (int q = 0; q < kRows / 8; ++q) {
+        for (int q = 0; q < n_q8; ++q) {
           const int row = (lt >> 4) + 8 * q;  // query row / kNk, key row % kNk
           const int key = row & (kNk - 1);
           const uint16_t* src = code_row(p, sRow[row]);
@@ -331,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t d = tmem + kColS + (gt & 1u) * kNk;
             const uint32_t kb = sKa + st * kStageBytes;
             issue_s(d, sQa, kb, idesc_s);
-            issue_s(d + (16u << 16), sQa + kQBytes / 2, kb + kSlotBytes, idesc_s);
+            issue_s(d + (16u << 16), sQa + kQBytes / 2, shared ? kb : kb + kSlotBytes, idesc_s);
             umma_commit(&sfull[gt & 1u]);
             if (it == ntiles - 1) umma_commit(qempty);
           }
@@ -345,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (issuer) {
             const uint32_t vb = sKa + sp * kStageBytes, pm = sPa + pb * kPBytes;
             issue_pv(tmem + kColO, pm, vb, idesc_pv, it > 1);
-            issue_pv(tmem + kColO + (16u << 16), pm + kPBytes / 2, vb + kSlotBytes, idesc_pv, it > 1);
+            issue_pv(tmem + kColO + (16u << 16), pm + kPBytes / 2, shared ? vb : vb + kSlotBytes, idesc_pv, it > 1);
             umma_commit(&kempty[sp]);
             umma_commit(&obar[pb]);
           }
