@@ -1537,7 +1537,8 @@ cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st) {
   // many queries in one call (a prefill chunk): the grouped scan reads each key once per group
   const bool grouped = tma_ok && p.n_q >= kGroupScanMinQueries && (p.n_heads_idx == 4 || p.n_heads_idx == 8);
   if (nv_max > 0 && grouped) {
-    if (p.d_idx == 64 && p.n_heads_idx == 4) e = launch_scan_group<2, 4>(p, n_sm, st);
+    if (scan_tc_supported(p)) e = launch_scan_tc(p, n_sm, st);
+    else if (p.d_idx == 64 && p.n_heads_idx == 4) e = launch_scan_group<2, 4>(p, n_sm, st);
     else if (p.d_idx == 64) e = launch_scan_group<2, 8>(p, n_sm, st);
     else if (p.n_heads_idx == 4) e = launch_scan_group<4, 4>(p, n_sm, st);
     else e = launch_scan_group<4, 8>(p, n_sm, st);
