@@ -17,7 +17,7 @@
 //     then cp.async of the 2 x 64 rows (16 threads per 256-byte row) into a
 //     128-byte-swizzled stage (four stages: the loaders run up to three tiles
 //     ahead, so the hand-offs of consecutive tiles overlap); Q of the pair by TMA;
-//   MMA (warp 4, one thread): S(t) = Q K^T (2 x 8 MMAs, M = 64, N = 64, K = 16)
+//   MMA (warp 4, lane 0 issues): S(t) = Q K^T (2 x 8 MMAs, M = 64, N = 64, K = 16)
 //     into S buffer t & 1; then O += P(t - 1) V (2 x 4 MMAs, N = d_v = 128, V read
 //     MN-major from the same stage: V is the first d_v channels of each key);
 //   softmax (warps 0-3): max pass over S(t) in tensor memory, lazy O rescale,
@@ -46,7 +46,6 @@ constexpr int kQBytes = 2 * kH * kD * 2;        // 32768: Q of both queries
 constexpr int kPBytes = 2 * kH * kNk * 2;       // 16384: P of both queries (one buffer)
 constexpr int kRows = 2 * kNk;                  // key rows of a tile (both queries)
 constexpr int kThreads = 288;       // warps 0-3 softmax, warp 4 MMA, warps 5-8 loads
-constexpr int kMmaThread = 128;
 constexpr int kLoadThread0 = 160;
 constexpr int kLoaders = kThreads - kLoadThread0;  // 128
 constexpr uint32_t kTmemCols = 512;
@@ -232,24 +231,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     // a sequence id outside the layer: the query's keys are all masked (zero output), as in the
     // other attention kernels, and the status word says why
     if (tid == 0 && ((!ok0 && k0.n > 0) || (b1 >= 0 && !ok1 && k1.n > 0))) report(p.status, CSKV_ERR_OUT_OF_RANGE);
-    const int nmax = n0 > n1 ? n0 : n1;
+    // HCA rows of a prefill chunk: consecutive positions t, t + 1 of one sequence see the same
+    // entries up to the last one of t + 1 and windows that differ by one row, so the pair shares
+    // one key list (window rows ws(t) .. t + 1, then the entries of t + 1) and every tile is loaded
+    // once for both; the valid-key bits tell each query which of the keys it sees.
+    const bool shared = !p.is_csa && p.x_chunk && ok0 && ok1 && s0 == s1 && k0.n > 0 && k1.n > 0 &&
+                        k1.t == k0.t + 1;
+    Keys ksh;  // the shared list (window start of t, last position t + 1)
+    ksh.t = k1.t;
+    ksh.ws = k0.ws;
+    ksh.n_w = static_cast<int>(k1.t - k0.ws + 1);
+    ksh.n = ksh.n_w + (k1.n - k1.n_w);
+    const int nmax = shared ? ksh.n : (n0 > n1 ? n0 : n1);
     const int ntiles = (nmax + kNk - 1) / kNk;
 
     if (tid >= kLoadThread0) {
       // ---------------------------------------------------------------- loaders
-      const int lt = tid - kLoadThread0;
-      if (lt == 0) {  // Q of both queries once the last item's S products are done with the buffer
-        bool okq = n_item == 0 || mbar_wait(qempty, (n_item - 1) & 1u, p.status);
-        if (okq) {
-          mbar_arrive_expect_tx(qfull, kQBytes);
-          const int qb1 = b1 >= 0 ? b1 : b0;  // a lone last query: its slot repeats it (never read out)
-          for (int h = 0; h < 2; ++h) {
-            tma_load_2d(sQ + h * (kH * 128), &tm_q, h * 64, b0 * kH, qfull);
-            tma_load_2d(sQ + kQBytes / 2 + h * (kH * 128), &tm_q, h * 64, qb1 * kH, qfull);
+      const int lt = tid - kLoadThread0, lw = lt >> 5, ll = lt & 31;
+      // The first loader warp takes the loaders' waits together (no lane of it waits on an
+      // mbarrier while the others sit at a barrier); lane 0 issues.
+      if (lw == 0) {  // Q of both queries once the last item's S products are done with the buffer
+        const bool okq = __all_sync(kFull, n_item == 0 || mbar_wait(qempty, (n_item - 1) & 1u, p.status));
+        if (ll == 0) {
+          if (okq) {
+            mbar_arrive_expect_tx(qfull, kQBytes);
+            const int qb1 = b1 >= 0 ? b1 : b0;  // a lone last query: its slot repeats it (never read out)
+            for (int h = 0; h < 2; ++h) {
+              tma_load_2d(sQ + h * (kH * 128), &tm_q, h * 64, b0 * kH, qfull);
+              tma_load_2d(sQ + kQBytes / 2 + h * (kH * 128), &tm_q, h * 64, qb1 * kH, qfull);
+            }
+          } else {
+            *sAbort = 1;
           }
-        } else {
-          *sAbort = 1;
         }
+        __syncwarp();
       }
       // this thread's part of every tile: the source row of key (lt & 63) of query lt >> 6, and
       // chunk (lt & 15) of rows (lt >> 4) + 8 q. A tile is signalled as soon as its copy has
@@ -258,8 +273,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int chunk = lt & 15, half = chunk >> 3, c8 = chunk & 7;
       const int my_slot = lt >> 6, my_key = lt & (kNk - 1);
       auto code_of = [&](int it) -> uint32_t {
-        const int u = it * kNk + my_key;
         uint32_t c = 0;
+        if (shared) {  // threads 0 .. kNk - 1: key lt of the shared list
+          const int u = it * kNk + lt;
+          if (lt < kNk && u < ksh.n) {
+            c = key_code(p, b1, s1, ksh, u);
+            if (!c) report(p.status, CSKV_ERR_OUT_OF_RANGE);
+          }
+          return c;
+        }
+        const int u = it * kNk + my_key;
         if (u < (my_slot ? n1 : n0)) {
           c = my_slot ? key_code(p, b1, s1, k1, u) : key_code(p, b0, s0, k0, u);
           if (!c) report(p.status, CSKV_ERR_OUT_OF_RANGE);
@@ -271,23 +294,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t gt = g + it;
         const int st = gt % kNS;
         const uint32_t c = nc;
-        if (lt == 0)
-          *sLdOk = !*sAbort && (gt < (uint32_t)kNS || mbar_wait(&kempty[st], ((gt / kNS) - 1) & 1u, p.status));
+        if (lw == 0) {
+          bool okw = __shfl_sync(kFull, *sAbort, 0) == 0;
+          if (okw && gt >= (uint32_t)kNS)
+            okw = __all_sync(kFull, mbar_wait(&kempty[st], ((gt / kNS) - 1) & 1u, p.status));
+          if (ll == 0) *sLdOk = okw;
+        }
         named_sync(3, kLoaders);  // sLdOk is set (and the last tile's issue has read sRow)
         if (!*sLdOk) {
           *sAbort = 1;
           break;
         }
         sRow[lt] = c;
-        {  // valid-key bits of the tile (the softmax reads them after kfull[st]): warp w of the
-           // loaders holds keys 32 (w & 1) .. + 31 of query w >> 1
+        if (shared) {  // loader warps 0 and 1 hold keys 32 w .. + 31 of the shared list
+          const int u = it * kNk + lt;
+          const bool win = u < ksh.n_w;
+          // t sees the window rows up to t (all but the last) and its own entries; t + 1 the rows
+          // from its window start and every entry of the list
+          const bool v0 = c != 0 && (win ? u < ksh.n_w - 1 : u - ksh.n_w < k0.n - k0.n_w);
+          const bool v1 = c != 0 && (!win || k0.ws + u >= k1.ws);
+          const unsigned m0 = __ballot_sync(kFull, v0), m1 = __ballot_sync(kFull, v1);
+          if (ll == 0 && lw < 2) {
+            sMask[st * 4 + lw] = m0;
+            sMask[st * 4 + 2 + lw] = m1;
+          }
+        } else {  // valid-key bits of the tile (the softmax reads them after kfull[st]): warp w of
+                  // the loaders holds keys 32 (w & 1) .. + 31 of query w >> 1
           const unsigned mw = __ballot_sync(kFull, c != 0);
           if ((lt & 31) == 0) sMask[st * 4 + (lt >> 5)] = mw;
         }
         named_sync(3, kLoaders);
         uint8_t* dst = sK + st * kStageBytes + half * kHalfBytes;
+        const int n_q8 = shared ? kNk / 8 : kRows / 8;  // 8-row steps: one list or two
 #pragma unroll 4
-        for (int q = 0; q < kRows / 8; ++q) {
+        for (int q = 0; q < n_q8; ++q) {
           const int row = (lt >> 4) + 8 * q;  // query row / kNk, key row % kNk
           const int key = row & (kNk - 1);
           const uint16_t* src = code_row(p, sRow[row]);
@@ -302,41 +342,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lt == 0) mbar_arrive(&kfull[st]);
         if (it + 1 < ntiles) nc = code_of(it + 1);
       }
-    } else if (tid == kMmaThread) {
+    } else if (warp == 4) {
       // ---------------------------------------------------------------- MMA issue
+      // The whole warp takes every wait (it never diverges around a barrier); lane 0 issues the
+      // MMAs and their commits.
+      const bool issuer = lane == 0;
       const uint32_t idesc_s = umma_idesc_bf16(kH, kNk, false);
       const uint32_t idesc_pv = umma_idesc_bf16(kH, kD, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sPa = smem_u32(sP);
-      bool ok = mbar_wait(qfull, n_item & 1u, p.status);
+      bool ok = __all_sync(kFull, mbar_wait(qfull, n_item & 1u, p.status));
       tc_fence_after();
-      for (int it = 0; it <= ntiles && ok && !*sAbort; ++it) {
+      for (int it = 0; it <= ntiles && ok; ++it) {
+        if (__shfl_sync(kFull, *sAbort, 0)) break;
         if (it < ntiles) {
           const uint32_t gt = g + it;
           const int st = gt % kNS;
-          if (!(ok = mbar_wait(&kfull[st], (gt / kNS) & 1u, p.status))) break;
+          if (!(ok = __all_sync(kFull, mbar_wait(&kfull[st], (gt / kNS) & 1u, p.status)))) break;
           tc_fence_after();
-          const uint32_t d = tmem + kColS + (gt & 1u) * kNk;
-          const uint32_t kb = sKa + st * kStageBytes;
-          issue_s(d, sQa, kb, idesc_s);
-          issue_s(d + (16u << 16), sQa + kQBytes / 2, kb + kSlotBytes, idesc_s);
-          umma_commit(&sfull[gt & 1u]);
-          if (it == ntiles - 1) umma_commit(qempty);
+          if (issuer) {
+            const uint32_t d = tmem + kColS + (gt & 1u) * kNk;
+            const uint32_t kb = sKa + st * kStageBytes;
+            issue_s(d, sQa, kb, idesc_s);
+            issue_s(d + (16u << 16), sQa + kQBytes / 2, shared ? kb : kb + kSlotBytes, idesc_s);
+            umma_commit(&sfull[gt & 1u]);
+            if (it == ntiles - 1) umma_commit(qempty);
+          }
+          __syncwarp();
         }
         if (it >= 1) {
           const uint32_t gp = g + it - 1;
           const int pb = gp & 1u, sp = gp % kNS;
-          if (!(ok = mbar_wait(&pfull[pb], (gp >> 1) & 1u, p.status))) break;
+          if (!(ok = __all_sync(kFull, mbar_wait(&pfull[pb], (gp >> 1) & 1u, p.status)))) break;
           tc_fence_after();
-          const uint32_t vb = sKa + sp * kStageBytes, pm = sPa + pb * kPBytes;
-          issue_pv(tmem + kColO, pm, vb, idesc_pv, it > 1);
-          issue_pv(tmem + kColO + (16u << 16), pm + kPBytes / 2, vb + kSlotBytes, idesc_pv, it > 1);
-          umma_commit(&kempty[sp]);
-          umma_commit(&obar[pb]);
+          if (issuer) {
+            const uint32_t vb = sKa + sp * kStageBytes, pm = sPa + pb * kPBytes;
+            issue_pv(tmem + kColO, pm, vb, idesc_pv, it > 1);
+            issue_pv(tmem + kColO + (16u << 16), pm + kPBytes / 2, shared ? vb : vb + kSlotBytes, idesc_pv, it > 1);
+            umma_commit(&kempty[sp]);
+            umma_commit(&obar[pb]);
+          }
+          __syncwarp();
         }
       }
-      if (ntiles == 0) umma_commit(qempty);
-      umma_commit(dbar);  // one completion per item, also after an abort
-      if (!ok) *sAbort = 1;
+      if (issuer) {
+        if (ntiles == 0) umma_commit(qempty);
+        umma_commit(dbar);  // one completion per item, also after an abort
+        if (!ok) *sAbort = 1;
+      }
+      __syncwarp();
     } else if (warp < 4) {
       // ---------------------------------------------------------------- softmax (one head row per thread)
       const int slot = lane >> 4, h = warp * 16 + (lane & 15);
@@ -364,18 +417,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t* valid = sMask + (gt % kNS) * 4 + slot * 2;
-        float mt = -INFINITY;
-        {  // both 32-key halves of the tile, one wait
-          uint32_t s[32], s2[32];
-          tmem_ld32(sb, s);
-          tmem_ld32(sb + 32, s2);
-          const uint32_t vw = valid[0], vw2 = valid[1];
+        // the tile's 64 logits of this row (two loads, one wait); the row max in four chains
+        const uint64_t vm = static_cast<uint64_t>(valid[0]) | (static_cast<uint64_t>(valid[1]) << 32);
+        float mt;
+        {
+          uint32_t s[kNk];
+          tmem_ld32(sb, *reinterpret_cast<uint32_t(*)[32]>(s));
+          tmem_ld32(sb + 32, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
           tmem_ld_wait();
+          float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if ((vw >> j) & 1u) mt = fmaxf(mt, __uint_as_float(s[j]) * sl2);
-            if ((vw2 >> j) & 1u) mt = fmaxf(mt, __uint_as_float(s2[j]) * sl2);
+          for (int j = 0; j < kNk; j += 4) {
+            if ((vm >> j) & 1u) m0 = fmaxf(m0, __uint_as_float(s[j]) * sl2);
+            if ((vm >> (j + 1)) & 1u) m1 = fmaxf(m1, __uint_as_float(s[j + 1]) * sl2);
+            if ((vm >> (j + 2)) & 1u) m2 = fmaxf(m2, __uint_as_float(s[j + 2]) * sl2);
+            if ((vm >> (j + 3)) & 1u) m3 = fmaxf(m3, __uint_as_float(s[j + 3]) * sl2);
           }
+          mt = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
         }
         float corr = 1.f;
         bool rescale = false;
@@ -413,24 +471,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st_wait();
         }
         uint8_t* pbuf = prow + (gt & 1u) * kPBytes;
-#pragma unroll 1
-        for (int c = 0; c < kNk / 32; ++c) {
-          uint32_t s[32];
-          tmem_ld32(sb + c * 32, s);
-          const uint32_t vw = valid[c];
+        {  // the logits again (two loads, one wait), their exponentials, the row sum in two chains
+          uint32_t s[kNk];
+          tmem_ld32(sb, *reinterpret_cast<uint32_t(*)[32]>(s));
+          tmem_ld32(sb + 32, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
           tmem_ld_wait();
-          uint32_t pp[16];
+          float l0 = 0.f, l1 = 0.f;
+          uint32_t pp[kNk / 2];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float e0 = (vw >> (2 * j)) & 1u ? exp2f(__uint_as_float(s[2 * j]) * sl2 - msub) : 0.f;
-            const float e1 = (vw >> (2 * j + 1)) & 1u ? exp2f(__uint_as_float(s[2 * j + 1]) * sl2 - msub) : 0.f;
-            l_run += e0 + e1;
+          for (int j = 0; j < kNk / 2; ++j) {
+            const float e0 = (vm >> (2 * j)) & 1u ? exp2f(__uint_as_float(s[2 * j]) * sl2 - msub) : 0.f;
+            const float e1 = (vm >> (2 * j + 1)) & 1u ? exp2f(__uint_as_float(s[2 * j + 1]) * sl2 - msub) : 0.f;
+            l0 += e0;
+            l1 += e1;
             pp[j] = pack_bf16(e0, e1);
           }
-          // keys 32 c .. 32 c + 31: 16-byte chunks 4 c .. 4 c + 3 of the row (one 64-key atom)
+          l_run += l0 + l1;
+          // keys 8 i .. 8 i + 7: 16-byte chunk i of the row (one 64-key atom)
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<uint4*>(pbuf + (((c * 4 + i) ^ sw) << 4)) =
+          for (int i = 0; i < kNk / 8; ++i)
+            *reinterpret_cast<uint4*>(pbuf + ((i ^ sw) << 4)) =
                 make_uint4(pp[4 * i], pp[4 * i + 1], pp[4 * i + 2], pp[4 * i + 3]);
         }
         fence_proxy_async_smem();
@@ -471,12 +531,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     g += ntiles;
   }
-  // after an abort, give tensor-core work and copies in flight a bounded chance to land
-  if (tid == kMmaThread && *sAbort) {
-    umma_commit(dbar);
+  // after an abort, give tensor-core work and copies in flight a bounded chance to land (each
+  // warp decides on lane 0's reading of the flag, so it stays converged)
+  if (warp == 4 && __shfl_sync(kFull, *sAbort, 0)) {
+    if (lane == 0) umma_commit(dbar);
+    __syncwarp();
     mbar_wait(dbar, n_item & 1u, nullptr);
   }
-  if (tid == kLoadThread0 && *sAbort) mbar_wait(qfull, n_item & 1u, nullptr);
+  if (warp == kLoadThread0 / 32 && __shfl_sync(kFull, *sAbort, 0)) mbar_wait(qfull, n_item & 1u, nullptr);
   cp_async_wait<0>();
   tc_fence_before();
   __syncthreads();

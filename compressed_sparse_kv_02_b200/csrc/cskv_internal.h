@@ -99,6 +99,10 @@ struct IndexParams {
 };
 
 size_t index_ws_bytes(int n_q, int64_t max_pos, int m, int n_win);
+// tensor-core (tcgen05) scores for calls with many queries: groups of 128 / H_I queries of one
+// sequence share every 128-key tile (bf16 keys, H_I = 4 or 8, d_I = 64 or 128)
+bool scan_tc_supported(const IndexParams& p);
+cudaError_t launch_scan_tc(IndexParams& p, int n_sm, cudaStream_t st);
 cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st);
 
 // Split-KV attention over window + compressed keys, then the LSE merge.

@@ -44,6 +44,7 @@ constexpr int kSliceCap = 32768;   // scores per CTA of the selection kernel
 constexpr int kMaxCluster = 16;   // CTAs per query in the selection kernel (above 8: non-portable)
 constexpr int kHistBins = 2048;   // bins of the score-key histogram the TMA scan leaves for the selection
 constexpr int kGroupScanMinQueries = 256;  // from this many queries per call the grouped scan is used
+constexpr int kStreamSelectMinQueries = 256;  // ... and the one-CTA-per-query streaming select
 
 __device__ __forceinline__ int64_t query_visible(const IndexParams& p, int b) {
   const int64_t t = p.q_pos[b];
@@ -1288,6 +1289,235 @@ cudaError_t launch_scan_group(IndexParams& p, int n_sm, cudaStream_t st) {
   return launch_pdl(kern, dim3(static_cast<unsigned>(n_sm)), dim3(kTmaThreads), smem, st, map, p);
 }
 
+// ---------------------------------------------------------------- top-k for many queries
+// One CTA of kStrThreads per query and ~25 KB of shared memory, so several queries share an SM
+// and their score reads overlap (a prefill block has thousands of queries of ~10^4 scores each).
+// The scores are streamed from global memory up to three times: the digit-A histogram (unless the
+// scan left one), the gather of the threshold bin, and the ordered output. The digits, the tie rule
+// (lower index first among keys equal to the k-th) and the ascending output are those of
+// index_select_kernel.
+constexpr int kStrThreads = 256;
+constexpr int kStrCandCap = 4096;
+
+// digit of the krem-th largest key from a histogram of nbins (nbins a multiple of kStrThreads)
+template <typename CountFn>
+__device__ __forceinline__ void find_digit_str(int nbins, int krem, CountFn count, int* s_w, uint32_t* s_res,
+                                               uint32_t& digit, int& krem_out, int& bin_cnt) {
+  const int per = nbins / kStrThreads;  // 4 or 8 bins per thread, from the top
+  int tot = 0;
+  for (int e = 0; e < per; ++e) tot += count(nbins - 1 - (threadIdx.x * per + e));
+  int all;
+  int run = block_exclusive_scan<kStrThreads>(tot, s_w, all);
+  if (run < krem && krem <= run + tot) {
+    for (int e = 0; e < per; ++e) {
+      const int bin = nbins - 1 - (threadIdx.x * per + e);
+      const int c = count(bin);
+      if (run < krem && krem <= run + c) {
+        s_res[0] = static_cast<uint32_t>(bin);
+        s_res[1] = static_cast<uint32_t>(krem - run);
+        s_res[2] = static_cast<uint32_t>(c);
+      }
+      run += c;
+    }
+  }
+  __syncthreads();
+  digit = s_res[0];
+  krem_out = static_cast<int>(s_res[1]);
+  bin_cnt = static_cast<int>(s_res[2]);
+  __syncthreads();
+}
+
+// count digit (key >> shift) & dmask of the keys with (key & mask) == prefix; warp-aggregated
+__device__ __forceinline__ void str_count(uint32_t key, bool valid, uint32_t mask, uint32_t prefix, int shift,
+                                          uint32_t dmask, uint32_t* hist) {
+  const bool ok = valid && (key & mask) == prefix;
+  const unsigned act = __ballot_sync(kFull, ok);
+  if (ok) {
+    const uint32_t dg = (key >> shift) & dmask;
+    const unsigned peers = __match_any_sync(act, dg);
+    if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[dg], static_cast<uint32_t>(__popc(peers)));
+  }
+}
+
+__global__ void __launch_bounds__(kStrThreads) index_select_stream_kernel(IndexParams p) {
+  __shared__ uint32_t s_h[kBinsA];          // digit histograms (A, then B, then C)
+  __shared__ uint32_t s_cand[kStrCandCap];  // keys of the threshold bin of digit A
+  __shared__ int s_w[32];
+  __shared__ uint32_t s_res[3];
+  __shared__ int s_n;
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+  const int k = p.k;
+  if (tid == 0) s_res[0] = s_res[1] = s_res[2] = 0u;
+  grid_dependency_wait();  // the scores (and the histogram, if any) come from the scan
+  grid_dependents_launch();
+  int64_t nv64 = query_visible(p, b);
+  if (nv64 < 0) nv64 = 0;
+  const int nv = static_cast<int>(nv64);
+  const float* sc = p.scores + (int64_t)b * p.vis_stride;
+  int32_t* oidx = p.out_idx + (int64_t)b * k;
+  float* osc = p.out_scores ? p.out_scores + (int64_t)b * k : nullptr;
+  if (nv <= k) {  // everything visible is chosen
+    for (int i = tid; i < k; i += kStrThreads) {
+      oidx[i] = i < nv ? i : -1;
+      if (osc) osc[i] = i < nv ? sc[i] : 0.f;
+    }
+    if (tid == 0) p.out_cnt[b] = nv;
+    return;
+  }
+  // one 4-key group per thread and step; the row is 256-byte aligned, the last 0..3 keys go alone
+  const int n4 = nv >> 2;
+  auto keys4 = [&](int g, uint32_t (&kk)[4], unsigned& valid) {
+    if (g < n4) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(sc) + g);
+      kk[0] = f2key(v.x); kk[1] = f2key(v.y); kk[2] = f2key(v.z); kk[3] = f2key(v.w);
+      valid = 15u;
+    } else {
+      valid = 0u;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = 4 * g + e;
+        kk[e] = i < nv ? f2key(sc[i]) : 0u;
+        valid |= (i < nv ? 1u : 0u) << e;
+      }
+    }
+  };
+  const int n_groups = (nv + 3) >> 2;
+  const int n_steps = (n_groups + kStrThreads - 1) / kStrThreads;
+
+  // digit A (bits 31..21)
+  uint32_t dA = 0u;
+  int krem = k, nA = 0;
+  if (p.hist) {
+    const uint32_t* gh = p.hist + (int64_t)b * kBinsA;
+    find_digit_str(kBinsA, k, [&](int bin) { return static_cast<int>(gh[bin]); }, s_w, s_res, dA, krem, nA);
+  } else {
+    for (int i = tid; i < kBinsA; i += kStrThreads) s_h[i] = 0u;
+    __syncthreads();
+    for (int s = 0; s < n_steps; ++s) {
+      const int g = s * kStrThreads + tid;
+      uint32_t kk[4];
+      unsigned valid = 0u;
+      if (g < n_groups) keys4(g, kk, valid);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) str_count(kk[e], (valid >> e) & 1u, 0u, 0u, 21, kBinsA - 1, s_h);
+    }
+    __syncthreads();
+    find_digit_str(kBinsA, k, [&](int bin) { return static_cast<int>(s_h[bin]); }, s_w, s_res, dA, krem, nA);
+  }
+  uint32_t prefix = dA << 21, mask = 0xFFE00000u;
+  uint32_t dB = 0u, dC = 0u;
+  int nB = 0, nC = 0;
+  if (nA <= kStrCandCap) {
+    // the keys of bin dA into shared memory, then digits B and C over that list
+    if (tid == 0) s_n = 0;
+    __syncthreads();
+    const unsigned below = (1u << lane) - 1u;
+    for (int s = 0; s < n_steps; ++s) {
+      const int g = s * kStrThreads + tid;
+      uint32_t kk[4];
+      unsigned valid = 0u;
+      if (g < n_groups) keys4(g, kk, valid);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool cand = ((valid >> e) & 1u) && (kk[e] & mask) == prefix;
+        const unsigned m = __ballot_sync(kFull, cand);
+        if (m) {
+          int at = 0;
+          if (lane == __ffs(m) - 1) at = atomicAdd(&s_n, __popc(m));
+          at = __shfl_sync(kFull, at, __ffs(m) - 1) + __popc(m & below);
+          if (cand && at < kStrCandCap) s_cand[at] = kk[e];
+        }
+      }
+    }
+    for (int i = tid; i < kBinsB; i += kStrThreads) s_h[i] = 0u;
+    __syncthreads();
+    const int nc = s_n < kStrCandCap ? s_n : kStrCandCap;
+    for (int i = tid; i < nc; i += kStrThreads)
+      if ((s_cand[i] & mask) == prefix) atomicAdd(&s_h[(s_cand[i] >> 10) & (kBinsB - 1)], 1u);
+    __syncthreads();
+    find_digit_str(kBinsB, krem, [&](int bin) { return static_cast<int>(s_h[bin]); }, s_w, s_res, dB, krem, nB);
+    prefix |= dB << 10;
+    mask |= 0x001FFC00u;
+    for (int i = tid; i < kBinsC; i += kStrThreads) s_h[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < nc; i += kStrThreads)
+      if ((s_cand[i] & mask) == prefix) atomicAdd(&s_h[s_cand[i] & (kBinsC - 1)], 1u);
+    __syncthreads();
+    find_digit_str(kBinsC, krem, [&](int bin) { return static_cast<int>(s_h[bin]); }, s_w, s_res, dC, krem, nC);
+  } else {
+    // a threshold bin too large for the list: masked histogram passes over the scores
+    for (int round = 0; round < 2; ++round) {
+      const int shift = round == 0 ? 10 : 0;
+      const int nb = round == 0 ? kBinsB : kBinsC;
+      for (int i = tid; i < nb; i += kStrThreads) s_h[i] = 0u;
+      __syncthreads();
+      for (int s = 0; s < n_steps; ++s) {
+        const int g = s * kStrThreads + tid;
+        uint32_t kk[4];
+        unsigned valid = 0u;
+        if (g < n_groups) keys4(g, kk, valid);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) str_count(kk[e], (valid >> e) & 1u, mask, prefix, shift, nb - 1, s_h);
+      }
+      __syncthreads();
+      uint32_t d = 0u;
+      int cnt = 0;
+      find_digit_str(nb, krem, [&](int bin) { return static_cast<int>(s_h[bin]); }, s_w, s_res, d, krem, cnt);
+      if (round == 0) {
+        dB = d;
+        prefix |= dB << 10;
+        mask |= 0x001FFC00u;
+      } else {
+        dC = d;
+      }
+    }
+  }
+  const uint32_t T = prefix | dC;  // the k-th largest key; the first krem keys equal to T are taken
+
+  // ordered output: per step, one scan of (keys above T, keys equal to T) packed in one int
+  int written = 0, eq_seen = 0;
+  for (int s = 0; s < n_steps; ++s) {
+    const int g = s * kStrThreads + tid;
+    uint32_t kk[4];
+    unsigned valid = 0u;
+    if (g < n_groups) keys4(g, kk, valid);
+    int ngt = 0, neq = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      ngt += ((valid >> e) & 1u) && kk[e] > T;
+      neq += ((valid >> e) & 1u) && kk[e] == T;
+    }
+    int tot;
+    const int ex = block_exclusive_scan<kStrThreads>(ngt | (neq << 16), s_w, tot);
+    const int gt_ex = ex & 0xFFFF, eq_ex = ex >> 16;
+    const int rem = krem - eq_seen > 0 ? krem - eq_seen : 0;  // equal keys still to take
+    int pos = written + gt_ex + (eq_ex < rem ? eq_ex : rem);
+    int eq_rank = eq_ex;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (!((valid >> e) & 1u)) continue;
+      bool take = kk[e] > T;
+      if (kk[e] == T) {
+        take = eq_rank < rem;
+        ++eq_rank;
+      }
+      if (take && pos < k) {
+        oidx[pos] = 4 * g + e;
+        if (osc) osc[pos] = key2f(kk[e]);
+        ++pos;
+      }
+    }
+    const int tot_gt = tot & 0xFFFF, tot_eq = tot >> 16;
+    written += tot_gt + (tot_eq < rem ? tot_eq : rem);
+    eq_seen += tot_eq;
+  }
+  if (tid == 0) p.out_cnt[b] = k;
+}
+
+cudaError_t launch_select_stream(IndexParams& p, cudaStream_t st) {
+  return launch_pdl(index_select_stream_kernel, dim3(static_cast<unsigned>(p.n_q)), dim3(kStrThreads), 0, st, p);
+}
+
 }  // namespace
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link)
@@ -1324,7 +1554,8 @@ cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st) {
   // many queries in one call (a prefill chunk): the grouped scan reads each key once per group
   const bool grouped = tma_ok && p.n_q >= kGroupScanMinQueries && (p.n_heads_idx == 4 || p.n_heads_idx == 8);
   if (nv_max > 0 && grouped) {
-    if (p.d_idx == 64 && p.n_heads_idx == 4) e = launch_scan_group<2, 4>(p, n_sm, st);
+    if (scan_tc_supported(p)) e = launch_scan_tc(p, n_sm, st);
+    else if (p.d_idx == 64 && p.n_heads_idx == 4) e = launch_scan_group<2, 4>(p, n_sm, st);
     else if (p.d_idx == 64) e = launch_scan_group<2, 8>(p, n_sm, st);
     else if (p.n_heads_idx == 4) e = launch_scan_group<4, 4>(p, n_sm, st);
     else e = launch_scan_group<4, 8>(p, n_sm, st);
@@ -1349,6 +1580,9 @@ cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st) {
     else return cudaErrorNotSupported;
     if (e != cudaSuccess) return e;
   }
+  if (p.n_q == 0) return cudaSuccess;
+  // many queries (a prefill block): one small CTA per query, several per SM
+  if (p.n_q >= kStreamSelectMinQueries) return launch_select_stream(p, st);
   // selection: a cluster of CL CTAs per query, each holding a slice of scores
   int cl_min = static_cast<int>((nv_max + kSliceCap - 1) / kSliceCap);
   if (cl_min < 1) cl_min = 1;
