@@ -1,88 +1,89 @@
 // attend_tc.cu -- CSA / HCA core attention on the 5th-generation tensor cores
 // (tcgen05) for the wide shared latent: d_qk = 576 (512 latent + 64 RoPE
-// channels), d_v = 512, query heads in groups of 128 (DeepSeek-V4 report
+// channels), d_v = 512, query heads in groups of 64 (DeepSeek-V4 report
 // digest, section 3: one softmax over the window and the selected / all
 // compressed entries; DeepSeek-V4-book ch.1, section 4: the MLA latent shared
 // by every head).
 //
 // With 128 heads on one 576-wide latent every key carries 2 x 128 x 1088
-// flops against 1152 bytes: the product sits at the B200's ridge point, so the
-// kernel must stream keys at HBM speed and keep the tensor core busy at once.
-// Work item = (query, 128-head group, key split), run by a cluster of two CTAs
-// that split the key channels:
-//   rank 0 holds Q channels 0..319 and loads key channels 0..319;
-//   rank 1 holds Q channels 320..575 and loads key channels 256..575;
-// each computes a partial S = Q K^T over its channels (heads as M = 128, 32
-// keys as N) in tensor memory, sends it to the other CTA through distributed
-// shared memory and adds the one it receives, so both hold the full S and run
-// the same online softmax (fp32; identical results, since a + b == b + a).
-// Each then accumulates O for its half of d_v: O[:, 256 r .. 256 r + 255] +=
-// P V, with P (bf16) as the tensor-memory A operand and V read MN-major from
-// the first four channel blocks of its key tile (V = the first d_v channels of
-// every key). No tensor work is duplicated. Each CTA keeps its last three Q
-// blocks in tensor memory (an MMA's A operand may come from there) and the
-// rest in shared memory, which leaves room for five key-tile stages and the
-// exchange buffers, so the loads run well ahead of the math.
-//   - key tiles arrive by TMA when their rows are contiguous (window rows of
-//     the ring, HCA entries of one page), by cp.async through a row table
-//     otherwise (the CSA selection);
-//   - each thread of the softmax warpgroup owns one head row; it sends tile
-//     t + 1's partial (asynchronous stores counted on the receiver's
-//     mbarrier) before it waits for tile t's, hiding the exchange;
-//   - O is rescaled only when a row's running max rises by more than 2^8 (the
-//     probabilities stay below 256 in bf16), so most tiles skip it.
-// Window keys are taken in ring-slot order (the softmax does not depend on the
-// order of its keys), which makes a window tile 32 consecutive ring rows. Each
-// item writes its normalised partial output and log-sum-exp;
-// attend_merge_kernel combines the splits.
-#include <cooperative_groups.h>
-
+// flops against 1152 bytes, at the B200's ridge point. O for 128 heads x 512
+// channels in fp32 would fill a whole SM's tensor memory, so a work item =
+// (query, 64-head group, key split): the two head groups of a split run on two
+// CTAs that read the same key tiles (the second read is served by L2) and never
+// talk to each other. Per CTA, everything is local:
+//   - S = Q K^T with the 64 heads as M and a 64-key tile as N, Q (64 x 576) and
+//     the key tile (64 x 576) in shared memory; the channel blocks alternate
+//     between two accumulators (a tcgen05.mma that accumulates into the tile of
+//     the one before it waits for it, ~90 cycles per step, while two chains run
+//     at the operand rate), the even blocks at tensor-memory lane offset 0 and
+//     the odd ones at lane offset 16 of the same columns (an M = 64 accumulator
+//     fills lanes 0-15 of each 32-lane quarter);
+//   - O = P V in two halves of 256 channels, O[:, 0:256] at lane offset 0 and
+//     O[:, 256:512] at lane offset 16 of columns 0-255, P (bf16) in shared
+//     memory as the A operand, V read MN-major from the key tile (V = the first
+//     d_v channels of every key);
+//   - thread (warp w, lane l) of the softmax warpgroup owns head row 16 w +
+//     (l & 15) and keys 32 (l >> 4) .. + 31 of each tile: it reads its lane's
+//     accumulator, swaps 32 values with lane l ^ 16 to form the full S of its
+//     keys, and the row max is one more swap; the two lanes of a row keep the
+//     same running max, and the rare O rescale touches exactly the O rows of
+//     every lane (both halves);
+//   - one warp issues only S, so the next tile's S runs while this tile's
+//     exponentials are taken; softmax thread 0 issues the tile's P V once every
+//     row has stored its P (a named barrier that also decides aborts uniformly);
+//   - loaders look up each tile's source rows just before its copy: TMA when a
+//     tile's rows are contiguous (window rows of the ring, HCA entries of one
+//     page), cp.async through the looked-up rows otherwise (the CSA selection),
+//     FP8 entries widened exactly to bf16.
+// O is rescaled only when a row's running max rises by more than 2^8 (the
+// probabilities stay below 256 in bf16), so most tiles skip it. Window keys are
+// taken in ring-slot order (the softmax does not depend on the order of its
+// keys), which makes a window tile 64 consecutive ring rows. Each item writes
+// its normalised partial output and log-sum-exp; attend_merge_t_kernel combines
+// the splits.
 #include "cskv_device.cuh"
 #include "cskv_internal.h"
-
-namespace cg = cooperative_groups;
 
 namespace cskv {
 namespace {
 
-constexpr int kDqk = 576, kDv = 512, kM = 128, kNk = 32;
-constexpr int kNb = 5;                         // 64-channel blocks of a key row loaded by each CTA
-constexpr int kStageBytes = kNb * kNk * 128;   // 20480 per key-tile stage
-// Q blocks of a CTA: the first kQSmem (rank 0: 2, rank 1: 1) in shared memory,
-// the last three in tensor memory (the A operand of an MMA may come from either)
-constexpr int kQTmem = 3;
-constexpr int kQBytes = 2 * kM * 128;          // 32768
-constexpr int kNS = 5;                         // key-tile stages
-constexpr int kRecvBytes = kM * kNk * 4;       // one partial S tile from the other CTA
-constexpr int kThreads = 256;                  // warps 0-3 softmax, warp 4 MMA, warps 5-7 loads
-constexpr int kMmaThread = 128;
+constexpr int kDqk = 576, kDv = 512, kH = 64, kNk = 64;
+constexpr int kNb = kDqk / 64;                  // 9 channel blocks of a key row
+constexpr int kBlkBytes = kNk * 128;            // 8192: one channel block of a 64-row tile
+constexpr int kStageBytes = kNb * kBlkBytes;    // 73728: a key tile (also the Q block set)
+constexpr int kNS = 2;                          // key-tile stages
+constexpr int kPBytes = kH * kNk * 2;           // 8192: P of the tile (bf16)
+constexpr int kThreads = 256;                   // warps 0-3 softmax, warp 4 S, warps 5-7 loads
 constexpr int kLoadThread0 = 160;
 constexpr int kLoaders = kThreads - kLoadThread0;  // 96
-constexpr int kRowCap = 1024;                  // keys per work item (row table in shared memory)
+constexpr int kChunks = kNk * kNb * 8;          // 16-byte chunks of a bf16 tile (4608)
+constexpr int kPer = (kChunks + kLoaders - 1) / kLoaders;  // 48
 constexpr uint32_t kTmemCols = 512;
-// O 256 | S 3 buffers x 32 | P 3 buffers x 16 (bf16 pairs) | Q 3 blocks x 32 (bf16 pairs)
-constexpr int kNSP = 3;  // S and P buffers
-constexpr uint32_t kColO = 0, kColS = 256, kColP = kColS + kNSP * 32, kColQ = kColP + kNSP * 16;
-static_assert(kColQ + kQTmem * 32 <= kTmemCols, "tensor memory budget");
+// O[:, 0:256] lanes +0 and O[:, 256:512] lanes +16 of columns 0-255; S buffer k at columns
+// 256 + 64 k (even channel blocks at lanes +0, odd ones at lanes +16)
+constexpr uint32_t kColO = 0, kColS = 256;
+constexpr uint32_t kLane16 = 16u << 16;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleThreshold = 8.0f;      // log2 units
-constexpr int kPrefetchTiles = 6;              // L2 prefetch distance of gathered key rows
+constexpr float kRescaleThreshold = 8.0f;       // log2 units
 
 struct Smem {
-  static constexpr int Q = 0;
-  static constexpr int K = kQBytes;                     // kNS stages (also the epilogue staging)
-  static constexpr int RECV = K + kNS * kStageBytes;    // two slots of the other CTA's partial S
-  static constexpr int SEND = RECV + 2 * kRecvBytes;    // two slots of this CTA's partial S on its way out
-  static constexpr int BAR = SEND + 2 * kRecvBytes;     // mbarriers
-  static constexpr int MASK = BAR + 256;                // valid-key bits, one word per tile
-  static constexpr int ROWS = MASK + kRowCap / 8;       // source row of every key of the item
-  static constexpr int SCALE = ROWS + kRowCap * 8;      // FP8 entries: the per-entry scale of every key
-  static constexpr int TMEM = SCALE + kRowCap * 4;      // allocated tensor-memory address
+  static constexpr int Q = 0;                          // 9 blocks of 64 heads x 128 B
+  static constexpr int K = Q + kStageBytes;            // kNS key tiles
+  static constexpr int P = K + kNS * kStageBytes;      // P of the tile (64 rows x 128 B)
+  static constexpr int CODE = P + kPBytes;             // [kNS][kNk] source-row codes of a stage's keys
+  static constexpr int SCALE = CODE + kNS * kNk * 4;   // [kNS][kNk] FP8 scale of each key (1 for bf16 rows)
+  static constexpr int MASK = SCALE + kNS * kNk * 4;   // [kNS][2] valid-key bits
+  static constexpr int BAR = MASK + 32;                // mbarriers
+  static constexpr int TMEM = BAR + 16 * 8;            // allocated tensor-memory address
   static constexpr int FLAGS = TMEM + 16;
-  static constexpr int PREF = FLAGS + 16;
+  static constexpr int PREF = FLAGS + 16;              // [n_q + 1] items per query, exclusive prefix
   static size_t bytes(int n_q) { return 1024 + PREF + sizeof(int) * (size_t)(n_q + 1); }
 };
+
+// source-row code: kind in bits [31:30] (0 none, 1 pool entry, 2 ring row, 3 chunk row), row below
+constexpr uint32_t kRowBits = 30;
+constexpr uint32_t kRowMask = (1u << kRowBits) - 1u;
 
 struct Keys {
   int64_t t, ws;
@@ -110,32 +111,34 @@ __device__ __forceinline__ Keys keys_of(const AttendParams& p, int b) {
   return r;
 }
 
-// Source row of key u. Window keys come first: in ring-slot order (slot u)
-// when every window row is in the ring, in position order when a prefill chunk
-// supplies some of them; then the compressed entries (bf16 rows, or FP8 rows
-// with their scale in `sc`). Null if invalid.
-__device__ __forceinline__ const void* key_src(const AttendParams& p, int b, int seq, const Keys& k, int64_t u,
-                                               float& sc) {
-  sc = 1.f;
+// Code of the source row of key u: window keys first, in ring-slot order (slot
+// u) when every window row is in the ring, in position order when a prefill
+// chunk supplies some of them; then the compressed entries. 0 if invalid.
+__device__ __forceinline__ uint32_t key_code(const AttendParams& p, int b, int seq, const Keys& k, int64_t u) {
   if (u < k.n_w) {
-    if (!p.x_chunk) return p.ring_x + ((int64_t)seq * p.n_win + u) * kDqk;
+    if (!p.x_chunk) return (2u << kRowBits) | static_cast<uint32_t>((int64_t)seq * p.n_win + u);
     const int64_t pos = k.ws + u;
-    if (pos >= p.chunk_pos0 && pos < p.chunk_pos0 + p.chunk_len) return p.x_chunk + (pos - p.chunk_pos0) * kDqk;
-    return p.ring_x + ((int64_t)seq * p.n_win + pos % p.n_win) * kDqk;
+    if (pos >= p.chunk_pos0 && pos < p.chunk_pos0 + p.chunk_len)
+      return (3u << kRowBits) | static_cast<uint32_t>(pos - p.chunk_pos0);
+    return (2u << kRowBits) | static_cast<uint32_t>((int64_t)seq * p.n_win + pos % p.n_win);
   }
   const int64_t jj = u - k.n_w;
   const int64_t j = p.is_csa ? static_cast<int64_t>(p.sel_idx[(int64_t)b * p.k + jj]) : jj;
-  if (j < 0 || j >= visible_entries(k.t, p.m, p.n_win)) return nullptr;
+  if (j < 0 || j >= visible_entries(k.t, p.m, p.n_win)) return 0;
   const int64_t pi = j / p.page_size;
-  if (pi >= p.max_pages_per_seq) return nullptr;
+  if (pi >= p.max_pages_per_seq) return 0;
   const int32_t page = p.page_table[(int64_t)seq * p.max_pages_per_seq + pi];
-  if (page < 0 || page >= p.n_pages) return nullptr;
-  const int64_t row = (int64_t)page * p.page_size + j % p.page_size;
-  if (p.kv_dtype == CSKV_FP8_E4M3) {
-    sc = p.kv_scale[row];
-    return static_cast<const uint8_t*>(p.kv_pool) + row * kDqk;
-  }
-  return static_cast<const uint16_t*>(p.kv_pool) + row * kDqk;
+  if (page < 0 || page >= p.n_pages) return 0;
+  return (1u << kRowBits) | static_cast<uint32_t>((int64_t)page * p.page_size + j % p.page_size);
+}
+
+// the bf16 row of a code (an FP8 pool row is read as codes by the loaders)
+__device__ __forceinline__ const uint16_t* code_row(const AttendParams& p, uint32_t c) {
+  const uint32_t kind = c >> kRowBits, row = c & kRowMask;
+  if (kind == 1) return static_cast<const uint16_t*>(p.kv_pool) + (size_t)row * kDqk;
+  if (kind == 2) return p.ring_x + (size_t)row * kDqk;
+  if (kind == 3) return p.x_chunk + (size_t)row * kDqk;
+  return nullptr;
 }
 
 // 8 E4M3 codes -> 8 bf16 (exact: every E4M3 value is a bf16 value)
@@ -151,77 +154,45 @@ __device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 c) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// byte offset of 16-byte chunk `ch` of row `r` in a swizzled block set whose
-// 64-channel (128-byte) blocks are `block_bytes` apart
-__device__ __forceinline__ uint32_t swz(int r, int ch, int block_bytes) {
-  return (ch >> 3) * block_bytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
-}
-
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
 }
-
-// ---------------------------------------------------------------- cluster helpers
-__device__ __forceinline__ uint32_t cluster_rank() {
+// named barrier over n threads that also returns the OR of `v` over them (the same in every thread)
+__device__ __forceinline__ bool named_sync_or(int id, int n, bool v) {
   uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
-  return r;
+  asm volatile(
+      "{\n .reg .pred q, p;\n setp.ne.u32 q, %1, 0;\n bar.red.or.pred p, %2, %3, q;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(r)
+      : "r"(v ? 1u : 0u), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
 }
-// shared::cluster address of `local` in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t peer_addr(const void* local, uint32_t rank) {
-  uint32_t a;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(a) : "r"(smem_u32(local)), "r"(rank));
-  return a;
-}
-__device__ __forceinline__ void st_peer_u32(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;\n" ::"r"(addr), "r"(v) : "memory");
-}
-// arrive on an mbarrier of another CTA (after this thread's reads of the slot
-// it frees; the other CTA only writes into that slot again after seeing it)
-__device__ __forceinline__ void mbar_arrive_peer(uint32_t addr) {
-  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];\n" ::"r"(addr) : "memory");
-}
-// bulk copy (by the TMA engine) of `bytes` from this CTA's shared memory into
-// another CTA's, counted as transaction bytes on that CTA's mbarrier (dst and
-// mbar are shared::cluster addresses). The source may be rewritten once that
-// mbarrier's phase has completed.
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
-  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-                   dst),
-               "r"(smem_u32(src)), "r"(bytes), "r"(mbar)
-               : "memory");
-}
-// Partial S of one key tile: NB channel blocks, the first NQS with Q in shared memory, the rest
-// with Q in tensor memory; fully unrolled, every descriptor built from its 32-bit address (the
-// constant upper half then folds away, which keeps the issue loop short).
-template <int NB, int NQS>
-__device__ __forceinline__ void issue_s(uint32_t d, uint32_t q_smem, uint32_t q_tmem, uint32_t k_smem,
-                                        uint32_t idesc) {
+
+// S of one key tile: 9 channel blocks x 4 K-steps (M = 64 heads, N = 64 keys); even blocks
+// accumulate at d (lanes +0), odd blocks at d + 16 lanes, the two chains issued alternately
+__device__ __forceinline__ void issue_s(uint32_t d, uint32_t q, uint32_t k, uint32_t idesc) {
 #pragma unroll
-  for (int k = 0; k < 4 * NB; ++k) {
-    const int j = k >> 2, ks = k & 3;
-    const uint64_t db = umma_desc_sw128(k_smem + j * (kNk * 128) + ks * 32, 16, 1024);
-    if (j < NQS)
-      umma_ss(d, umma_desc_sw128(q_smem + j * (kM * 128) + ks * 32, 16, 1024), db, idesc, k > 0 ? 1u : 0u);
-    else
-      umma_ts(d, q_tmem + (j - NQS) * 32 + ks * 8, db, idesc, k > 0 ? 1u : 0u);
+  for (int s = 0; s < 20; ++s) {
+    const int ia = 2 * (s >> 2), ks = s & 3;
+    umma_ss(d, umma_desc_sw128(q + ia * kBlkBytes + ks * 32, 16, 1024),
+            umma_desc_sw128(k + ia * kBlkBytes + ks * 32, 16, 1024), idesc, s > 0 ? 1u : 0u);
+    if (s < 16) {
+      const int ib = ia + 1;
+      umma_ss(d + kLane16, umma_desc_sw128(q + ib * kBlkBytes + ks * 32, 16, 1024),
+              umma_desc_sw128(k + ib * kBlkBytes + ks * 32, 16, 1024), idesc, s > 0 ? 1u : 0u);
+    }
   }
 }
 
-// Pipeline (per CTA; tiles numbered gt across the items of the cluster, the
-// same in both CTAs; stage gt % kNS, S / P buffer gt % 3, exchange slot gt & 1):
-//   loaders  : wait kempty (P V of tile gt - kNS done) -> TMA, or cp.async +
-//              proxy fence, into the stage -> kfull
-//   MMA      : wait kfull -> partial S(gt) -> commit sfull; then wait pfull of
-//              tile gt - 2 -> O += P V -> commit kempty, obar
-//   softmax  : wait sfull(gt + 1) -> send its partial to the other CTA (async
-//              stores that count bytes on the receiver's rfull); wait rfull(gt)
-//              -> S(gt) = own + received -> free the slot (remote rempty) ->
-//              P(gt) (+ rare O rescale after P V of tile gt - 1) -> arrive pfull
-// S(gt) needs the softmax only up to tile gt - 3 and the softmax needs S only
-// one tile ahead, so neither waits on the other's latest step.
-// FP8: the pool holds E4M3 entries with an fp32 scale each (a separate instantiation keeps
-// the bf16 kernel's code, and so its instruction-cache footprint, small)
+// Pipeline (per CTA; tiles numbered gt across its items; stage and S buffer gt & 1):
+//   loaders : look up the tile's source rows -> wait kempty (P V of tile gt - 2 done) ->
+//             TMA, or cp.async / widened FP8 stores, into the stage -> kfull
+//   S warp  : wait kfull, sfree (softmax has read S(gt - 2)) -> S(gt) -> commit sfull
+//   softmax : wait sfull -> read S, swap halves with lane ^ 16, arrive sfree -> P(gt) ->
+//             wait obar (P V of gt - 1 done: P buffer free, O settled; rare rescale) ->
+//             store P -> named barrier -> thread 0: O += P V(gt) -> commit kempty, obar
+// FP8: the pool holds E4M3 entries with an fp32 scale each (a separate
+// instantiation keeps the bf16 kernel's code small)
 template <bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ring,
@@ -230,54 +201,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = sm + Smem::Q;
   uint8_t* sK = sm + Smem::K;
-  uint8_t* sRecv = sm + Smem::RECV;
-  uint8_t* sSend = sm + Smem::SEND;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Smem::BAR);
-  uint64_t* kfull = bars;             // [kNS] loaders -> MMA
-  uint64_t* kempty = bars + kNS;      // [kNS] MMA -> loaders (commit)
-  uint64_t* sfull = bars + 2 * kNS;   // [3] MMA -> softmax (commit)
-  uint64_t* pfull = sfull + kNSP;     // [3] softmax -> MMA (128 arrivals)
-  uint64_t* obar = pfull + kNSP;      // [3] MMA -> softmax (commit after the P V of that P buffer)
-  uint64_t* rfull = obar + kNSP;      // [2] other CTA's partial S landed (one arrival + 16 KB of bytes)
-  uint64_t* rempty = rfull + 2;       // [2] other CTA has read what this one sent (4 remote arrivals)
-  uint64_t* qbar = rempty + 2;        //     Q landed (TMA)
-  uint64_t* dbar = qbar + 1;          //     MMA -> epilogue (commit after the item's last P V)
-  uint32_t* sMask = reinterpret_cast<uint32_t*>(sm + Smem::MASK);
-  const void** sRow = reinterpret_cast<const void**>(sm + Smem::ROWS);
+  uint8_t* sP = sm + Smem::P;
+  uint32_t* sCode = reinterpret_cast<uint32_t*>(sm + Smem::CODE);
   float* sScale = reinterpret_cast<float*>(sm + Smem::SCALE);
+  uint32_t* sMask = reinterpret_cast<uint32_t*>(sm + Smem::MASK);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Smem::BAR);
+  uint64_t* kfull = bars;             // [2] loaders -> S warp (and the softmax, for the stage's key bits)
+  uint64_t* kempty = bars + 2;        // [2] P V of the stage's tile done (commit)
+  uint64_t* sfull = bars + 4;         // [2] S of the buffer's tile done (commit)
+  uint64_t* sfree = bars + 6;         // [2] softmax has read the buffer (128 arrivals)
+  uint64_t* obar = bars + 8;          //     a tile's P V done (commit)
+  uint64_t* qbar = bars + 9;          //     Q of the item landed (TMA)
+  uint64_t* dbar = bars + 10;         //     the item's last P V done (commit)
   constexpr bool fp8 = FP8;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + Smem::TMEM);
   volatile int* sAbort = reinterpret_cast<int*>(sm + Smem::FLAGS);
-  volatile int* sLdOk = reinterpret_cast<int*>(sm + Smem::FLAGS) + 1;  // [2] loader wait results, then [1] send flag
+  volatile int* sLdOk = reinterpret_cast<int*>(sm + Smem::FLAGS) + 1;
   int* sPref = reinterpret_cast<int*>(sm + Smem::PREF);
   __shared__ int s_wsum[32];
 
-  cg::cluster_group cluster = cg::this_cluster();
-  const uint32_t rank = cluster_rank(), peer = rank ^ 1u;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int groups = p.n_heads / kM;
+  const int groups = p.n_heads / kH;
   const int kps = p.keys_per_split;
-  const int kb_load0 = rank ? 4 : 0;  // first 64-channel block of the key rows this CTA loads
-  const int n_sblk = rank ? 4 : 5;    // blocks of its S partial (Q blocks 0.. of this CTA)
-  const int n_qs = n_sblk - kQTmem;   // of which in shared memory
-  const int qkb0 = rank ? 5 : 0;      // channel block of its Q block 0
-  const int s_blk0 = rank ? 1 : 0;    // first S block inside a stage (blocks 0..3 are V)
 
   if (tid == 0) {
-    for (int i = 0; i < kNS; ++i) {
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&kfull[i], 1);
       mbar_init(&kempty[i], 1);
-    }
-    for (int i = 0; i < kNSP; ++i) {
       mbar_init(&sfull[i], 1);
-      mbar_init(&pfull[i], kM);
-      mbar_init(&obar[i], 1);
+      mbar_init(&sfree[i], 128);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&rfull[i], 1);
-      mbar_init(&rempty[i], 4);
-    }
-    mbar_init(qbar, 1 + kM);  // the TMA's arrival and one per softmax thread (tensor-memory blocks)
+    mbar_init(obar, 1);
+    mbar_init(qbar, 1);
     mbar_init(dbar, 1);
     fence_barrier_init();
     *sAbort = 0;
@@ -292,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  cluster.sync();  // barriers of both CTAs initialised before any remote arrival
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *sTmem;
   // the set-up above overlaps the tail of the kernel launched before this one; its
@@ -320,11 +275,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = tid; b < p.n_q; b += kThreads)
       if (p.q_pos[b] < 0 || p.q_pos[b] > p.max_pos) report(p.status, CSKV_ERR_INVALID_ARG);
   const int total = sPref[p.n_q];
-  const int n_clusters = gridDim.x / 2;
-  uint32_t g = 0;       // tiles processed by this cluster before the current item
+  uint32_t g = 0;       // tiles processed by this CTA before the current item
   uint32_t n_item = 0;  // items processed before the current one (qbar / dbar phase)
 
-  for (int item = blockIdx.x / 2; item < total; item += n_clusters, ++n_item) {
+  // consecutive items are the head groups of one split, so the CTAs reading the same keys run together
+  for (int item = blockIdx.x; item < total; item += gridDim.x, ++n_item) {
     int lo = 0, hi = p.n_q - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -340,44 +295,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t u0 = (int64_t)split * kps;
     const int nk = static_cast<int>(kk.n - u0 < kps ? kk.n - u0 : kps);
     const int ntiles = (nk + kNk - 1) / kNk;
-
-    // source rows of this item's keys and one valid-bit word per tile, visible
-    // to every role after the barrier; four independent lookups per thread
-    for (int i0 = 0; i0 < ntiles * kNk; i0 += 4 * kThreads) {
-      const void* src[4];
-      float sc[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int i = i0 + q * kThreads + tid;
-        sc[q] = 0.f;
-        src[q] = (i < nk && seq_ok) ? key_src(p, b, seq, kk, u0 + i, sc[q]) : nullptr;
-      }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int i = i0 + q * kThreads + tid;
-        if (i < nk) {
-          if (!src[q] && rank == 0) report(p.status, CSKV_ERR_OUT_OF_RANGE);
-          sRow[i] = src[q];
-        }
-        if (i < ntiles * kNk) sScale[i] = src[q] ? sc[q] : 0.f;  // finite for every slot of every tile
-        const unsigned bits = __ballot_sync(kFull, src[q] != nullptr);
-        if (lane == 0 && i < ntiles * kNk) sMask[i >> 5] = bits;
-      }
-    }
-    __syncthreads();
+    if (tid == 0 && grp == 0 && !seq_ok && kk.n > 0) report(p.status, CSKV_ERR_OUT_OF_RANGE);
 
     if (tid >= kLoadThread0) {
       // ------------------------------------------------------------ loaders
-      const int lt = tid - kLoadThread0;
-      if (lt == 0) {  // this CTA's shared-memory Q blocks of the head group: 128-row TMA boxes
-        mbar_arrive_expect_tx(qbar, n_qs * kM * 128);
-        const int qrow = b * p.n_heads + grp * kM;
-        for (int j = 0; j < n_qs; ++j) tma_load_2d(sQ + j * (kM * 128), &tm_q, (qkb0 + j) * 64, qrow, qbar);
+      const int lt = tid - kLoadThread0, lw = lt >> 5, ll = lt & 31;
+      if (lw == 0) {  // Q of the head group: 9 boxes of 64 rows x 64 channels
+        if (ll == 0) {
+          mbar_arrive_expect_tx(qbar, kStageBytes);
+          const int qrow = b * p.n_heads + grp * kH;
+          for (int j = 0; j < kNb; ++j) tma_load_2d(sQ + j * kBlkBytes, &tm_q, j * 64, qrow, qbar);
+        }
+        __syncwarp();
       }
-      // TMA source of tile it: 0 = ring rows, 1 = pool rows, -1 = gathered (cp.async)
+      // TMA source of tile it: 0 = ring rows, 1 = pool rows (row0 set), -1 = looked-up rows
       auto tile_src = [&](int it, int& row0) -> int {
         const int64_t a = u0 + (int64_t)it * kNk;
-        if (!seq_ok) return -1;
+        if (!seq_ok || (it + 1) * kNk > nk) return -1;  // a partial tile: rows past its end are not zero
         if (!p.x_chunk && a + kNk <= kk.n_w) {
           row0 = static_cast<int>((int64_t)seq * p.n_win + a);
           return 0;
@@ -385,8 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!p.is_csa && !fp8 && a >= kk.n_w) {
           const int64_t j0 = a - kk.n_w;
           const int64_t pi = j0 / p.page_size;
-          // whole tile inside one page and inside the item (rows past the end are not zero)
-          if (j0 % p.page_size + kNk > p.page_size || pi >= p.max_pages_per_seq || (it + 1) * kNk > nk) return -1;
+          if (j0 % p.page_size + kNk > p.page_size || pi >= p.max_pages_per_seq) return -1;
           const int32_t page = p.page_table[(int64_t)seq * p.max_pages_per_seq + pi];
           if (page < 0 || page >= p.n_pages) return -1;
           row0 = static_cast<int>((int64_t)page * p.page_size + j0 % p.page_size);
@@ -394,59 +327,57 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         return -1;
       };
-      auto prefetch_tile = [&](int it) {
-        if (lt < kNk && it < ntiles) {
-          const int i = it * kNk + lt;
-          if (i < nk && sRow[i]) {
-            const bool row8 = fp8 && u0 + i >= kk.n_w;  // FP8 entry (window rows are bf16)
-            prefetch_l2(static_cast<const uint8_t*>(sRow[i]) + kb_load0 * 64 * (row8 ? 1 : 2), kNb * (row8 ? 64 : 128));
-          }
+      // the source row of key lt of tile it (threads 0 .. kNk - 1), and its FP8 scale
+      auto code_of = [&](int it, float& sc) -> uint32_t {
+        sc = 0.f;
+        const int i = it * kNk + lt;
+        if (lt >= kNk || i >= nk || !seq_ok) return 0u;
+        const uint32_t c = key_code(p, b, seq, kk, u0 + i);
+        if (!c) {
+          if (grp == 0) report(p.status, CSKV_ERR_OUT_OF_RANGE);
+          return 0u;
         }
+        sc = (fp8 && (c >> kRowBits) == 1u) ? p.kv_scale[c & kRowMask] : 1.f;
+        return c;
       };
-      const bool gathered_item = p.is_csa || p.x_chunk || fp8;
-      if (gathered_item)
-        for (int it = 0; it < kPrefetchTiles; ++it) prefetch_tile(it);
-      // Gathered tiles are pipelined by one: tile it's loads are issued before tile it-1 is finished
-      // (its FP8 rows widened, its cp.async group waited for) and signalled.
-      constexpr int kItems = kNk * kNb * 8;
-      constexpr int kPer = (kItems + kLoaders - 1) / kLoaders;
-      uint2 pend_codes[kPer];
-      int pend_it = -1;  // gathered tile still to be finished
-      bool stopped = false;  // uniform over the loaders (decided after a named barrier)
-      auto finish = [&](int pit, bool newer_group) {
-        const uint32_t pgt = g + pit;
-        uint8_t* pdst = sK + (pgt % kNS) * kStageBytes;
-        if (fp8) {
-#pragma unroll
-          for (int q = 0; q < kPer; ++q) {
-            const int id = lt + q * kLoaders;
-            if (id < kItems) {
-              const int kr = id / (kNb * 8), c = id % (kNb * 8);
-              const int i = pit * kNk + kr;
-              if (i < nk && sRow[i] && u0 + i >= kk.n_w)
-                *reinterpret_cast<uint4*>(pdst + swz(kr, c, kNk * 128)) = e4m3x8_to_bf16x8(pend_codes[q]);
-            }
-          }
-        }
-        if (newer_group) cp_async_wait<1>(); else cp_async_wait<0>();
-        fence_proxy_async_smem();
-        named_sync(3, kLoaders);
-        if (lt == 0) mbar_arrive(&kfull[pgt % kNS]);
+      auto prefetch = [&](uint32_t c) {  // the row into L2 ahead of its copy
+        if (!c) return;
+        if (fp8 && (c >> kRowBits) == 1u)
+          prefetch_l2(static_cast<const uint8_t*>(p.kv_pool) + (size_t)(c & kRowMask) * kDqk, kDqk);
+        else
+          prefetch_l2(code_row(p, c), kDqk * 2);
       };
+      float nsc = 0.f;
+      uint32_t ncode = ntiles > 0 ? code_of(0, nsc) : 0u;
+      {
+        int rr0;
+        if (ntiles > 0 && tile_src(0, rr0) < 0) prefetch(ncode);
+      }
       for (int it = 0; it < ntiles; ++it) {
         const uint32_t gt = g + it;
-        const int st = gt % kNS;
-        if (gathered_item) prefetch_tile(it + kPrefetchTiles);
-        // one thread waits and the loaders agree on its result, so no loader can
-        // leave the loop while another waits at a named barrier below
-        if (lt == 0)
-          sLdOk[it & 1] = !*sAbort && (gt < (uint32_t)kNS || mbar_wait(&kempty[st], ((gt / kNS) - 1) & 1u, p.status));
+        const int st = gt & 1;
+        const uint32_t code = ncode;
+        const float scale = nsc;
+        // the first loader warp takes the stage wait (all lanes; lane 0 records the result)
+        if (lw == 0) {
+          bool okw = __shfl_sync(kFull, *sAbort, 0) == 0;
+          if (okw && gt >= 2u) okw = __all_sync(kFull, mbar_wait(&kempty[st], ((gt >> 1) - 1) & 1u, p.status));
+          if (ll == 0) *sLdOk = okw;
+        }
         named_sync(3, kLoaders);
-        if (!sLdOk[it & 1]) {
+        if (!*sLdOk) {
           *sAbort = 1;
-          stopped = true;
           break;
         }
+        if (lt < kNk) {
+          sCode[st * kNk + lt] = code;
+          sScale[st * kNk + lt] = code ? scale : 0.f;  // finite for every key of the tile
+        }
+        if (lw < 2) {
+          const unsigned bits = __ballot_sync(kFull, code != 0u);
+          if (ll == 0) sMask[st * 2 + lw] = bits;
+        }
+        named_sync(3, kLoaders);
         uint8_t* dst = sK + st * kStageBytes;
         int row0 = 0;
         const int mode = tile_src(it, row0);
@@ -454,258 +385,254 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lt == 0) {
             mbar_arrive_expect_tx(&kfull[st], kStageBytes);
             const CUtensorMap* map = mode == 0 ? &tm_ring : &tm_kv;
-            for (int j = 0; j < kNb; ++j)
-              tma_load_2d(dst + j * (kNk * 128), map, (kb_load0 + j) * 64, row0, &kfull[st]);
+            for (int j = 0; j < kNb; ++j) tma_load_2d(dst + j * kBlkBytes, map, j * 64, row0, &kfull[st]);
           }
-          if (pend_it >= 0) finish(pend_it, false);
-          pend_it = -1;
+          if (it + 1 < ntiles) {
+            ncode = code_of(it + 1, nsc);
+            int rr0;
+            if (tile_src(it + 1, rr0) < 0) prefetch(ncode);
+          }
         } else {
-          // consecutive threads take consecutive 16-byte chunks of a row (coalesced); bf16 rows go
-          // by cp.async, FP8 entries into registers (widened into the tile when it is finished)
-          uint2 codes[kPer];
+          // consecutive threads take consecutive 16-byte chunks of a row (coalesced): chunk c of key
+          // kr is 16-byte piece c & 7 of channel block c >> 3; FP8 entries are read as 8 codes and
+          // widened, in passes of kPer / 2 chunks to bound the registers they hold
 #pragma unroll
-          for (int q = 0; q < kPer; ++q) {
-            const int id = lt + q * kLoaders;
-            codes[q] = make_uint2(0u, 0u);
-            if (id < kItems) {
-              const int kr = id / (kNb * 8), c = id % (kNb * 8);
-              const int i = it * kNk + kr;
-              const void* src = i < nk ? sRow[i] : nullptr;
-              if (src && fp8 && u0 + i >= kk.n_w)
-                codes[q] = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(src) + kb_load0 * 64 +
-                                                                c * 8));
-              else
-                cp_async16(dst + swz(kr, c, kNk * 128),
-                           src ? static_cast<const void*>(static_cast<const uint16_t*>(src) + kb_load0 * 64 + c * 8)
-                               : p.q,
-                           src ? 16 : 0);
+          for (int half = 0; half < 2; ++half) {
+            uint2 codes8[kPer / 2];
+#pragma unroll
+            for (int q = 0; q < kPer / 2; ++q) {
+              const int id = lt + (half * (kPer / 2) + q) * kLoaders;
+              codes8[q] = make_uint2(0u, 0u);
+              if (id < kChunks) {
+                const int kr = id / (kNb * 8), c = id % (kNb * 8);
+                const uint32_t cd = sCode[st * kNk + kr];
+                if (fp8 && (cd >> kRowBits) == 1u) {
+                  codes8[q] = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(p.kv_pool) +
+                                                                   (size_t)(cd & kRowMask) * kDqk + c * 8));
+                } else {
+                  const uint16_t* src = code_row(p, cd);
+                  cp_async16(dst + (c >> 3) * kBlkBytes + kr * 128 + (((c & 7) ^ (kr & 7)) << 4),
+                             src ? static_cast<const void*>(src + c * 8) : static_cast<const void*>(p.q),
+                             src ? 16 : 0);
+                }
+              }
+            }
+            if (fp8) {
+#pragma unroll
+              for (int q = 0; q < kPer / 2; ++q) {
+                const int id = lt + (half * (kPer / 2) + q) * kLoaders;
+                if (id < kChunks) {
+                  const int kr = id / (kNb * 8), c = id % (kNb * 8);
+                  if ((sCode[st * kNk + kr] >> kRowBits) == 1u)
+                    *reinterpret_cast<uint4*>(dst + (c >> 3) * kBlkBytes + kr * 128 + (((c & 7) ^ (kr & 7)) << 4)) =
+                        e4m3x8_to_bf16x8(codes8[q]);
+                }
+              }
             }
           }
           cp_async_commit();
-          if (pend_it >= 0) finish(pend_it, true);
-#pragma unroll
-          for (int q = 0; q < kPer; ++q) pend_codes[q] = codes[q];
-          pend_it = it;
-        }
-      }
-      if (pend_it >= 0 && !stopped) finish(pend_it, false);
-    } else if (tid == kMmaThread) {
-      // ------------------------------------------------------------ MMA issue
-      const uint32_t idesc_s = umma_idesc_bf16(kM, kNk, false);
-      const uint32_t idesc_pv = umma_idesc_bf16(kM, 256, true);
-      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK);
-      bool ok = mbar_wait(qbar, n_item & 1u, p.status);
-      for (int it = 0; it <= ntiles + 1 && ok && !*sAbort; ++it) {
-        if (it < ntiles) {
-          const uint32_t gt = g + it;
-          const int st = gt % kNS, buf = gt % kNSP;
-          // the tile is shared memory written by TMA or fenced cp.async / stores: the mbarrier
-          // orders it; tensor memory reuse is ordered by the fence after the P waits below
-          if (!(ok = mbar_wait(&kfull[st], (gt / kNS) & 1u, p.status))) break;
-          const uint32_t d = tmem + kColS + buf * kNk;
-          const uint32_t kb = sKa + st * kStageBytes + s_blk0 * (kNk * 128);
-          // 20 (rank 0) or 16 (rank 1) MMAs into one accumulator
-          if (rank == 0)
-            issue_s<5, 2>(d, sQa, tmem + kColQ, kb, idesc_s);
-          else
-            issue_s<4, 1>(d, sQa, tmem + kColQ, kb, idesc_s);
-          umma_commit(&sfull[buf]);
-        }
-        if (it >= 2) {
-          const uint32_t gp = g + it - 2;
-          const int pb = gp % kNSP, sp = gp % kNS;
-          if (!(ok = mbar_wait(&pfull[pb], (gp / kNSP) & 1u, p.status))) break;
-          tc_fence_after();
-          const uint32_t vb = sKa + sp * kStageBytes;  // blocks 0..3 of the stage: this CTA's V
-#pragma unroll
-          for (int k2 = 0; k2 < 2; ++k2)
-            umma_ts(tmem + kColO, tmem + kColP + pb * 16 + k2 * 8,
-                    umma_desc_sw128(vb + k2 * 16 * 128, kNk * 128, 1024), idesc_pv, (it > 2 || k2 > 0) ? 1u : 0u);
-          umma_commit(&kempty[sp]);
-          umma_commit(&obar[pb]);
-        }
-      }
-      umma_commit(dbar);  // one completion per item, also after an abort
-      if (!ok) *sAbort = 1;
-    } else if (warp < 4) {
-      // ------------------------------------------------------------ softmax (one head row per thread)
-      const float sl2 = p.sm_scale * kLog2e;
-      const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-      const uint32_t recv_peer = peer_addr(sRecv, peer);
-      const uint32_t rfull_peer = peer_addr(rfull, peer);
-      const uint32_t rempty_peer = peer_addr(rempty, peer);
-      const int rr = tid;  // head row
-      float m_used = -INFINITY, l_run = 0.f;
-      // Loop control is per warp (the four warps never meet at a barrier inside the loop); a
-      // failed wait raises the abort flag, and the other warps stop at their next bounded wait.
-      bool ok = true;
-      float part[32];
-      // own partial of tile gt into part[], and one bulk copy of it into the other CTA's slot gt & 1
-      auto produce = [&](uint32_t gt) -> bool {
-        const int buf = gt % kNSP, slot = gt & 1;
-        if (!__all_sync(kFull, mbar_wait(&sfull[buf], (gt / kNSP) & 1u, p.status))) *sAbort = 1;
-        tc_fence_after();
-        uint32_t s0[32];
-        tmem_ld32(tmem + lane_base + kColS + buf * kNk, s0);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) part[j] = __uint_as_float(s0[j]);
-        // slot gt & 1 of the send buffers here and of the receive slots there held tile gt - 2:
-        // both are free once the other CTA has read that tile. Each warp sends its own 32 rows
-        // (4 KB) by its own bulk copy, so the warps need not meet.
-        bool sent = !*sAbort;
-        if (lane == 0 && sent && gt >= 2) sent = mbar_wait(&rempty[slot], ((gt >> 1) - 1) & 1u, p.status);
-        sent = __shfl_sync(kFull, sent, 0);
-        if (sent) {
-          uint8_t* row = sSend + slot * kRecvBytes + rr * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(row + ((c ^ (rr & 7)) << 4)) =
-                make_uint4(__float_as_uint(part[4 * c]), __float_as_uint(part[4 * c + 1]),
-                           __float_as_uint(part[4 * c + 2]), __float_as_uint(part[4 * c + 3]));
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0)
-            bulk_copy_to_peer(recv_peer + slot * kRecvBytes + warp * 4096, sSend + slot * kRecvBytes + warp * 4096,
-                              4096, rfull_peer + slot * 8);
-        }
-        return sent;
-      };
-      {  // this thread's head row of the tensor-memory Q blocks (bf16 pairs, low half first)
-        const uint16_t* qg = p.q + ((int64_t)b * p.n_heads + grp * kM + rr) * kDqk + (qkb0 + n_qs) * 64;
-#pragma unroll 1
-        for (int t = 0; t < kQTmem; ++t) {
-          uint32_t qv[32];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 v = ldg16(qg + t * 64 + c * 8);
-            qv[4 * c] = v.x;
-            qv[4 * c + 1] = v.y;
-            qv[4 * c + 2] = v.z;
-            qv[4 * c + 3] = v.w;
+          if (it + 1 < ntiles) {  // the next tile's rows are looked up while this tile's copies fly
+            ncode = code_of(it + 1, nsc);
+            int rr0;
+            if (tile_src(it + 1, rr0) < 0) prefetch(ncode);
           }
-          tmem_st32(tmem + lane_base + kColQ + t * 32, qv);
+          cp_async_wait<0>();
+          fence_proxy_async_smem();
+          named_sync(3, kLoaders);
+          if (lt == 0) mbar_arrive(&kfull[st]);
         }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(qbar);
       }
-      if (ntiles > 0) ok = produce(g);
+    } else if (warp == 4) {
+      // ------------------------------------------------------------ S issue (lane 0; the warp waits together)
+      const bool issuer = lane == 0;
+      const uint32_t idesc_s = umma_idesc_bf16(kH, kNk, false);
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK);
+      bool ok = __all_sync(kFull, mbar_wait(qbar, n_item & 1u, p.status));
+      tc_fence_after();
       for (int it = 0; it < ntiles && ok; ++it) {
+        if (__shfl_sync(kFull, *sAbort, 0)) break;
         const uint32_t gt = g + it;
-        const int buf = gt % kNSP, slot = gt & 1;
-        float cur[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) cur[j] = part[j];
-        if (it + 1 < ntiles && !(ok = produce(gt + 1))) break;
-        // the other CTA's partial of tile gt: one arrival (here) and 16 KB of its bulk copy
-        if (tid == 0) mbar_arrive_expect_tx(&rfull[slot], kRecvBytes);
-        if (!__all_sync(kFull, mbar_wait(&rfull[slot], (gt >> 1) & 1u, p.status))) *sAbort = 1;
-        const uint8_t* src = sRecv + slot * kRecvBytes + rr * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v = lds16(src + ((c ^ (rr & 7)) << 4));
-          cur[4 * c] += __uint_as_float(v.x);
-          cur[4 * c + 1] += __uint_as_float(v.y);
-          cur[4 * c + 2] += __uint_as_float(v.z);
-          cur[4 * c + 3] += __uint_as_float(v.w);
+        const int k = gt & 1;
+        // the stage is shared memory written by TMA or fenced cp.async / stores: the mbarrier
+        // orders it; S buffer k is free once the softmax has read S(gt - 2)
+        if (!(ok = __all_sync(kFull, mbar_wait(&kfull[k], (gt >> 1) & 1u, p.status)))) break;
+        if (gt >= 2 && !(ok = __all_sync(kFull, mbar_wait(&sfree[k], ((gt >> 1) - 1) & 1u, p.status)))) break;
+        tc_fence_after();
+        if (issuer) {
+          issue_s(tmem + kColS + k * kNk, sQa, sKa + k * kStageBytes, idesc_s);
+          umma_commit(&sfull[k]);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive_peer(rempty_peer + slot * 8);
-        const uint32_t valid = sMask[it];
-        float v[32];
-        float mt = -INFINITY;
-        if (fp8) {  // an FP8 entry's logit and value carry its scale
-#pragma unroll
-          for (int j = 0; j < 32; ++j) cur[j] *= sScale[it * kNk + j];
-        }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          v[j] = ((valid >> j) & 1u) ? cur[j] * sl2 : -INFINITY;  // keys past nk have no row
-          mt = fmaxf(mt, v[j]);
-        }
-        float corr = 1.f;
-        bool rescale = false;
-        if (mt > m_used + kRescaleThreshold || (m_used == -INFINITY && mt != -INFINITY)) {
-          corr = exp2f(m_used - mt);  // 0 when m_used is -inf
-          rescale = it > 0;
-          l_run *= corr;
-          m_used = mt;
-        }
-        const float msub = m_used == -INFINITY ? 0.f : m_used;
-        uint32_t pp[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float p0 = exp2f(v[2 * j] - msub), p1 = exp2f(v[2 * j + 1] - msub);
-          l_run += p0 + p1;
-          pp[j] = fp8 ? pack_bf16(p0 * sScale[it * kNk + 2 * j], p1 * sScale[it * kNk + 2 * j + 1]) : pack_bf16(p0, p1);
-        }
-        // P buffer gt % 3 was read by the P V of tile gt - 3
-        if (gt >= (uint32_t)kNSP && !__all_sync(kFull, mbar_wait(&obar[buf], ((gt / kNSP) - 1) & 1u, p.status)))
-          *sAbort = 1;
-        if (__any_sync(kFull, rescale)) {
-          // O takes the rescale once the P V of tile gt - 1 (and so every earlier one) has landed
-          const uint32_t gq = gt - 1;
-          if (!__all_sync(kFull, mbar_wait(&obar[gq % kNSP], (gq / kNSP) & 1u, p.status))) *sAbort = 1;
+      }
+      if (!ok && issuer) *sAbort = 1;
+      __syncwarp();
+    } else if (warp < 4) {
+      // ------------------------------------------------------------ softmax
+      // thread (warp, lane): head row hr = 16 warp + (lane & 15), keys 32 kh .. + 31 of each tile
+      const float sl2 = p.sm_scale * kLog2e;
+      const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+      const int hr = warp * 16 + (lane & 15), kh = lane >> 4;
+      const uint32_t idesc_pv = umma_idesc_bf16(kH, 256, true);
+      const uint32_t sKa = smem_u32(sK), sPa = smem_u32(sP);
+      uint8_t* prow = sP + hr * 128;
+      float m_used = -INFINITY, l_run = 0.f;
+      bool ok = true;
+      // Every softmax warp reaches the named barrier of every tile; a failed bounded wait only
+      // marks the tile bad, and the barrier's OR over the 128 threads decides for all of them.
+      for (int it = 0; it < ntiles && ok; ++it) {
+        const uint32_t gt = g + it;
+        const int k = gt & 1;
+        bool good = __all_sync(kFull, mbar_wait(&sfull[k], (gt >> 1) & 1u, p.status));
+        float s[32];
+        if (good) {
           tc_fence_after();
-#pragma unroll 1
-          for (int c = 0; c < 256; c += 32) {
-            uint32_t orow[32];
-            tmem_ld32(tmem + lane_base + kColO + c, orow);
-            tmem_ld_wait();
+          // this lane's accumulator row (all 64 keys); keep my 32 keys, swap the other 32 with lane ^ 16
+          uint32_t a[32], o[32];
+          tmem_ld32(tmem + lane_base + kColS + k * kNk, a);
+          tmem_ld32(tmem + lane_base + kColS + k * kNk + 32, o);
+          tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) orow[j] = __float_as_uint(__uint_as_float(orow[j]) * corr);
-            tmem_st32(tmem + lane_base + kColO + c, orow);
+          for (int j = 0; j < 32; ++j) {
+            const float mine = __uint_as_float(kh ? o[j] : a[j]);
+            const float give = __uint_as_float(kh ? a[j] : o[j]);
+            s[j] = mine + __shfl_xor_sync(kFull, give, 16);
           }
         }
-        tmem_st16(tmem + lane_base + kColP + buf * 16, pp);
-        tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&pfull[buf]);
+        mbar_arrive(&sfree[k]);
+        // the stage's key bits and scales (written before the loaders' kfull arrival; that phase
+        // cannot move on before this tile's P V, which waits for this thread's P)
+        if (good) good = __all_sync(kFull, mbar_wait(&kfull[k], (gt >> 1) & 1u, p.status));
+        bool rescale = false;
+        float corr = 1.f;
+        uint32_t pp[16];
+        if (good) {
+          const uint32_t vm = sMask[k * 2 + kh];
+          const float* scl = sScale + k * kNk + 32 * kh;
+          if (fp8) {  // an FP8 entry's logit and value carry its scale
+#pragma unroll
+            for (int j = 0; j < 32; ++j) s[j] *= scl[j];
+          }
+          float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            s[j] = ((vm >> j) & 1u) ? s[j] * sl2 : -INFINITY;  // keys past nk have no row
+            s[j + 1] = ((vm >> (j + 1)) & 1u) ? s[j + 1] * sl2 : -INFINITY;
+            s[j + 2] = ((vm >> (j + 2)) & 1u) ? s[j + 2] * sl2 : -INFINITY;
+            s[j + 3] = ((vm >> (j + 3)) & 1u) ? s[j + 3] * sl2 : -INFINITY;
+            m0 = fmaxf(m0, s[j]);
+            m1 = fmaxf(m1, s[j + 1]);
+            m2 = fmaxf(m2, s[j + 2]);
+            m3 = fmaxf(m3, s[j + 3]);
+          }
+          float mt = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+          mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, 16));  // the row's max over the tile's 64 keys
+          if (mt > m_used + kRescaleThreshold || (m_used == -INFINITY && mt != -INFINITY)) {
+            corr = exp2f(m_used - mt);  // 0 when m_used is -inf
+            rescale = it > 0;
+            l_run *= corr;
+            m_used = mt;
+          }
+          const float msub = m_used == -INFINITY ? 0.f : m_used;
+          float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float e0 = exp2f(s[2 * j] - msub), e1 = exp2f(s[2 * j + 1] - msub);
+            l0 += e0;
+            l1 += e1;
+            pp[j] = fp8 ? pack_bf16(e0 * scl[2 * j], e1 * scl[2 * j + 1]) : pack_bf16(e0, e1);
+          }
+          l_run += l0 + l1;
+          // the P buffer was read by the P V of tile gt - 1, which also finished O
+          if (gt >= 1) good = __all_sync(kFull, mbar_wait(obar, (gt - 1) & 1u, p.status));
+        }
+        if (good) {
+          tc_fence_after();
+          if (__any_sync(kFull, rescale)) {
+            // lanes +0 hold O[:, 0:256], lanes +16 O[:, 256:512] of the same head rows, and both lanes
+            // of a row carry the same corr
+#pragma unroll 1
+            for (int c = 0; c < 256; c += 32) {
+              uint32_t orow[32];
+              tmem_ld32(tmem + lane_base + kColO + c, orow);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) orow[j] = __float_as_uint(__uint_as_float(orow[j]) * corr);
+              tmem_st32(tmem + lane_base + kColO + c, orow);
+            }
+            tmem_st_wait();
+          }
+          // keys 32 kh + 8 i .. + 7: 16-byte chunk 4 kh + i of the row (one 64-key swizzle atom)
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<uint4*>(prow + (((4 * kh + i) ^ (hr & 7)) << 4)) =
+                make_uint4(pp[4 * i], pp[4 * i + 1], pp[4 * i + 2], pp[4 * i + 3]);
+          fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        // every row's P is in shared memory, or some warp met a wait that gave up (uniform answer)
+        if (named_sync_or(1, 128, !good || *sAbort)) {
+          *sAbort = 1;
+          ok = false;
+          break;
+        }
+        if (tid == 0) {
+          tc_fence_after();
+          const uint32_t vb = sKa + k * kStageBytes;  // channel blocks 0..7 of the tile: V
+#pragma unroll
+          for (int ks = 0; ks < kNk / 16; ++ks) {
+            const uint64_t pa = umma_desc_sw128(sPa + ks * 32, 16, 1024);
+            const uint32_t acc = (it > 0 || ks > 0) ? 1u : 0u;
+            umma_ss(tmem + kColO, pa, umma_desc_sw128(vb + ks * 16 * 128, kBlkBytes, 1024), idesc_pv, acc);
+            umma_ss(tmem + kColO + kLane16, pa, umma_desc_sw128(vb + 4 * kBlkBytes + ks * 16 * 128, kBlkBytes, 1024),
+                    idesc_pv, acc);
+          }
+          umma_commit(&kempty[k]);
+          umma_commit(obar);
+        }
       }
-      // epilogue: normalised partial output of this split and half, and its log-sum-exp
+      if (tid == 0) umma_commit(dbar);  // one completion per item, also after an abort
+      // epilogue: normalised partial output of this split and head group, and its log-sum-exp
       ok = __all_sync(kFull, mbar_wait(dbar, n_item & 1u, p.status)) && ok;
       if (!ok) *sAbort = 1;
       tc_fence_after();
-      const int head0 = grp * kM;
-      const int64_t prow0 = ((int64_t)b * p.max_splits + split) * p.n_heads + head0;
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      // each thread writes its head row straight from tensor memory: part_o is
-      // head-minor ([query x split][d_v / 4][heads][4]), so a warp's 16-byte
-      // stores cover 32 consecutive heads, 512 contiguous bytes
+      const float l_row = l_run + __shfl_xor_sync(kFull, l_run, 16);
+      const int head = grp * kH + hr;
+      const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
+      // part_o is head-minor ([query x split][d_v / 4][heads][4]): the 16 lanes of a half-warp
+      // write 16 consecutive heads, 256 contiguous bytes
       float4* po = reinterpret_cast<float4*>(p.part_o) +
-                   (((int64_t)b * p.max_splits + split) * (kDv / 4) + rank * 64) * p.n_heads + head0 + rr;
+                   (((int64_t)b * p.max_splits + split) * (kDv / 4) + kh * 64) * p.n_heads + head;
 #pragma unroll 1
       for (int c = 0; c < 256; c += 32) {
         uint32_t orow[32];
-        if (ok) {
+        if (ok) {  // warp-uniform
           tmem_ld32(tmem + lane_base + kColO + c, orow);
           tmem_ld_wait();
         }
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float4 v = ok ? make_float4(__uint_as_float(orow[4 * k]) * inv, __uint_as_float(orow[4 * k + 1]) * inv,
-                                            __uint_as_float(orow[4 * k + 2]) * inv, __uint_as_float(orow[4 * k + 3]) * inv)
+        for (int q = 0; q < 8; ++q) {
+          const float4 v = ok ? make_float4(__uint_as_float(orow[4 * q]) * inv, __uint_as_float(orow[4 * q + 1]) * inv,
+                                            __uint_as_float(orow[4 * q + 2]) * inv, __uint_as_float(orow[4 * q + 3]) * inv)
                               : make_float4(0.f, 0.f, 0.f, 0.f);
-          po[(int64_t)(c / 4 + k) * p.n_heads] = v;
+          po[(int64_t)(c / 4 + q) * p.n_heads] = v;
         }
       }
-      if (rank == 0) p.part_lse[prow0 + tid] = l_run > 0.f ? (m_used + log2f(l_run)) * kLn2 : -INFINITY;
+      if (kh == 0)
+        p.part_lse[((int64_t)b * p.max_splits + split) * p.n_heads + head] =
+            l_row > 0.f ? (m_used + log2f(l_row)) * kLn2 : -INFINITY;
     }
     g += ntiles;
     tc_fence_before();
     __syncthreads();  // shared and tensor memory are reused by the next item
     tc_fence_after();
-    if (*sAbort) {
-      if (tid == 0) st_peer_u32(peer_addr(const_cast<int*>(sAbort), peer), 1u);  // stop the other CTA too
-      break;
-    }
+    if (*sAbort) break;
   }
   // after an abort, give tensor-core work in flight a bounded chance to land before freeing
-  if (*sAbort && tid == kMmaThread) mbar_wait(dbar, n_item & 1u, nullptr);
+  if (*sAbort && warp == 0) mbar_wait(dbar, n_item & 1u, nullptr);
   cp_async_wait<0>();
   tc_fence_before();
-  cluster.sync();  // the other CTA may still write into this one's shared memory until here
+  __syncthreads();
   tc_fence_after();
   if (warp == 4) tmem_dealloc(tmem, kTmemCols);
 }
@@ -725,20 +652,19 @@ bool encode_rows(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box
 }  // namespace
 
 bool attend_tc_supported(int d_qk, int d_v, int n_heads, int kv_dtype, int n_q) {
-  return d_qk == kDqk && d_v == kDv && n_heads % kM == 0 && (kv_dtype == CSKV_BF16 || kv_dtype == CSKV_FP8_E4M3) &&
-         Smem::bytes(n_q) <= 232448;  // the per-query prefix table shares shared memory with the tiles
+  return d_qk == kDqk && d_v == kDv && n_heads % kH == 0 && (kv_dtype == CSKV_BF16 || kv_dtype == CSKV_FP8_E4M3) &&
+         Smem::bytes(n_q) + 128 <= 232448;  // the per-query prefix table shares shared memory with the tiles
 }
 
-// keys per split: queries x head groups x splits ~ one CTA pair per two SMs
+// keys per split: queries x head groups x splits ~ one CTA per SM
 void attend_tc_plan(AttendParams& p, int n_sm) {
-  const int64_t groups = p.n_heads / kM;
+  const int64_t groups = p.n_heads / kH;
   const int64_t n_max = (int64_t)p.n_win + (p.is_csa ? p.k : visible_entries(p.max_pos, p.m, p.n_win));
-  int64_t splits = (n_sm / 2) / ((int64_t)p.n_q * groups);
+  int64_t splits = n_sm / ((int64_t)p.n_q * groups);
   if (splits < 1) splits = 1;
   int64_t kps = (n_max + splits - 1) / splits;
   kps = (kps + kNk - 1) / kNk * kNk;
   if (kps < kNk) kps = kNk;
-  if (kps > kRowCap) kps = kRowCap;
   p.keys_per_split = static_cast<int>(kps);
   p.max_splits = static_cast<int>((n_max + kps - 1) / kps);
   if (p.max_splits < 1) p.max_splits = 1;
@@ -748,8 +674,9 @@ cudaError_t launch_attend_tc(AttendParams& p, int n_sm, cudaStream_t st) {
   CUtensorMap tm_q, tm_ring, tm_kv;
   const uint64_t kv_rows = static_cast<uint64_t>(p.n_pages) * p.page_size;
   const uint64_t ring_rows = static_cast<uint64_t>(p.n_seqs_layer) * p.n_win;
-  if (kv_rows >= (1ull << 31) || ring_rows >= (1ull << 31)) return cudaErrorNotSupported;
-  if (!encode_rows(&tm_q, p.q, static_cast<uint64_t>(p.n_q) * p.n_heads, kM) ||
+  if (kv_rows > kRowMask || ring_rows > kRowMask || static_cast<uint64_t>(p.chunk_len) > kRowMask)
+    return cudaErrorNotSupported;
+  if (!encode_rows(&tm_q, p.q, static_cast<uint64_t>(p.n_q) * p.n_heads, kH) ||
       !encode_rows(&tm_ring, p.ring_x, ring_rows, kNk) ||
       // an FP8 pool is never read by TMA (its tiles are widened by the loaders)
       !encode_rows(&tm_kv, p.kv_dtype == CSKV_FP8_E4M3 ? static_cast<const void*>(p.ring_x) : p.kv_pool,
@@ -761,25 +688,11 @@ cudaError_t launch_attend_tc(AttendParams& p, int n_sm, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int64_t upper = (int64_t)p.n_q * p.max_splits * (p.n_heads / kM);
-  int64_t clusters = upper < n_sm / 2 ? upper : n_sm / 2;
-  if (clusters < 1) clusters = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  const int64_t items = (int64_t)p.n_q * p.max_splits * (p.n_heads / kH);
+  const int grid = static_cast<int>(items < n_sm ? items : n_sm);
   p.part_t = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, tm_q, tm_ring, tm_kv, p);
+  e = launch_pdl(kern, dim3(static_cast<unsigned>(grid < 1 ? 1 : grid)), dim3(kThreads), smem, st, tm_q, tm_ring,
+                 tm_kv, p);
   if (e != cudaSuccess) return e;
   return launch_attend_merge(p, st);
 }
