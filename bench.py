@@ -17,7 +17,11 @@ replays of a captured CUDA graph of the step (max over ranks); `e2e` is the
 same through the Python entry points with per-step host->device copies of the
 step's inputs and device->host copies of its outputs; `roofline` covers the
 indexer op (its algorithmic bytes = the visible indexer keys) timed with
-events captured around it inside the graph.
+events captured around it inside the graph. The default run then adds, under
+`secondary`, the metric's other figures from the same GPU: the prefill pass
+(65,536 new tokens on 65,536 cached; tokens/s against the sustained bf16
+tensor peak) and the mixed-length paged FP8 / FP4 decode (queries/s against
+HBM), each with its own roofline, e2e and clock record.
 """
 from __future__ import annotations
 
@@ -719,6 +723,25 @@ def run_reference(args, rank, world):
     }
 
 
+def secondary_workloads(args, rank, world):
+    """The metric's other two figures, measured in the same run on the same GPU after the headline decode:
+    the prefill pass (tokens/s against the sustained bf16 tensor peak) and the mixed-length paged FP8 / FP4
+    decode (queries/s against HBM). Each keeps its own roofline, e2e and clock record; the oracle is not
+    run for them here (`--config prefill` / `--config mixed` give their full lines with a cpu_baseline)."""
+    import copy
+    out = {}
+    for name, steps in (("prefill", 6), ("mixed", 64)):
+        a = copy.copy(args)
+        a.config, a.steps, a.warmup, a.no_cpu_baseline, a.batch = name, steps, 3, True, 0
+        torch.cuda.empty_cache()
+        r = run_prefill(a, rank, world) if name == "prefill" else run_ours(a, rank, world)
+        keep = ("value", "unit", "ms_per_step", "steps", "warmup", "dtype", "config", "clocks", "roofline", "e2e",
+                "gpu_launches", "op_ms_untimed_breakdown", "path_roofline", "attention_tflops_untimed")
+        out[name] = {k: r[k] for k in keep if k in r}
+        torch.cuda.synchronize()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -729,6 +752,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling captures)")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the prefill and mixed-workload figures that the default (pro) run adds")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -744,6 +769,8 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
         out = run_prefill(args, rank, world) if args.config == "prefill" else run_ours(args, rank, world)
+        if args.config == "pro" and not args.no_secondary:
+            out["secondary"] = secondary_workloads(args, rank, world)
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:

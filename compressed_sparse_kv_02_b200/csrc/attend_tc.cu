@@ -66,6 +66,7 @@ constexpr uint32_t kLane16 = 16u << 16;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;       // log2 units
+constexpr int kMaxSplitKeys = 1024;             // keys of one HCA work item at most (16 tiles)
 
 struct Smem {
   static constexpr int Q = 0;                          // 9 blocks of 64 heads x 128 B
@@ -665,6 +666,10 @@ void attend_tc_plan(AttendParams& p, int n_sm) {
   int64_t kps = (n_max + splits - 1) / splits;
   kps = (kps + kNk - 1) / kNk * kNk;
   if (kps < kNk) kps = kNk;
+  // HCA key counts grow with the context (n / 128 + 128): with many queries of mixed lengths one split
+  // per query would leave the longest ones on one CTA, so no HCA item takes more than kMaxSplitKeys
+  // keys (a CSA query has at most n_win + k keys, all of similar count)
+  if (!p.is_csa && kps > kMaxSplitKeys) kps = kMaxSplitKeys;
   p.keys_per_split = static_cast<int>(kps);
   p.max_splits = static_cast<int>((n_max + kps - 1) / kps);
   if (p.max_splits < 1) p.max_splits = 1;

@@ -326,23 +326,8 @@ constexpr int kAppendWarps = 16;  // an FP8 entry is folded whole by one CTA: 36
 constexpr int kAppendThreads = 32 * kAppendWarps;
 constexpr int kSliceCh = 64;       // channels per CTA of the append kernel (whole row for FP8)
 constexpr int kAppendMaxD = 1024;  // channels of the row buffer
-
-// Online-softmax state (max of the base-2 logits, denominator, weighted sum)
-// of 16 channels, merged from another lane's state.
-__device__ __forceinline__ void merge16(float (&mx)[16], float (&den)[16], float (&acc)[16], int o) {
-#pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    const float m2 = __shfl_xor_sync(kFull, mx[e], o);
-    const float d2 = __shfl_xor_sync(kFull, den[e], o);
-    const float a2 = __shfl_xor_sync(kFull, acc[e], o);
-    const float M = fmaxf(mx[e], m2);
-    const float f1 = mx[e] == -INFINITY ? 0.f : exp2f(mx[e] - M);
-    const float f2 = m2 == -INFINITY ? 0.f : exp2f(m2 - M);
-    den[e] = den[e] * f1 + d2 * f2;
-    acc[e] = acc[e] * f1 + a2 * f2;
-    mx[e] = M;
-  }
-}
+constexpr int kFoldPairs = 32;     // channel pairs of one fold pass (64 channels)
+constexpr int kFoldGroups = kAppendThreads / kFoldPairs;  // 16 token groups
 
 // Store channels [c_lo, c_hi) of one folded entry from the row buffer `sv`
 // (fp32, indexed by channel) into pool row `row` in the stream's storage type:
@@ -408,16 +393,17 @@ __device__ void store_row(const FoldStream& S, int64_t row, const float* sv, int
 // new rows into the rings, then folds its channels of every block the new
 // tokens complete (old rows from the ring, new rows from the input; the slots
 // written and the slots read never coincide because n_new + m - 1 <= n_win).
-// A group of lanes folds 16 channels: each lane runs the online softmax over
-// its tokens of the block and the group's partial states merge by shuffles
-// (a group is 32 lanes for m >= 32, else the next power of two >= m, so a warp
-// folds several 16-channel units at once); the entry is stored from a
-// shared-memory row buffer.
+// All 512 threads fold: thread (token group g, channel pair) runs the online
+// softmax of the gate over tokens g, g + 16, ... of the block for its two
+// channels, and one thread per channel merges the 16 groups' states from
+// shared memory; the entry is stored from a shared-memory row buffer.
 __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
   __shared__ float sv[kAppendMaxD];
   __shared__ float s_red[kAppendWarps];
+  __shared__ float s_mx[kFoldGroups][2 * kFoldPairs], s_den[kFoldGroups][2 * kFoldPairs],
+      s_acc[kFoldGroups][2 * kFoldPairs];
   const int b = blockIdx.x, slice = blockIdx.y, si = blockIdx.z;
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int t = threadIdx.x;
   grid_dependency_wait();  // every input may come from the kernel launched before this one
   grid_dependents_launch();
   const int seq = p.seq_ids[b];
@@ -450,25 +436,17 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
   // blocks completed by positions pos .. pos+n_new-1
   const int64_t j_first = pos / p.m;                 // first block ending at or after pos
   const int64_t j_last = (pos + p.n_new) / p.m - 1;  // last block ending before pos+n_new
-  int merge_span = 1;  // power of two >= min(m, 32)
-  while (merge_span < 32 && merge_span < p.m) merge_span <<= 1;
+  // every thread folds a channel pair over a group of the block's tokens (tokens tg, tg + 16, ...);
+  // the 16 groups' partial states (running max in base 2, denominator, weighted sum) then merge
+  // per channel through shared memory
+  const int cp = t % kFoldPairs, tg = t / kFoldPairs;
   for (int64_t j = j_first; j <= j_last; ++j) {
     const int64_t row = entry_row(p, seq, j);  // uniform across the block
-    // lanes in groups of merge_span (a power of two >= min(m, 32)): group g of the warp folds
-    // 16-channel unit (base + g) with one lane per token
-    const int per_warp = 32 / merge_span;
-    const int grp = lane / merge_span, tok = lane % merge_span;
-    for (int u0 = c_lo / 16 + warp * per_warp; u0 < c_hi / 16; u0 += kAppendWarps * per_warp) {
-      const int c0 = (u0 + grp) * 16;
-      const bool active = c0 < c_hi;
-      float mx[16], den[16], acc[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        mx[e] = -INFINITY;
-        den[e] = 0.f;
-        acc[e] = 0.f;
-      }
-      for (int i = tok; active && i < p.m; i += merge_span) {
+    for (int c0 = c_lo; c0 < c_hi; c0 += 2 * kFoldPairs) {  // 64 channels per pass
+      const int c = c0 + 2 * cp;
+      const bool active = c < c_hi;
+      float mx[2] = {-INFINITY, -INFINITY}, den[2] = {0.f, 0.f}, acc[2] = {0.f, 0.f};
+      for (int i = tg; active && i < p.m; i += kFoldGroups) {
         const int64_t q = j * p.m + i;
         const uint16_t* xr;
         const uint16_t* zr;
@@ -480,36 +458,20 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
           xr = S.ring_x + ((int64_t)seq * p.n_win + slot) * S.d;
           zr = S.ring_z + ((int64_t)seq * p.n_win + slot) * S.gc;
         }
-        float xf[16], zl[16];
-        {
-          float h[8];
-          unpack8(ldg16(xr + c0), h);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) xf[e] = h[e];
-          unpack8(ldg16(xr + c0 + 8), h);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) xf[8 + e] = h[e];
-        }
+        const uint32_t xv = __ldg(reinterpret_cast<const uint32_t*>(xr + c));
+        float zl[2];
         if (S.gc == 1) {
-          const float zz = bf16_bits_to_f32(zr[0]);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) zl[e] = zz;
+          zl[0] = zl[1] = bf16_bits_to_f32(__ldg(zr));
         } else {
-          float h[8];
-          unpack8(ldg16(zr + c0), h);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) zl[e] = h[e];
-          unpack8(ldg16(zr + c0 + 8), h);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) zl[8 + e] = h[e];
+          const uint32_t zv = __ldg(reinterpret_cast<const uint32_t*>(zr + c));
+          zl[0] = __uint_as_float(zv << 16);
+          zl[1] = __uint_as_float(zv & 0xffff0000u);
         }
-        if (S.bias) {
+        const float xf[2] = {__uint_as_float(xv << 16), __uint_as_float(xv & 0xffff0000u)};
 #pragma unroll
-          for (int e = 0; e < 16; ++e) zl[e] += S.bias[(int64_t)i * S.d + c0 + e];
-        }
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float l2 = zl[e] * kLog2e;  // base-2 weights: 2^(l2 - max) = e^(z - max_z)
+        for (int e = 0; e < 2; ++e) {
+          const float bias = S.bias ? S.bias[(int64_t)i * S.d + c + e] : 0.f;
+          const float l2 = (zl[e] + bias) * kLog2e;  // base-2 weights: 2^(l2 - max) = e^(z - max_z)
           const float M = fmaxf(mx[e], l2);
           const float corr = mx[e] == -INFINITY ? 0.f : exp2f(mx[e] - M);
           const float pw = exp2f(l2 - M);
@@ -518,13 +480,29 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
           mx[e] = M;
         }
       }
-      // lanes >= m hold nothing: merge only across the lanes that ran tokens
-      for (int o = merge_span >> 1; o > 0; o >>= 1) merge16(mx, den, acc, o);
-      if (active && tok == 0)
+      if (active) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) sv[c0 + e] = acc[e] / den[e];
+        for (int e = 0; e < 2; ++e) {
+          s_mx[tg][2 * cp + e] = mx[e];
+          s_den[tg][2 * cp + e] = den[e];
+          s_acc[tg][2 * cp + e] = acc[e];
+        }
+      }
+      __syncthreads();
+      if (t < 2 * kFoldPairs && c0 + t < c_hi) {  // one thread per channel merges the groups that ran tokens
+        const int ng = p.m < kFoldGroups ? p.m : kFoldGroups;
+        float M = -INFINITY;
+        for (int gi = 0; gi < ng; ++gi) M = fmaxf(M, s_mx[gi][t]);
+        float dd = 0.f, aa = 0.f;
+        for (int gi = 0; gi < ng; ++gi) {
+          const float f = s_mx[gi][t] == -INFINITY ? 0.f : exp2f(s_mx[gi][t] - M);
+          dd += s_den[gi][t] * f;
+          aa += s_acc[gi][t] * f;
+        }
+        sv[c0 + t] = aa / dd;
+      }
+      __syncthreads();
     }
-    __syncthreads();
     if (row >= 0) store_row(S, row, sv, c_lo, c_hi, s_red);
     __syncthreads();  // the row buffer is reused by the next block
   }
