@@ -81,6 +81,9 @@ def _L():
             "orc_mat_decode": (ctypes.c_int, [MP, P]),
             "orc_store_rows": (ctypes.c_int, [P, I64, I64, ctypes.c_int32, P, P]),
             "orc_compress": (ctypes.c_int, [MP, MP, P, I64, P]),
+            "orc_compress_overlap": (ctypes.c_int, [MP, MP, P, I64, I64, P]),
+            "orc_round_scores_bf16": (ctypes.c_int, [P, I64, P]),
+            "orc_inverse_rope": (ctypes.c_int, [P, I64, I64, I64, I64, I64, D]),
             "orc_visible_entries": (I64, [I64, I64, I64]),
             "orc_window_start": (I64, [I64, I64]),
             "orc_index_scores": (ctypes.c_int, [MP, P, MP, I64, P]),
@@ -247,6 +250,43 @@ def compress(x: Stored, z: Stored, m: int, bias: Optional[np.ndarray] = None) ->
     rc = _L().orc_compress(ctypes.byref(xm), ctypes.byref(zm), _ptr(b), m, out.ctypes.data)
     if rc:
         raise ValueError("orc_compress failed (%d)" % rc)
+    return out
+
+
+def compress_overlap(x: Stored, z: Stored, m: int, ov: int, bias: Optional[np.ndarray] = None) -> np.ndarray:
+    """Fold of every block of m rows plus the ov rows before it (x, z: the stream from position 0;
+    bias: [m + ov, d] or None) -> fp64 [n/m, d]. ov = 0 is `compress`."""
+    if x.rows % m:
+        raise ValueError("token count %d is not a multiple of m=%d" % (x.rows, m))
+    out = np.empty((x.rows // m, x.cols), np.float64)
+    b = None if bias is None else np.ascontiguousarray(bias, np.float64).reshape(m + ov, x.cols)
+    xm, zm = x.mat(), z.mat()
+    rc = _L().orc_compress_overlap(ctypes.byref(xm), ctypes.byref(zm), _ptr(b), m, ov, out.ctypes.data)
+    if rc:
+        raise ValueError("orc_compress_overlap failed (%d)" % rc)
+    return out
+
+
+def round_scores_bf16(scores: np.ndarray) -> np.ndarray:
+    """Index scores as the BF16-score selection sees them: fp64 -> fp32 -> bf16 (RNE), back to fp64."""
+    s = np.ascontiguousarray(scores, np.float64).ravel()
+    out = np.empty_like(s)
+    _L().orc_round_scores_bf16(s.ctypes.data, s.size, out.ctypes.data)
+    return out
+
+
+def topk_bf16(scores: np.ndarray, k: int):
+    """Top-k of the bf16-rounded scores (order: rounded score desc, index asc) -> (idx, k_eff)."""
+    return topk(round_scores_bf16(scores), k)
+
+
+def inverse_rope(o: np.ndarray, r0: int, d_rope: int, t: int, base: float = 10000.0) -> np.ndarray:
+    """Channels [r0, r0 + d_rope) of every row of o rotated by -t theta_i (pairs 2i, 2i+1) -> new array."""
+    out = np.array(o, np.float64, copy=True, order="C")
+    rows, cols = out.shape
+    rc = _L().orc_inverse_rope(out.ctypes.data, rows, cols, r0, d_rope, t, float(base))
+    if rc:
+        raise ValueError("orc_inverse_rope failed (%d)" % rc)
     return out
 
 

@@ -319,6 +319,92 @@ int orc_compress(const orc_mat* x, const orc_mat* z, const double* bias, int64_t
 }
 
 /* ------------------------------------------------------------------ */
+/* a1 / a2 with block overlap ([10100] 2.1: block compression "combined */
+/* with position weighting and block overlap", width unstated).         */
+/* Reading: entry j also folds the last `ov` tokens of the block before */
+/* it, i.e. the tokens at positions max(0, j*m - ov) .. j*m + m - 1 of  */
+/* the stream, under one softmax; the position bias then has m + ov     */
+/* rows, row r for the token at position j*m - ov + r. x and z hold the */
+/* stream from position 0; ov = 0 is the plain fold above. The entry is */
+/* complete when its own block is, so visibility does not change.       */
+/*   l_p   = Z[p, c] + B[p - (j*m - ov), c]                             */
+/*   a_p   = exp(l_p - max l) / sum_p exp(l_p - max l)                  */
+/*   C[j,c] = sum_p a_p X[p, c]     (p over the positions above)        */
+/* ------------------------------------------------------------------ */
+int orc_compress_overlap(const orc_mat* x, const orc_mat* z, const double* bias, int64_t m, int64_t ov,
+                         double* out) {
+  int64_t n = x->rows, d = x->cols;
+  if (m <= 0 || ov < 0 || n % m != 0) return ORC_EINVAL;
+  if (z->rows != n || (z->cols != 1 && z->cols != d)) return ORC_EINVAL;
+  int64_t nb = n / m;
+#pragma omp parallel for schedule(static)
+  for (int64_t j = 0; j < nb; ++j) {
+    int64_t first = j * m - ov < 0 ? 0 : j * m - ov;
+    int64_t last = j * m + m - 1;
+    double* l = (double*)malloc(sizeof(double) * (size_t)(m + ov));
+    for (int64_t c = 0; c < d; ++c) {
+      double mx = -INFINITY;
+      for (int64_t p = first; p <= last; ++p) {
+        double v = orc_mat_at(z, p, z->cols == 1 ? 0 : c) + (bias ? bias[(p - (j * m - ov)) * d + c] : 0.0);
+        l[p - first] = v;
+        if (v > mx) mx = v;
+      }
+      double den = 0.0;
+      for (int64_t p = first; p <= last; ++p) den += exp(l[p - first] - mx);
+      double acc = 0.0;
+      for (int64_t p = first; p <= last; ++p) acc += (exp(l[p - first] - mx) / den) * orc_mat_at(x, p, c);
+      out[j * d + c] = acc;
+    }
+    free(l);
+  }
+  return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* BF16 index scores ([digest] section 7: the indexer's scores are kept */
+/* in BF16 instead of FP32, which halves the selector's cost at 99.7%   */
+/* recall of the FP32 selection). Reading: each score, computed in      */
+/* fp32, is rounded to bf16 (round to nearest even) and the top-k of    */
+/* the rounded scores is taken with the usual order (score desc, index  */
+/* asc), so entries whose scores round together are taken in index      */
+/* order. This function does the rounding: fp64 -> fp32 -> bf16.       */
+/* ------------------------------------------------------------------ */
+int orc_round_scores_bf16(const double* scores, int64_t n, double* out) {
+  for (int64_t j = 0; j < n; ++j) out[j] = orc_bf16_to_f64(orc_f32_to_bf16_bits(to_f32(scores[j])));
+  return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Inverse RoPE on the attention output ([essay] "约束1 -> 创新1": with */
+/* 128 tokens sharing one compressed entry, position is restored by an */
+/* inverse-RoPE correction applied to the attention output). Reading:  */
+/* the channels [r0, r0 + d_rope) of each output row form d_rope / 2   */
+/* pairs (r0 + 2i, r0 + 2i + 1) carrying RoPE at frequency             */
+/*   theta_i = base^(-2i / d_rope);                                    */
+/* a value rotated by its key's position p, summed with attention      */
+/* weights, becomes relative to the query at position t after a        */
+/* rotation by -t theta_i:                                             */
+/*   (a, b) <- (a cos(t theta_i) + b sin(t theta_i),                   */
+/*              -a sin(t theta_i) + b cos(t theta_i)).                 */
+/* o is [rows, cols], rotated in place.                                */
+/* ------------------------------------------------------------------ */
+int orc_inverse_rope(double* o, int64_t rows, int64_t cols, int64_t r0, int64_t d_rope, int64_t t, double base) {
+  if (d_rope <= 0 || d_rope % 2 || r0 < 0 || r0 + d_rope > cols || base <= 0.0) return ORC_EINVAL;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t i = 0; i < d_rope / 2; ++i) {
+      double theta = pow(base, -2.0 * (double)i / (double)d_rope);
+      double ang = (double)t * theta;
+      double cs = cos(ang), sn = sin(ang);
+      double* a = o + r * cols + r0 + 2 * i;
+      double x = a[0], y = a[1];
+      a[0] = x * cs + y * sn;
+      a[1] = -x * sn + y * cs;
+    }
+  }
+  return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
 /* visibility (reading: an entry is visible iff its block starts before */
 /* the window of the last n_win raw tokens; [digest] section 3: both    */
 /* branches add the last n_win = 128 uncompressed tokens)               */
