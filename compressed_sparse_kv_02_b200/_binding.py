@@ -76,7 +76,7 @@ class IndexArgs(ctypes.Structure):
         ("struct_size", ctypes.c_uint32), ("layer", ctypes.POINTER(LayerStruct)), ("n_q", _I32),
         ("n_heads_idx", _I32), ("q_seq", _P), ("q_pos", _P), ("max_pos", _I64), ("q_idx", _P),
         ("q_idx_scale", _P), ("w", _P), ("k", _I32), ("out_idx", _P), ("out_cnt", _P),
-        ("out_scores", _P), ("d_status", _P),
+        ("out_scores", _P), ("d_status", _P), ("score_bf16", _I32),
     ]
 
 
@@ -86,6 +86,7 @@ class AttendArgs(ctypes.Structure):
         ("n_heads", _I32), ("q_seq", _P), ("q_pos", _P), ("max_pos", _I64), ("q", _P),
         ("sel_idx", _P), ("sel_cnt", _P), ("k", _I32), ("sm_scale", ctypes.c_float), ("out", _P),
         ("lse", _P), ("x_chunk", _P), ("chunk_pos0", _I64), ("chunk_len", _I64), ("d_status", _P),
+        ("rope_dims", _I32), ("rope_base", ctypes.c_float),
     ]
 
 
@@ -349,11 +350,12 @@ def cskv_cache_append(layer: Layer, seq_ids, pos, x, z, xi=None, zi=None, ring_o
     _check(lib().cskv_cache_append(ctypes.byref(a), _stream(stream)), "cskv_cache_append")
 
 
-def _index_args(layer, q_seq, q_pos, max_pos, q_idx, w, k, out_idx, out_cnt, out_scores, q_idx_scale, status):
+def _index_args(layer, q_seq, q_pos, max_pos, q_idx, w, k, out_idx, out_cnt, out_scores, q_idx_scale, status,
+                score_bf16=False):
     n_q, h_i = w.shape
     return IndexArgs(ctypes.sizeof(IndexArgs), ctypes.pointer(layer.struct), n_q, h_i, _ptr(q_seq), _ptr(q_pos),
                      int(max_pos), _ptr(q_idx), _ptr(q_idx_scale), _ptr(w), int(k), _ptr(out_idx), _ptr(out_cnt),
-                     _ptr(out_scores), _ptr(status))
+                     _ptr(out_scores), _ptr(status), 1 if score_bf16 else 0)
 
 
 def csa_index_ws_bytes(layer: Layer, n_q: int, n_heads_idx: int, max_pos: int, k: int) -> int:
@@ -365,8 +367,10 @@ def csa_index_ws_bytes(layer: Layer, n_q: int, n_heads_idx: int, max_pos: int, k
 
 
 def csa_index_score_topk(layer: Layer, q_seq, q_pos, max_pos: int, q_idx, w, k: int, out_idx, out_cnt,
-                         out_scores=None, q_idx_scale=None, workspace=None, status=None, stream=None):
-    """Indexer scores of every visible CSA entry and the ascending top-k ids per query."""
+                         out_scores=None, q_idx_scale=None, workspace=None, status=None, stream=None,
+                         score_bf16=False):
+    """Indexer scores of every visible CSA entry and the ascending top-k ids per query (score_bf16: select
+    on the scores rounded to bf16)."""
     if not layer.is_csa:
         raise ValueError("csa_index_score_topk needs a CSA layer")
     _need(w, "w", torch.float32)
@@ -385,7 +389,8 @@ def csa_index_score_topk(layer: Layer, q_seq, q_pos, max_pos: int, q_idx, w, k: 
     if workspace is None:
         workspace = torch.empty(csa_index_ws_bytes(layer, n_q, h_i, max_pos, k), dtype=torch.uint8,
                                 device=w.device)
-    a = _index_args(layer, q_seq, q_pos, max_pos, q_idx, w, k, out_idx, out_cnt, out_scores, q_idx_scale, status)
+    a = _index_args(layer, q_seq, q_pos, max_pos, q_idx, w, k, out_idx, out_cnt, out_scores, q_idx_scale, status,
+                    score_bf16)
     _check(lib().csa_index_score_topk(ctypes.byref(a), _ptr(workspace), workspace.numel(), _stream(stream)),
            "csa_index_score_topk")
 
@@ -412,7 +417,7 @@ def csa_index_score_topk_static(layer: Layer, q_seq, q_pos, max_pos: int, q_idx,
 
 
 def _attend_args(layer, q_seq, q_pos, max_pos, q, sel_idx, sel_cnt, k, sm_scale, out, lse, x_chunk, chunk_pos0,
-                 status, n_q=None, n_heads=None):
+                 status, n_q=None, n_heads=None, rope_dims=0, rope_base=10000.0):
     if q is not None:
         n_q, n_heads = q.shape[0], q.shape[1]
     if sm_scale is None:
@@ -420,7 +425,8 @@ def _attend_args(layer, q_seq, q_pos, max_pos, q, sel_idx, sel_cnt, k, sm_scale,
     return AttendArgs(ctypes.sizeof(AttendArgs), ctypes.pointer(layer.struct), n_q, n_heads, _ptr(q_seq),
                       _ptr(q_pos), int(max_pos), _ptr(q), _ptr(sel_idx), _ptr(sel_cnt), int(k), float(sm_scale),
                       _ptr(out), _ptr(lse), _ptr(x_chunk), int(chunk_pos0),
-                      0 if x_chunk is None else int(x_chunk.shape[0]), _ptr(status))
+                      0 if x_chunk is None else int(x_chunk.shape[0]), _ptr(status), int(rope_dims),
+                      float(rope_base))
 
 
 def cskv_attend_ws_bytes(layer: Layer, n_q: int, n_heads: int, max_pos: int, k: int = 0) -> int:
@@ -431,7 +437,7 @@ def cskv_attend_ws_bytes(layer: Layer, n_q: int, n_heads: int, max_pos: int, k: 
 
 
 def _attend(fn, where, layer, q_seq, q_pos, max_pos, q, sel_idx, sel_cnt, k, out, lse, sm_scale, workspace,
-            x_chunk, chunk_pos0, status, stream):
+            x_chunk, chunk_pos0, status, stream, rope_dims=0, rope_base=10000.0):
     n_q, n_heads = q.shape[0], q.shape[1]
     _need(q_seq, "q_seq", torch.int32, (n_q,))
     _need(q_pos, "q_pos", torch.int64, (n_q,))
@@ -444,29 +450,33 @@ def _attend(fn, where, layer, q_seq, q_pos, max_pos, q, sel_idx, sel_cnt, k, out
         workspace = torch.empty(cskv_attend_ws_bytes(layer, n_q, n_heads, max_pos, k), dtype=torch.uint8,
                                 device=q.device)
     a = _attend_args(layer, q_seq, q_pos, max_pos, q, sel_idx, sel_cnt, k, sm_scale, out, lse, x_chunk, chunk_pos0,
-                     status)
+                     status, rope_dims=rope_dims, rope_base=rope_base)
     _check(fn(ctypes.byref(a), _ptr(workspace), workspace.numel(), _stream(stream)), where)
 
 
 def csa_attend(layer: Layer, q_seq, q_pos, max_pos: int, q, sel_idx, sel_cnt, out, lse=None, sm_scale=None,
-               workspace=None, x_chunk=None, chunk_pos0: int = 0, status=None, stream=None):
-    """One softmax over the window and the selected CSA entries, every head sharing the latent KV."""
+               workspace=None, x_chunk=None, chunk_pos0: int = 0, status=None, stream=None, rope_dims: int = 0,
+               rope_base: float = 10000.0):
+    """One softmax over the window and the selected CSA entries, every head sharing the latent KV
+    (rope_dims > 0: inverse RoPE on the output's last rope_dims channels at each query's position)."""
     if not layer.is_csa:
         raise ValueError("csa_attend needs a CSA layer")
     k = sel_idx.shape[1]
     _need(sel_idx, "sel_idx", torch.int32, (q.shape[0], k))
     _need(sel_cnt, "sel_cnt", torch.int32, (q.shape[0],))
     _attend(lib().csa_attend, "csa_attend", layer, q_seq, q_pos, max_pos, q, sel_idx, sel_cnt, k, out, lse,
-            sm_scale, workspace, x_chunk, chunk_pos0, status, stream)
+            sm_scale, workspace, x_chunk, chunk_pos0, status, stream, rope_dims, rope_base)
 
 
 def hca_attend(layer: Layer, q_seq, q_pos, max_pos: int, q, out, lse=None, sm_scale=None, workspace=None,
-               x_chunk=None, chunk_pos0: int = 0, status=None, stream=None):
-    """One softmax over the window and every visible HCA entry."""
+               x_chunk=None, chunk_pos0: int = 0, status=None, stream=None, rope_dims: int = 0,
+               rope_base: float = 10000.0):
+    """One softmax over the window and every visible HCA entry (rope_dims > 0: inverse RoPE on the
+    output's last rope_dims channels at each query's position)."""
     if layer.is_csa:
         raise ValueError("hca_attend needs an HCA layer")
     _attend(lib().hca_attend, "hca_attend", layer, q_seq, q_pos, max_pos, q, None, None, 0, out, lse, sm_scale,
-            workspace, x_chunk, chunk_pos0, status, stream)
+            workspace, x_chunk, chunk_pos0, status, stream, rope_dims, rope_base)
 
 
 def cskv_get_status(status: torch.Tensor, stream=None) -> int:

@@ -2,6 +2,7 @@
 // argument checks on the host, workspace sizing, and kernel dispatch. No
 // allocation, no synchronisation (except cskv_get_status), no state.
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
 #include <string.h>
 
@@ -130,8 +131,16 @@ cskv_status compress_impl(const cskv_compress_args* a, void* stream, int kind) {
   return from_cuda(cskv::launch_fold_bulk(p, static_cast<cudaStream_t>(stream)));
 }
 
+// struct_size of the index args before score_bf16 was added (such callers get fp32 selection)
+constexpr size_t kIndexArgsV1 = offsetof(cskv_index_args, score_bf16);
+
+int32_t index_score_bf16(const cskv_index_args* a) {
+  return a->struct_size >= offsetof(cskv_index_args, score_bf16) + sizeof(int32_t) ? a->score_bf16 : 0;
+}
+
 cskv_status check_index(const cskv_index_args* a) {
-  if (!a || a->struct_size < sizeof(cskv_index_args)) return CSKV_ERR_INVALID_ARG;
+  if (!a || a->struct_size < kIndexArgsV1) return CSKV_ERR_INVALID_ARG;
+  if (index_score_bf16(a) != 0 && index_score_bf16(a) != 1) return CSKV_ERR_INVALID_ARG;
   const cskv_layer* L = a->layer;
   cskv_status s = check_layer_shape(L);
   if (s) return s;
@@ -145,8 +154,20 @@ cskv_status check_index(const cskv_index_args* a) {
   return CSKV_OK;
 }
 
+// struct_size of the attend args before the inverse-RoPE fields (such callers get none)
+constexpr size_t kAttendArgsV1 = offsetof(cskv_attend_args, rope_dims);
+
+int32_t attend_rope_dims(const cskv_attend_args* a) {
+  return a->struct_size >= offsetof(cskv_attend_args, rope_base) + sizeof(float) ? a->rope_dims : 0;
+}
+
 cskv_status check_attend(const cskv_attend_args* a, int kind) {
-  if (!a || a->struct_size < sizeof(cskv_attend_args)) return CSKV_ERR_INVALID_ARG;
+  if (!a || a->struct_size < kAttendArgsV1) return CSKV_ERR_INVALID_ARG;
+  {
+    const int32_t rd = attend_rope_dims(a);
+    if (rd < 0 || rd % 2 || (a->layer && rd > a->layer->d_v) || (rd > 0 && !(a->rope_base > 0.f)))
+      return CSKV_ERR_INVALID_ARG;
+  }
   const cskv_layer* L = a->layer;
   cskv_status s = check_layer_shape(L);
   if (s) return s;
@@ -192,6 +213,8 @@ void fill_attend(AttendParams& p, const cskv_attend_args* a, int kind) {
   p.chunk_pos0 = a->chunk_pos0;
   p.chunk_len = a->chunk_len;
   p.status = a->d_status;
+  p.rope_dims = attend_rope_dims(a);
+  p.rope_base = p.rope_dims > 0 ? a->rope_base : 0.f;
 }
 
 cskv_status attend_impl(const cskv_attend_args* a, void* ws, size_t ws_bytes, void* stream, int kind) {
@@ -315,6 +338,7 @@ cskv_status csa_index_score_topk(const cskv_index_args* a, void* ws, size_t ws_b
   p.out_cnt = a->out_cnt;
   p.out_scores = a->out_scores;
   p.status = a->d_status;
+  p.score_bf16 = index_score_bf16(a);
   return from_cuda(cskv::launch_index(p, ws, sm_count(), static_cast<cudaStream_t>(stream)));
 }
 

@@ -380,7 +380,9 @@ __global__ void __launch_bounds__(256) attend_merge_kernel(AttendParams p) {
       }
     }
     const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-    uint2 packed = make_uint2(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv));
+    float v[4] = {acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv};
+    inverse_rope4(v, c4, p.d_v, p.rope_dims, p.rope_base, p.q_pos[b]);
+    uint2 packed = make_uint2(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]));
     *reinterpret_cast<uint2*>(p.out + ((int64_t)b * p.n_heads + h) * p.d_v + c4) = packed;
     if (p.lse && c4 == 0) p.lse[(int64_t)b * p.n_heads + h] = wsum > 0.f ? L + logf(wsum) : -INFINITY;
   }
@@ -429,7 +431,9 @@ __global__ void __launch_bounds__(256) attend_merge_t_kernel(AttendParams p) {
     }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  const uint2 packed = make_uint2(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv));
+  float v[4] = {acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv};
+  inverse_rope4(v, g4 * 4, p.d_v, p.rope_dims, p.rope_base, p.q_pos[b]);
+  const uint2 packed = make_uint2(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]));
   *reinterpret_cast<uint2*>(p.out + ((int64_t)b * p.n_heads + h) * p.d_v + g4 * 4) = packed;
   if (p.lse && g4 == 0) p.lse[(int64_t)b * p.n_heads + h] = wsum > 0.f ? L + logf(wsum) : -INFINITY;
 }

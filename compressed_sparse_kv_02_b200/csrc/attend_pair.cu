@@ -514,13 +514,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait();
         }
         if (write) {
+          const int64_t tq = p.q_pos[b_mine];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = has ? __uint_as_float(o[8 * i + e]) * inv : 0.f;
+            if (p.rope_dims > 0 && has) {  // inverse RoPE of the output's last rope_dims channels
+              float a4[4] = {f[0], f[1], f[2], f[3]}, b4[4] = {f[4], f[5], f[6], f[7]};
+              inverse_rope4(a4, c + 8 * i, kD, p.rope_dims, p.rope_base, tq);
+              inverse_rope4(b4, c + 8 * i + 4, kD, p.rope_dims, p.rope_base, tq);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                f[e] = a4[e];
+                f[4 + e] = b4[e];
+              }
+            }
             uint4 v;
-            v.x = has ? pack_bf16(__uint_as_float(o[8 * i]) * inv, __uint_as_float(o[8 * i + 1]) * inv) : 0u;
-            v.y = has ? pack_bf16(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv) : 0u;
-            v.z = has ? pack_bf16(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv) : 0u;
-            v.w = has ? pack_bf16(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv) : 0u;
+            v.x = pack_bf16(f[0], f[1]);
+            v.y = pack_bf16(f[2], f[3]);
+            v.z = pack_bf16(f[4], f[5]);
+            v.w = pack_bf16(f[6], f[7]);
             *reinterpret_cast<uint4*>(orow + c + 8 * i) = v;
           }
         }

@@ -33,6 +33,35 @@ __device__ __host__ __forceinline__ int64_t window_start(int64_t t, int n_win) {
   return s < 0 ? 0 : s;
 }
 
+// Inverse RoPE of output channel pair i (of rope_dims) for the query at position t: (a, b) rotated
+// by -t theta_i, theta_i = base^(-2i / rope_dims). The angle reaches ~1e6 radians at 1M positions,
+// beyond what fp32 represents to a useful fraction of a turn, so it and its sine and cosine are
+// taken in fp64; the rotation itself is fp32.
+__device__ __forceinline__ void inverse_rope_pair(float& a, float& b, int64_t t, int i, int rope_dims, float base) {
+  const double theta = pow(static_cast<double>(base), -2.0 * static_cast<double>(i) / static_cast<double>(rope_dims));
+  double sn, cs;
+  sincos(static_cast<double>(t) * theta, &sn, &cs);
+  const float c = static_cast<float>(cs), s = static_cast<float>(sn);
+  const float x = a, y = b;
+  a = x * c + y * s;
+  b = -x * s + y * c;
+}
+// applies it to four consecutive output channels ch0 .. ch0 + 3 (ch0 even) of a row of d_v channels
+__device__ __forceinline__ void inverse_rope4(float (&v)[4], int ch0, int d_v, int rope_dims, float base, int64_t t) {
+  if (rope_dims <= 0) return;
+  const int c0 = d_v - rope_dims;
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int ch = ch0 + 2 * e;
+    if (ch >= c0) inverse_rope_pair(v[2 * e], v[2 * e + 1], t, (ch - c0) >> 1, rope_dims, base);
+  }
+}
+
+// the score as the selection sees it: fp32, or rounded to bf16 (nearest even) when asked
+__device__ __forceinline__ float selected_score(float s, int bf16) {
+  return bf16 ? __bfloat162float(__float2bfloat16_rn(s)) : s;
+}
+
 // Order-preserving map float -> uint32 (larger float, larger key); -0 and
 // +0 map to the same key.
 __device__ __forceinline__ uint32_t f2key(float f) {

@@ -90,6 +90,7 @@ struct IndexParams {
   int32_t* out_cnt;
   float* out_scores;
   int32_t* status;
+  int score_bf16;       // scores rounded to bf16 before they are written (and selected)
   // workspace
   float* scores;        // [n_q, vis_stride]
   int64_t vis_stride;
@@ -128,6 +129,8 @@ struct AttendParams {
   const uint16_t* x_chunk;
   int64_t chunk_pos0, chunk_len;
   int32_t* status;
+  int rope_dims;    // inverse RoPE on the last rope_dims output channels (0: none)
+  float rope_base;
   // workspace / plan
   float* part_o;   // [n_q * max_splits * n_heads, d_v], or with part_t: [n_q * max_splits, d_v / 4, n_heads, 4]
   int part_t;      // part_o in the head-minor layout (written by attend_tc_kernel)

@@ -285,8 +285,8 @@ __global__ void __launch_bounds__(kScanThreads, 2) index_scan_kernel(IndexParams
       s1 += __shfl_xor_sync(kFull, s1, 2);
       if (!(wt.valid & (1u << s))) s0 = s1 = -INFINITY;
       if (c == 0) {
-        if (j + g < nv) out[j + g] = s0;
-        if (j + g + 8 < nv) out[j + g + 8] = s1;
+        if (j + g < nv) out[j + g] = selected_score(s0, p.score_bf16);
+        if (j + g + 8 < nv) out[j + g + 8] = selected_score(s1, p.score_bf16);
       }
     }
   };
@@ -527,6 +527,8 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
         s0 += __shfl_xor_sync(kFull, s0, 2);
         s1 += __shfl_xor_sync(kFull, s1, 1);
         s1 += __shfl_xor_sync(kFull, s1, 2);
+        s0 = selected_score(s0, p.score_bf16);
+        s1 = selected_score(s1, p.score_bf16);
       }
       if (c == 0) {
         float* out = p.scores + (int64_t)b * p.vis_stride;
@@ -788,8 +790,8 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
       if (writer) {
         const int64_t nv = nvw[nt];
         float* out = p.scores + (int64_t)(gs + m) * p.vis_stride;
-        if (j + pg < nv) out[j + pg] = s0;
-        if (j + pg + 8 < nv) out[j + pg + 8] = s1;
+        if (j + pg < nv) out[j + pg] = selected_score(s0, p.score_bf16);
+        if (j + pg + 8 < nv) out[j + pg + 8] = selected_score(s1, p.score_bf16);
       }
     }
     __syncwarp();

@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         float s = 0.f;
 #pragma unroll
         for (int h = 0; h < HI; ++h) s += w[m * HI + h] * fmaxf(__uint_as_float(d[m * HI + h]), 0.f);
-        if (m < gn && j < sNv[qb * kNQ + m]) p.scores[(int64_t)(gs + m) * p.vis_stride + j] = s;
+        if (m < gn && j < sNv[qb * kNQ + m]) p.scores[(int64_t)(gs + m) * p.vis_stride + j] = selected_score(s, p.score_bf16);
       }
     }
     if (cur_e >= 0 && ok) mbar_arrive(&qempty[qb]);

@@ -220,6 +220,13 @@ cskv_status cskv_cache_append(const cskv_append_args* args, void* stream);
  *   out_idx    [n_q, k] int32: ascending entry ids, -1 padded
  *   out_cnt    [n_q] int32: k_eff = min(k, visible entries)
  *   out_scores [n_q, k] fp32 or NULL: the score of each chosen entry (0 for padding)
+ *   score_bf16: 0 = select on the fp32 scores; 1 = round every score to bf16
+ *     (round to nearest even) before the selection, which then ranks the
+ *     rounded scores with the same order (entries whose scores round to the
+ *     same value are taken in index order); out_scores then holds the rounded
+ *     scores. Report digest section 7: the indexer's scores kept in BF16
+ *     rather than FP32 halve the selector's cost at 99.7% recall of the FP32
+ *     selection. A caller whose struct_size ends before this field gets 0.
  * The query dtype is layer->idx_dtype. Workspace: csa_index_ws_bytes().
  */
 typedef struct {
@@ -238,6 +245,7 @@ typedef struct {
   int32_t* out_cnt;
   float* out_scores;
   int32_t* d_status;
+  int32_t score_bf16;
 } cskv_index_args;
 
 cskv_status csa_index_ws_bytes(const cskv_index_args* args, size_t* bytes);
@@ -289,6 +297,16 @@ cskv_status csa_index_score_topk_static(const cskv_index_args* args, void* strea
  *   positions chunk_pos0 .. chunk_pos0 + chunk_len - 1 come from x_chunk
  *   [chunk_len, d_qk] bf16 instead (prefill of one sequence: the ring then
  *   still holds the tokens before the chunk).
+ *   rope_dims, rope_base: inverse RoPE on the output ("constraint chain"
+ *     essay, innovation 1: with many tokens sharing one compressed entry,
+ *     position is restored by an inverse-RoPE correction of the attention
+ *     output). When rope_dims > 0 (even, <= d_v), output channels
+ *     c0 + 2i, c0 + 2i + 1 (c0 = d_v - rope_dims) are rotated by -t theta_i,
+ *     theta_i = rope_base^(-2i / rope_dims), t = the query's position:
+ *     (a, b) <- (a cos + b sin, -a sin + b cos). It makes values that carry
+ *     RoPE at their key positions relative to the query; it is meaningful
+ *     when V includes the RoPE channels (d_v = d_qk). lse is unchanged.
+ *     A caller whose struct_size ends before these fields gets none.
  * Workspace: cskv_attend_ws_bytes().
  */
 typedef struct {
@@ -310,6 +328,8 @@ typedef struct {
   int64_t chunk_pos0;
   int64_t chunk_len;
   int32_t* d_status;
+  int32_t rope_dims;
+  float rope_base;
 } cskv_attend_args;
 
 cskv_status cskv_attend_ws_bytes(const cskv_attend_args* args, size_t* bytes);

@@ -39,7 +39,7 @@ def _fill(ck, L, B, n_e, g, sharp, fp8=False, std=None):
 
 
 def _run(ck, orc, kind, d_qk, d_v, H, positions, sharp=False, fp8=False, k=64, seed=0, with_lse=True,
-         sel_mode="random"):
+         sel_mode="random", rope_dims=0):
     B = len(positions)
     m = 4 if kind == "csa" else 128
     n_e = max(positions) // m + 2
@@ -64,9 +64,9 @@ def _run(ck, orc, kind, d_qk, d_v, H, positions, sharp=False, fp8=False, k=64, s
             sel[b, :c] = torch.from_numpy(ids.astype(np.int32))
             cnt[b] = c
         sel, cnt = sel.cuda(), cnt.cuda()
-        ck.csa_attend(L, seq, pos, max(positions), q, sel, cnt, out, lse, status=status)
+        ck.csa_attend(L, seq, pos, max(positions), q, sel, cnt, out, lse, status=status, rope_dims=rope_dims)
     else:
-        ck.hca_attend(L, seq, pos, max(positions), q, out, lse, status=status)
+        ck.hca_attend(L, seq, pos, max(positions), q, out, lse, status=status, rope_dims=rope_dims)
     assert ck.cskv_get_status(status) == ck.OK
     scale = 1.0 / math.sqrt(d_qk)
     atol, rel = (ATOL_LP, REL_LP) if fp8 else (ATOL_BF16, REL_BF16)
@@ -83,6 +83,8 @@ def _run(ck, orc, kind, d_qk, d_v, H, positions, sharp=False, fp8=False, k=64, s
             o, l = orc.attend(qb, orc.f64(keys), d_v, scale)
         else:
             o, l = orc.hca_query(t, m, 128, qb, win, ent if nv else ent.rows_subset(0, 0), d_v, scale)
+        if rope_dims:
+            o = orc.inverse_rope(o, d_v - rope_dims, rope_dims, t)
         assert_close(got_o[b], o, atol, rel, "%s o b=%d t=%d" % (kind, b, t))
         if with_lse:
             assert np.allclose(lse[b].cpu().numpy(), l, rtol=0, atol=2e-3), "lse b=%d" % b
@@ -174,7 +176,8 @@ def test_invalid_selection_is_reported(ck, orc):
     assert_close(out[0].float().cpu().numpy(), o, ATOL_BF16, REL_BF16, "masked")
 
 
-def _many(ck, orc, kind, n_q, n_seq, max_t, k=512, seed=0, sharp=False, short_every=0, bad_query=None):
+def _many(ck, orc, kind, n_q, n_seq, max_t, k=512, seed=0, sharp=False, short_every=0, bad_query=None,
+          rope_dims=0):
     """n_q queries (64 heads, d = 128) over n_seq sequences: enough queries for the query-pair
     tensor-core kernel (it takes calls with at least four queries per SM). Positions are random
     with the edge cases first; q_seq cycles through the sequences; a sample is checked.
@@ -220,9 +223,9 @@ def _many(ck, orc, kind, n_q, n_seq, max_t, k=512, seed=0, sharp=False, short_ev
             nv = orc.visible_entries(int(pos[i]), m, 128)
             sel[i, 1] = nv + 3
         ck.csa_attend(L, seq_t, pos_t, int(max_t), q, torch.from_numpy(sel).cuda(), torch.from_numpy(cnt).cuda(),
-                      out, lse, status=status)
+                      out, lse, status=status, rope_dims=rope_dims)
     else:
-        ck.hca_attend(L, seq_t, pos_t, int(max_t), q, out, lse, status=status)
+        ck.hca_attend(L, seq_t, pos_t, int(max_t), q, out, lse, status=status, rope_dims=rope_dims)
     want = ck.ERR_OUT_OF_RANGE if bad_query is not None else ck.OK
     assert ck.cskv_get_status(status) == want
     scale = 1.0 / math.sqrt(d)
@@ -243,6 +246,8 @@ def _many(ck, orc, kind, n_q, n_seq, max_t, k=512, seed=0, sharp=False, short_ev
             o, l = orc.attend(qb, orc.f64(keys), d, scale)
         else:
             o, l = orc.hca_query(t, m, 128, qb, win, ent if nv else ent.rows_subset(0, 0), d, scale)
+        if rope_dims:
+            o = orc.inverse_rope(o, d - rope_dims, rope_dims, t)
         assert_close(got_o[i], o, ATOL_BF16, REL_BF16, "%s many i=%d t=%d" % (kind, i, t))
         assert np.allclose(got_l[i], l, rtol=0, atol=2e-3), "lse i=%d" % i
 
