@@ -51,7 +51,7 @@ class LayerStruct(ctypes.Structure):
         ("n_seqs", _I32), ("max_pages_per_seq", _I32), ("n_pages", _I64),
         ("page_table", _P), ("kv_pool", _P), ("kv_scale", _P), ("idx_pool", _P), ("idx_scale", _P),
         ("ring_x", _P), ("ring_z", _P), ("ring_xi", _P), ("ring_zi", _P),
-        ("pos_bias", _P), ("pos_bias_idx", _P),
+        ("pos_bias", _P), ("pos_bias_idx", _P), ("overlap", _I32),
     ]
 
 
@@ -86,7 +86,7 @@ class AttendArgs(ctypes.Structure):
         ("n_heads", _I32), ("q_seq", _P), ("q_pos", _P), ("max_pos", _I64), ("q", _P),
         ("sel_idx", _P), ("sel_cnt", _P), ("k", _I32), ("sm_scale", ctypes.c_float), ("out", _P),
         ("lse", _P), ("x_chunk", _P), ("chunk_pos0", _I64), ("chunk_len", _I64), ("d_status", _P),
-        ("rope_dims", _I32), ("rope_base", ctypes.c_float),
+        ("rope_dims", _I32), ("rope_base", ctypes.c_float), ("chunk_desc", _P),
     ]
 
 
@@ -196,6 +196,7 @@ class Layer:
     ring_zi: torch.Tensor = None
     pos_bias: torch.Tensor = None
     pos_bias_idx: torch.Tensor = None
+    overlap: int = 0  # block overlap: an entry also folds the last `overlap` tokens of the block before it
     _struct: LayerStruct = field(default=None, repr=False)
 
     @property
@@ -206,7 +207,7 @@ class Layer:
         s = LayerStruct()
         s.struct_size = ctypes.sizeof(LayerStruct)
         for f in ("kind", "m", "n_win", "d_qk", "d_v", "d_idx", "page_size", "kv_dtype", "idx_dtype",
-                  "gate_cols", "gate_cols_idx", "n_seqs", "max_pages_per_seq", "n_pages"):
+                  "gate_cols", "gate_cols_idx", "n_seqs", "max_pages_per_seq", "n_pages", "overlap"):
             setattr(s, f, int(getattr(self, f)))
         return s
 
@@ -221,12 +222,12 @@ class Layer:
     def allocate(cls, kind: int, m: int, d_qk: int, d_v: int, n_seqs: int, n_pages: int,
                  max_pages_per_seq: int, page_size: int = 64, n_win: int = 128, d_idx: int = 0,
                  kv_dtype: int = BF16, idx_dtype: int = BF16, gate_cols: Optional[int] = None,
-                 gate_cols_idx: Optional[int] = None, device="cuda") -> "Layer":
+                 gate_cols_idx: Optional[int] = None, device="cuda", overlap: int = 0) -> "Layer":
         L = cls(kind=kind, m=m, n_win=n_win, d_qk=d_qk, d_v=d_v, d_idx=d_idx if kind == LAYER_CSA else 0,
                 page_size=page_size, kv_dtype=kv_dtype, idx_dtype=idx_dtype if kind == LAYER_CSA else BF16,
                 gate_cols=d_qk if gate_cols is None else gate_cols,
                 gate_cols_idx=(d_idx if gate_cols_idx is None else gate_cols_idx) if kind == LAYER_CSA else 1,
-                n_seqs=n_seqs, max_pages_per_seq=max_pages_per_seq, n_pages=n_pages)
+                n_seqs=n_seqs, max_pages_per_seq=max_pages_per_seq, n_pages=n_pages, overlap=overlap)
         sz = L.buffer_bytes()
         rows = n_pages * page_size
         u8 = dict(dtype=torch.uint8, device=device)
@@ -417,7 +418,7 @@ def csa_index_score_topk_static(layer: Layer, q_seq, q_pos, max_pos: int, q_idx,
 
 
 def _attend_args(layer, q_seq, q_pos, max_pos, q, sel_idx, sel_cnt, k, sm_scale, out, lse, x_chunk, chunk_pos0,
-                 status, n_q=None, n_heads=None, rope_dims=0, rope_base=10000.0):
+                 status, n_q=None, n_heads=None, rope_dims=0, rope_base=10000.0, chunk_desc=None):
     if q is not None:
         n_q, n_heads = q.shape[0], q.shape[1]
     if sm_scale is None:
@@ -426,7 +427,7 @@ def _attend_args(layer, q_seq, q_pos, max_pos, q, sel_idx, sel_cnt, k, sm_scale,
                       _ptr(q_pos), int(max_pos), _ptr(q), _ptr(sel_idx), _ptr(sel_cnt), int(k), float(sm_scale),
                       _ptr(out), _ptr(lse), _ptr(x_chunk), int(chunk_pos0),
                       0 if x_chunk is None else int(x_chunk.shape[0]), _ptr(status), int(rope_dims),
-                      float(rope_base))
+                      float(rope_base), _ptr(chunk_desc))
 
 
 def cskv_attend_ws_bytes(layer: Layer, n_q: int, n_heads: int, max_pos: int, k: int = 0) -> int:

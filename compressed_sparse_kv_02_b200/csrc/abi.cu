@@ -31,11 +31,18 @@ int sm_count() {
   return n;
 }
 
+// block overlap of a layer (0 for callers whose struct_size ends before the field)
+int32_t layer_overlap(const cskv_layer* L) {
+  return L->struct_size >= offsetof(cskv_layer, overlap) + sizeof(int32_t) ? L->overlap : 0;
+}
+
 // Shape/dtype rules of a layer (pointers not checked here).
 cskv_status check_layer_shape(const cskv_layer* L) {
-  if (!L || L->struct_size < sizeof(cskv_layer)) return CSKV_ERR_INVALID_ARG;
+  if (!L || L->struct_size < offsetof(cskv_layer, overlap)) return CSKV_ERR_INVALID_ARG;
   if (L->kind != CSKV_LAYER_CSA && L->kind != CSKV_LAYER_HCA) return CSKV_ERR_INVALID_ARG;
   if (L->n_win < 1 || !pow2(L->m) || L->m > L->n_win) return CSKV_ERR_INVALID_ARG;
+  // the ov tokens an entry borrows from the block before it must still be in the ring
+  if (layer_overlap(L) < 0 || layer_overlap(L) > L->n_win - L->m) return CSKV_ERR_INVALID_ARG;
   if (L->d_qk < 16 || L->d_qk > 1024 || L->d_qk % 16) return CSKV_ERR_INVALID_ARG;
   if (L->d_v < 16 || L->d_v > L->d_qk || L->d_v % 16) return CSKV_ERR_INVALID_ARG;
   if (L->page_size < 16 || L->page_size % 16) return CSKV_ERR_INVALID_ARG;
@@ -96,6 +103,7 @@ void fill_streams(FoldParams& p, const cskv_layer* L, const void* x, const void*
     p.n_streams = 2;
   }
   p.m = L->m;
+  p.ov = layer_overlap(L);
   p.n_win = L->n_win;
   p.page_size = L->page_size;
   p.max_pages_per_seq = L->max_pages_per_seq;
@@ -215,6 +223,7 @@ void fill_attend(AttendParams& p, const cskv_attend_args* a, int kind) {
   p.status = a->d_status;
   p.rope_dims = attend_rope_dims(a);
   p.rope_base = p.rope_dims > 0 ? a->rope_base : 0.f;
+  p.chunk_desc = a->struct_size >= offsetof(cskv_attend_args, chunk_desc) + sizeof(void*) ? a->chunk_desc : nullptr;
 }
 
 cskv_status attend_impl(const cskv_attend_args* a, void* ws, size_t ws_bytes, void* stream, int kind) {
@@ -274,7 +283,7 @@ cskv_status cskv_cache_append(const cskv_append_args* a, void* stream) {
   if ((s = check_layer_ptrs(L))) return s;
   if (a->n_seq < 0 || a->n_new < 0) return CSKV_ERR_INVALID_ARG;
   if (a->n_seq == 0 || a->n_new == 0) return CSKV_OK;
-  if (!a->ring_only && a->n_new + L->m - 1 > L->n_win) return CSKV_ERR_INVALID_ARG;
+  if (!a->ring_only && a->n_new + L->m - 1 + layer_overlap(L) > L->n_win) return CSKV_ERR_INVALID_ARG;
   if (a->ring_only && a->n_new > L->n_win) return CSKV_ERR_INVALID_ARG;
   const bool csa = L->kind == CSKV_LAYER_CSA;
   if (!a->seq_ids || !a->pos || !a->x || !a->z || !aligned16(a->x)) return CSKV_ERR_INVALID_ARG;

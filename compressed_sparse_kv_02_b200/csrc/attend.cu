@@ -65,8 +65,8 @@ __device__ __forceinline__ uintptr_t key_row(const AttendParams& p, int b, int s
   scale = 1.f;
   if (u < qk.n_w) {
     const int64_t pos = qk.ws + u;
-    if (p.x_chunk && pos >= p.chunk_pos0 && pos < p.chunk_pos0 + p.chunk_len)
-      return reinterpret_cast<uintptr_t>(p.x_chunk + (pos - p.chunk_pos0) * p.d_qk);
+    const int64_t cr = chunk_row(p, seq, pos);
+    if (cr >= 0) return reinterpret_cast<uintptr_t>(p.x_chunk + cr * p.d_qk);
     return reinterpret_cast<uintptr_t>(p.ring_x + ((int64_t)seq * p.n_win + pos % p.n_win) * p.d_qk);
   }
   const int64_t jj = u - qk.n_w;

@@ -119,8 +119,8 @@ __device__ __forceinline__ uint32_t key_code(const AttendParams& p, int b, int s
   if (u < k.n_w) {
     if (!p.x_chunk) return (2u << kRowBits) | static_cast<uint32_t>((int64_t)seq * p.n_win + u);
     const int64_t pos = k.ws + u;
-    if (pos >= p.chunk_pos0 && pos < p.chunk_pos0 + p.chunk_len)
-      return (3u << kRowBits) | static_cast<uint32_t>(pos - p.chunk_pos0);
+    const int64_t cr = chunk_row(p, seq, pos);
+    if (cr >= 0) return (3u << kRowBits) | static_cast<uint32_t>(cr);
     return (2u << kRowBits) | static_cast<uint32_t>((int64_t)seq * p.n_win + pos % p.n_win);
   }
   const int64_t jj = u - k.n_w;

@@ -54,6 +54,7 @@ struct FoldParams {
   FoldStream s[2];
   int n_streams;
   int m, n_win, page_size, max_pages_per_seq;
+  int ov;  // block overlap: an entry also folds the last ov tokens of the block before it
   int64_t n_pages;
   const int32_t* page_table;
   int n_seq;
@@ -131,6 +132,7 @@ struct AttendParams {
   int32_t* status;
   int rope_dims;    // inverse RoPE on the last rope_dims output channels (0: none)
   float rope_base;
+  const int64_t* chunk_desc;  // [n_seqs_layer, 3] (first row, first position, length) of each sequence's chunk, or null
   // workspace / plan
   float* part_o;   // [n_q * max_splits * n_heads, d_v], or with part_t: [n_q * max_splits, d_v / 4, n_heads, 4]
   int part_t;      // part_o in the head-minor layout (written by attend_tc_kernel)
@@ -140,6 +142,26 @@ struct AttendParams {
 };
 
 size_t attend_ws_bytes(const AttendParams& p, int n_sm);
+
+// Row of x_chunk that holds position pos of sequence seq, or -1 (the row is then in the ring).
+// One sequence (no chunk_desc): x_chunk holds positions chunk_pos0 .. chunk_pos0 + chunk_len - 1.
+// Several (chunk_desc): sequence s's chunk sits at rows desc[s][0] .. + desc[s][2] - 1 of x_chunk
+// and holds positions desc[s][1] .. + desc[s][2] - 1; x_chunk has chunk_len rows in all. A
+// descriptor that points outside x_chunk is reported and its rows read from the ring.
+__device__ __forceinline__ int64_t chunk_row(const AttendParams& p, int seq, int64_t pos) {
+  if (!p.x_chunk) return -1;
+  int64_t r0 = 0, p0 = p.chunk_pos0, len = p.chunk_len;
+  if (p.chunk_desc) {
+    r0 = p.chunk_desc[3 * (int64_t)seq];
+    p0 = p.chunk_desc[3 * (int64_t)seq + 1];
+    len = p.chunk_desc[3 * (int64_t)seq + 2];
+    if (r0 < 0 || len < 0 || r0 + len > p.chunk_len) {
+      if (p.status) atomicCAS(p.status, 0, CSKV_ERR_OUT_OF_RANGE);
+      return -1;
+    }
+  }
+  return (pos >= p0 && pos < p0 + len) ? r0 + pos - p0 : -1;
+}
 cudaError_t launch_attend(AttendParams& p, void* ws, int n_sm, cudaStream_t st);
 bool attend_supported(int d_qk, int d_v, int n_heads, int kv_dtype);
 cudaError_t launch_attend_merge(AttendParams& p, cudaStream_t st);

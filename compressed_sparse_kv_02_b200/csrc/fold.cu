@@ -39,10 +39,13 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
 }
 
 // Online-softmax partial state of channels [c0, c0+8) over tokens i0 .. i1-1
-// of one block: running max (of the logits times log2 e), denominator and
-// weighted sum (fp32). rows(i, xr, zr) yields token i's raw row and gate row.
+// of one block (token i < 0 is one of the ov tokens of the previous block that
+// the entry overlaps): running max (of the logits times log2 e), denominator
+// and weighted sum (fp32). rows(i, xr, zr) yields token i's raw row and gate
+// row, or false when the token lies before the start of the stream; the
+// position bias row of token i is i + ov.
 template <class Rows>
-__device__ __forceinline__ void fold_partial(const FoldStream& S, int i0, int i1, int c0, Rows rows,
+__device__ __forceinline__ void fold_partial(const FoldStream& S, int i0, int i1, int c0, Rows rows, int ov,
                                              float (&mx)[8], float (&den)[8], float (&acc)[8]) {
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
@@ -54,7 +57,7 @@ __device__ __forceinline__ void fold_partial(const FoldStream& S, int i0, int i1
   for (int i = i0; i < i1; ++i) {
     const uint16_t* xr;
     const uint16_t* zr;
-    rows(i, xr, zr);
+    if (!rows(i, xr, zr)) continue;
     float xf[8], zl[8];
     unpack8(ldg16(xr + c0), xf);
     if (S.gc == 1) {
@@ -66,7 +69,7 @@ __device__ __forceinline__ void fold_partial(const FoldStream& S, int i0, int i1
     }
     if (S.bias) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) zl[e] += S.bias[(int64_t)i * S.d + c0 + e];
+      for (int e = 0; e < 8; ++e) zl[e] += S.bias[(int64_t)(i + ov) * S.d + c0 + e];
     }
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -86,10 +89,10 @@ __device__ __forceinline__ void fold_partial(const FoldStream& S, int i0, int i1
 
 // Fold channels [c0, c0+8) over tokens i0 .. i1-1 (a whole block) into out.
 template <class Rows>
-__device__ __forceinline__ void fold_group(const FoldStream& S, int m, int i0, int i1, int c0, Rows rows,
+__device__ __forceinline__ void fold_group(const FoldStream& S, int m, int i0, int i1, int c0, Rows rows, int ov,
                                            float (&out)[8]) {
   float mx[8], den[8], acc[8];
-  fold_partial(S, i0, i1, c0, rows, mx, den, acc);
+  fold_partial(S, i0, i1, c0, rows, ov, mx, den, acc);
 #pragma unroll
   for (int e = 0; e < 8; ++e) out[e] = acc[e] / den[e];
 }
@@ -166,7 +169,7 @@ __device__ __forceinline__ void store_groups(const FoldStream& S, int64_t row, i
 // Fold one entry with one warp (small m: every lane runs the m tokens of its
 // channel groups) and store it at pool row `row`.
 template <class Rows>
-__device__ void fold_entry_warp(const FoldStream& S, int m, int64_t row, Rows rows) {
+__device__ void fold_entry_warp(const FoldStream& S, int m, int ov, int64_t row, Rows rows) {
   const int lane = threadIdx.x & 31;
   const int G = S.d / 8;
   float v[kGroupsPerLane][8];
@@ -175,7 +178,7 @@ __device__ void fold_entry_warp(const FoldStream& S, int m, int64_t row, Rows ro
   for (int gi = 0; gi < kGroupsPerLane; ++gi) {
     const int grp = lane + 32 * gi;
     if (grp < G) {
-      fold_group(S, m, 0, m, grp * 8, rows, v[gi]);
+      fold_group(S, m, -ov, m, grp * 8, rows, ov, v[gi]);
 #pragma unroll
       for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[gi][e]));
     }
@@ -191,21 +194,22 @@ __device__ void fold_entry_warp(const FoldStream& S, int m, int64_t row, Rows ro
 // merged through shared memory. `sm` holds 3 * blockDim.x * 8 floats. For an
 // FP8 entry the range must be the whole row (its scale is the row's amax).
 template <class Rows>
-__device__ void fold_entry_block(const FoldStream& S, int m, int64_t row, Rows rows, float* sm, int c_lo,
+__device__ void fold_entry_block(const FoldStream& S, int m, int ov, int64_t row, Rows rows, float* sm, int c_lo,
                                  int c_hi) {
   const int G = (c_hi - c_lo) / 8;
   const int t = threadIdx.x;
+  const int nt = m + ov;    // tokens of the entry: -ov .. m - 1
   int ns = blockDim.x / G;  // token slices
-  if (ns > m) ns = m;
-  const int per = (m + ns - 1) / ns;
+  if (ns > nt) ns = nt;
+  const int per = (nt + ns - 1) / ns;
   const int g = t % G, sl = t / G;
   float* smx = sm;
   float* sden = sm + blockDim.x * 8;
   float* sacc = sm + 2 * blockDim.x * 8;
   if (sl < ns) {
     float mx[8], den[8], acc[8];
-    const int i0 = sl * per, i1 = min(m, i0 + per);
-    fold_partial(S, i0, i1, c_lo + g * 8, rows, mx, den, acc);
+    const int i0 = sl * per - ov, i1 = min(m, i0 + per);
+    fold_partial(S, i0, i1, c_lo + g * 8, rows, ov, mx, den, acc);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       smx[(sl * G + g) * 8 + e] = mx[e];
@@ -274,13 +278,27 @@ __device__ __forceinline__ int64_t entry_row(const FoldParams& p, int seq, int64
 constexpr int kWarpFoldMaxM = 16;  // up to this many tokens per entry one warp folds an entry
 constexpr int kBlockFoldThreads = 512;
 
-// rows of the bulk input: token i of entry jj of row block b
+// rows of the bulk input: token i of entry jj of row block b (input row t0 + i,
+// stream position pos0 + i); an overlap token before the segment's first
+// position comes from the sequence's ring, one before position 0 does not exist
 struct BulkRows {
   const FoldStream* S;
-  int64_t t0;
-  __device__ void operator()(int i, const uint16_t*& xr, const uint16_t*& zr) const {
-    xr = S->x + (t0 + i) * S->d;
-    zr = S->z + (t0 + i) * S->gc;
+  int64_t t0, seg0, pos0;  // input row of token 0, input row of the segment start, position of token 0
+  int64_t tok0;            // position of the segment's first token
+  int64_t ring_row0;       // seq * n_win
+  int n_win;
+  __device__ bool operator()(int i, const uint16_t*& xr, const uint16_t*& zr) const {
+    const int64_t pos = pos0 + i;
+    if (pos < 0) return false;
+    if (pos >= tok0) {
+      xr = S->x + (t0 + i) * S->d;
+      zr = S->z + (t0 + i) * S->gc;
+    } else {
+      const int64_t r = ring_row0 + pos % n_win;
+      xr = S->ring_x + r * S->d;
+      zr = S->ring_z + r * S->gc;
+    }
+    return true;
   }
 };
 
@@ -293,6 +311,11 @@ __device__ __forceinline__ void bulk_item(const FoldParams& p, int64_t it, int& 
   row = entry_row(p, p.seq_ids[b], p.tok0 / p.m + jj);
   r.S = &p.s[si];
   r.t0 = (int64_t)b * p.n_tok + jj * p.m;
+  r.seg0 = (int64_t)b * p.n_tok;
+  r.pos0 = p.tok0 + jj * p.m;
+  r.tok0 = p.tok0;
+  r.ring_row0 = (int64_t)p.seq_ids[b] * p.n_win;
+  r.n_win = p.n_win;
 }
 
 // small m (CSA): one warp per entry
@@ -305,7 +328,7 @@ __global__ void __launch_bounds__(256) fold_bulk_warp_kernel(FoldParams p) {
     int64_t row;
     BulkRows r;
     bulk_item(p, it, si, row, r);
-    if (row >= 0) fold_entry_warp(p.s[si], p.m, row, r);
+    if (row >= 0) fold_entry_warp(p.s[si], p.m, p.ov, row, r);
   }
 }
 
@@ -318,7 +341,7 @@ __global__ void __launch_bounds__(kBlockFoldThreads) fold_bulk_block_kernel(Fold
     int64_t row;
     BulkRows r;
     bulk_item(p, it, si, row, r);
-    if (row >= 0) fold_entry_block(p.s[si], p.m, row, r, sm, 0, p.s[si].d);  // row is uniform across the block
+    if (row >= 0) fold_entry_block(p.s[si], p.m, p.ov, row, r, sm, 0, p.s[si].d);  // row is uniform across the block
   }
 }
 
@@ -436,9 +459,10 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
   // blocks completed by positions pos .. pos+n_new-1
   const int64_t j_first = pos / p.m;                 // first block ending at or after pos
   const int64_t j_last = (pos + p.n_new) / p.m - 1;  // last block ending before pos+n_new
-  // every thread folds a channel pair over a group of the block's tokens (tokens tg, tg + 16, ...);
-  // the 16 groups' partial states (running max in base 2, denominator, weighted sum) then merge
-  // per channel through shared memory
+  // every thread folds a channel pair over a group of the entry's tokens (tokens tg - ov,
+  // tg - ov + 16, ... of the block, the first ov of them the overlap with the block before); the 16
+  // groups' partial states (running max in base 2, denominator, weighted sum) then merge per
+  // channel through shared memory
   const int cp = t % kFoldPairs, tg = t / kFoldPairs;
   for (int64_t j = j_first; j <= j_last; ++j) {
     const int64_t row = entry_row(p, seq, j);  // uniform across the block
@@ -446,8 +470,9 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
       const int c = c0 + 2 * cp;
       const bool active = c < c_hi;
       float mx[2] = {-INFINITY, -INFINITY}, den[2] = {0.f, 0.f}, acc[2] = {0.f, 0.f};
-      for (int i = tg; active && i < p.m; i += kFoldGroups) {
+      for (int i = tg - p.ov; active && i < p.m; i += kFoldGroups) {
         const int64_t q = j * p.m + i;
+        if (q < 0) continue;  // before the start of the stream
         const uint16_t* xr;
         const uint16_t* zr;
         if (q >= pos) {
@@ -470,7 +495,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
         const float xf[2] = {__uint_as_float(xv << 16), __uint_as_float(xv & 0xffff0000u)};
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const float bias = S.bias ? S.bias[(int64_t)i * S.d + c + e] : 0.f;
+          const float bias = S.bias ? S.bias[(int64_t)(i + p.ov) * S.d + c + e] : 0.f;
           const float l2 = (zl[e] + bias) * kLog2e;  // base-2 weights: 2^(l2 - max) = e^(z - max_z)
           const float M = fmaxf(mx[e], l2);
           const float corr = mx[e] == -INFINITY ? 0.f : exp2f(mx[e] - M);
@@ -490,7 +515,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
       }
       __syncthreads();
       if (t < 2 * kFoldPairs && c0 + t < c_hi) {  // one thread per channel merges the groups that ran tokens
-        const int ng = p.m < kFoldGroups ? p.m : kFoldGroups;
+        const int ng = p.m + p.ov < kFoldGroups ? p.m + p.ov : kFoldGroups;
         float M = -INFINITY;
         for (int gi = 0; gi < ng; ++gi) M = fmaxf(M, s_mx[gi][t]);
         float dd = 0.f, aa = 0.f;

@@ -200,3 +200,170 @@ def main(argv=None) -> int:
 
 if __name__ == "__main__":
     raise SystemExit(main())
+
+
+class VarlenPrefillModel:
+    """One prefill pass over several sequences at once, each with its own cached length and chunk length
+    (DeepSeek-V4 report digest, section 7 / Figure 6: the state cache carries each sequence's window
+    between chunks; 10100.com article, section 6: the compressed cache is extended chunk by chunk).
+
+    Sequence b holds cached[b] tokens (compressed entries plus its last n_win raw rows in the rings) and
+    receives chunk[b] new tokens. The chunks are packed one after another: query row r of the pass is
+    position cached[b] + i of sequence b. One pass:
+      rings  : restored to the cached state (one ring-only append for all sequences)
+      fold   : csa_compress_kv / hca_compress_kv of each sequence's chunk (its own tok0 and length)
+      blocks of up to q_block query rows, spanning sequences:
+               csa_index_score_topk -> csa_attend, hca_attend, with the packed chunk rows and a
+               per-sequence chunk descriptor (first row, first position, length) for the window rows
+      rings  : the last n_win rows of every chunk (one ring-only append for all sequences).
+    cached[b] and chunk[b] are multiples of m' = 128, cached[b] >= n_win, chunk[b] >= n_win.
+    """
+
+    def __init__(self, cfg: synth.Config, cached, chunk, device="cuda", q_block: int = 4096):
+        cached, chunk = [int(c) for c in cached], [int(c) for c in chunk]
+        if len(cached) != len(chunk) or not cached:
+            raise ValueError("one cached and one chunk length per sequence")
+        for c0, T in zip(cached, chunk):
+            if c0 % cfg.m_hca or T % cfg.m_hca or c0 < cfg.n_win or T < cfg.n_win:
+                raise ValueError("cached and chunk lengths must be multiples of m' and at least n_win")
+        self.cfg, self.device = cfg, device
+        self.cached, self.chunk = cached, chunk
+        self.n_seqs = Bn = len(cached)
+        self.total = sum(chunk)
+        self.q_block = min(q_block, self.total)
+        self.row0 = [sum(chunk[:b]) for b in range(Bn)]
+        ends = [c0 + T for c0, T in zip(cached, chunk)]
+        self.max_pos = max(ends) - 1
+        P = cfg.page_size
+        self.layers = []
+        for kind, m in ((B.LAYER_CSA, cfg.m_csa), (B.LAYER_HCA, cfg.m_hca)):
+            pages = [-(-(n // m) // P) for n in ends]
+            L = B.Layer.allocate(kind, m, cfg.d_qk, cfg.d_v, n_seqs=Bn, n_pages=sum(pages),
+                                 max_pages_per_seq=max(pages), page_size=P, n_win=cfg.n_win, d_idx=cfg.d_idx,
+                                 device=device)
+            perm = synth.page_permutation(sum(pages), cfg.seed, 700 + kind, device)
+            o = 0
+            for b, npg in enumerate(pages):
+                L.set_pages(b, perm[o:o + npg])
+                o += npg
+            self.layers.append(L)
+        self.seq = torch.arange(Bn, dtype=torch.int32, device=device)
+        self.q_seq = torch.cat([torch.full((T,), b, dtype=torch.int32) for b, T in enumerate(chunk)]).to(device)
+        self.q_pos = torch.cat([torch.arange(c0, c0 + T, dtype=torch.int64)
+                                for c0, T in zip(cached, chunk)]).to(device)
+        self.chunk_desc = torch.tensor([[self.row0[b], cached[b], chunk[b]] for b in range(Bn)], dtype=torch.int64,
+                                       device=device)
+        H, k = cfg.heads, cfg.k
+        self.idx = torch.zeros(self.total, k, dtype=torch.int32, device=device)
+        self.cnt = torch.zeros(self.total, dtype=torch.int32, device=device)
+        self.o_csa = torch.zeros(self.total, H, cfg.d_v, dtype=torch.bfloat16, device=device)
+        self.o_hca = torch.zeros(self.total, H, cfg.d_v, dtype=torch.bfloat16, device=device)
+        csa, hca = self.layers
+        qb = self.q_block
+        self.ws_index = torch.empty(B.csa_index_ws_bytes(csa, qb, cfg.heads_idx, self.max_pos, k), dtype=torch.uint8,
+                                    device=device)
+        self.ws_csa = torch.empty(B.cskv_attend_ws_bytes(csa, qb, H, self.max_pos, k), dtype=torch.uint8,
+                                  device=device)
+        self.ws_hca = torch.empty(B.cskv_attend_ws_bytes(hca, qb, H, self.max_pos), dtype=torch.uint8,
+                                  device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.inputs = None
+        self._calls = None
+
+    def fill_synthetic(self):
+        """Per sequence: cached entries in stored form, the cached tail as raw rows; the packed chunks and
+        their queries."""
+        cfg, dev = self.cfg, self.device
+        s = cfg.seed
+        csa, hca = self.layers
+        d, di, nw = cfg.d_qk, cfg.d_idx, cfg.n_win
+        for b, c0 in enumerate(self.cached):
+            csa.write_entries(b, 0, kv=synth.normal((c0 // cfg.m_csa, d), 1.0 / math.sqrt(d),
+                                                    synth.generator(s, 100 + b, dev), dev),
+                              idx=synth.normal((c0 // cfg.m_csa, di), 1.0, synth.generator(s, 200 + b, dev), dev))
+            hca.write_entries(b, 0, kv=synth.normal((c0 // cfg.m_hca, d), 1.0 / math.sqrt(d),
+                                                    synth.generator(s, 300 + b, dev), dev))
+        inp = {}
+        for name, dd, st in (("x", d, 10), ("xi", di, 20), ("x_h", d, 30)):
+            tail_x, tail_z = synth.raw_stream(self.n_seqs, nw, dd, s, st, dev)
+            x, z = synth.raw_stream(1, self.total, dd, s, st + 2, dev)
+            inp["tail_" + name], inp["tail_z" + name[1:]] = tail_x, tail_z
+            inp[name], inp["z" + name[1:]] = x[0], z[0]  # packed chunks [total, dd]
+        inp["q"] = synth.normal((self.total, cfg.heads, d), 1.0, synth.generator(s, 40, dev), dev)
+        inp["q_h"] = synth.normal((self.total, cfg.heads, d), 1.0, synth.generator(s, 41, dev), dev)
+        inp["q_idx"] = synth.normal((self.total, cfg.heads_idx, di), 1.0, synth.generator(s, 42, dev), dev)
+        inp["w"] = synth.uniform((self.total, cfg.heads_idx), 0.0, 1.0, synth.generator(s, 43, dev), dev)
+        self.inputs = inp
+        torch.cuda.synchronize()
+
+    def prepare(self):
+        L = B.lib()
+        cfg, inp, qb, nw = self.cfg, self.inputs, self.q_block, self.cfg.n_win
+        csa, hca = self.layers
+        sm = 1.0 / math.sqrt(cfg.d_qk)
+        keep = [csa.struct, hca.struct]
+        lc, lh = ctypes.pointer(keep[0]), ctypes.pointer(keep[1])
+        calls = []
+        Bn = self.n_seqs
+        tail_pos = torch.tensor([c0 - nw for c0 in self.cached], dtype=torch.int64, device=self.device)
+        end_pos = torch.tensor([c0 + T - nw for c0, T in zip(self.cached, self.chunk)], dtype=torch.int64,
+                               device=self.device)
+        # the last n_win rows of every chunk, stacked [n_seqs, n_win, d]
+        last = {k_: torch.stack([inp[k_][r + T - nw:r + T] for r, T in zip(self.row0, self.chunk)]).contiguous()
+                for k_ in ("x", "z", "xi", "zi", "x_h", "z_h")}
+        chunks = []  # per-sequence chunk views [1, T, d] for the folds
+        for b, (r, T) in enumerate(zip(self.row0, self.chunk)):
+            chunks.append({k_: inp[k_][r:r + T].unsqueeze(0).contiguous()
+                           for k_ in ("x", "z", "xi", "zi", "x_h", "z_h")})
+        self._keep_tensors = (tail_pos, end_pos, last, chunks)
+        calls.append(_Call(L.cskv_cache_append, B.AppendArgs(
+            ctypes.sizeof(B.AppendArgs), lc, Bn, nw, B._ptr(self.seq), B._ptr(tail_pos), B._ptr(inp["tail_x"]),
+            B._ptr(inp["tail_z"]), B._ptr(inp["tail_xi"]), B._ptr(inp["tail_zi"]), 1, B._ptr(self.status)),
+            where="cskv_cache_append"))
+        calls.append(_Call(L.cskv_cache_append, B.AppendArgs(
+            ctypes.sizeof(B.AppendArgs), lh, Bn, nw, B._ptr(self.seq), B._ptr(tail_pos), B._ptr(inp["tail_x_h"]),
+            B._ptr(inp["tail_z_h"]), None, None, 1, B._ptr(self.status)), where="cskv_cache_append"))
+        for b in range(Bn):
+            c = chunks[b]
+            sq = self.seq[b:b + 1]
+            calls.append(_Call(L.csa_compress_kv, B.CompressArgs(
+                ctypes.sizeof(B.CompressArgs), lc, 1, B._ptr(sq), self.cached[b], self.chunk[b], B._ptr(c["x"]),
+                B._ptr(c["z"]), B._ptr(c["xi"]), B._ptr(c["zi"]), B._ptr(self.status)), where="csa_compress_kv"))
+            calls.append(_Call(L.hca_compress_kv, B.CompressArgs(
+                ctypes.sizeof(B.CompressArgs), lh, 1, B._ptr(sq), self.cached[b], self.chunk[b], B._ptr(c["x_h"]),
+                B._ptr(c["z_h"]), None, None, B._ptr(self.status)), where="hca_compress_kv"))
+        for q0 in range(0, self.total, qb):
+            sl = slice(q0, min(self.total, q0 + qb))
+            ia = B._index_args(csa, self.q_seq[sl], self.q_pos[sl], self.max_pos, inp["q_idx"][sl], inp["w"][sl],
+                               cfg.k, self.idx[sl], self.cnt[sl], None, None, self.status)
+            ia.layer = lc
+            calls.append(_Call(L.csa_index_score_topk, ia, self.ws_index, "csa_index_score_topk"))
+            aa = B._attend_args(csa, self.q_seq[sl], self.q_pos[sl], self.max_pos, inp["q"][sl], self.idx[sl],
+                                self.cnt[sl], cfg.k, sm, self.o_csa[sl], None, inp["x"], 0, self.status,
+                                chunk_desc=self.chunk_desc)
+            aa.layer = lc
+            calls.append(_Call(L.csa_attend, aa, self.ws_csa, "csa_attend"))
+            ha = B._attend_args(hca, self.q_seq[sl], self.q_pos[sl], self.max_pos, inp["q_h"][sl], None, None, 0, sm,
+                                self.o_hca[sl], None, inp["x_h"], 0, self.status, chunk_desc=self.chunk_desc)
+            ha.layer = lh
+            calls.append(_Call(L.hca_attend, ha, self.ws_hca, "hca_attend"))
+        calls.append(_Call(L.cskv_cache_append, B.AppendArgs(
+            ctypes.sizeof(B.AppendArgs), lc, Bn, nw, B._ptr(self.seq), B._ptr(end_pos), B._ptr(last["x"]),
+            B._ptr(last["z"]), B._ptr(last["xi"]), B._ptr(last["zi"]), 1, B._ptr(self.status)),
+            where="cskv_cache_append"))
+        calls.append(_Call(L.cskv_cache_append, B.AppendArgs(
+            ctypes.sizeof(B.AppendArgs), lh, Bn, nw, B._ptr(self.seq), B._ptr(end_pos), B._ptr(last["x_h"]),
+            B._ptr(last["z_h"]), None, None, 1, B._ptr(self.status)), where="cskv_cache_append"))
+        self._keep = keep
+        self._calls = calls
+        return calls
+
+    def step(self, stream=None):
+        if self._calls is None:
+            self.prepare()
+        st = B._stream(stream)
+        for c in self._calls:
+            c(st)
+
+    def check_status(self) -> int:
+        return B.cskv_get_status(self.status)

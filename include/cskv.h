@@ -103,6 +103,15 @@ typedef int32_t cskv_status;
  *   ring_z  [n_seqs, n_win, gate_cols]  bf16 gate logits of the KV stream
  *   ring_xi [n_seqs, n_win, d_idx]      bf16 raw indexer keys (CSA)
  *   ring_zi [n_seqs, n_win, gate_cols_idx] bf16 gate logits of the indexer-key stream (CSA)
+ * Block overlap (10100.com article, section 2.1: block compression with
+ * position weighting and block overlap; the width is a reading): with
+ * overlap = ov > 0, entry j folds the tokens at positions max(0, j*m - ov) ..
+ * j*m + m - 1 under one softmax (the last ov tokens of the block before it
+ * too), and pos_bias / pos_bias_idx have m + ov rows, row r for the token at
+ * position j*m - ov + r. The entry is complete when its own block is, so
+ * visibility does not change. Requires ov <= n_win - m; a bulk compression
+ * that starts at tok0 > 0 reads the ov tokens before tok0 from the ring.
+ * overlap = 0 (or a struct_size that ends before the field) is the plain fold.
  * Constraints: m a power of two with m <= n_win; page_size a multiple of 16;
  * d_qk, d_v, d_idx multiples of 16 (d_idx of 32 for FP4); d_v <= d_qk.
  */
@@ -131,8 +140,9 @@ typedef struct {
   void* ring_z;
   void* ring_xi;
   void* ring_zi;
-  const float* pos_bias;     /* [m, d_qk] fp32 or NULL (position weighting) */
-  const float* pos_bias_idx; /* [m, d_idx] fp32 or NULL */
+  const float* pos_bias;     /* [m + overlap, d_qk] fp32 or NULL (position weighting) */
+  const float* pos_bias_idx; /* [m + overlap, d_idx] fp32 or NULL */
+  int32_t overlap;           /* block overlap ov (0 = none) */
 } cskv_layer;
 
 /*
@@ -187,9 +197,9 @@ cskv_status hca_compress_kv(const cskv_compress_args* args, void* stream);
  *   seq_ids [n_seq], pos [n_seq] int64
  *   x [n_seq, n_new, d_qk], z [n_seq, n_new, gate_cols],
  *   xi [n_seq, n_new, d_idx], zi [n_seq, n_new, gate_cols_idx] (CSA)
- * Requires n_new + m - 1 <= n_win (every completed block is still in the
- * ring). ring_only = 1 writes the rings and emits nothing (used after a bulk
- * compression of the same tokens).
+ * Requires n_new + m - 1 + overlap <= n_win (every completed block, and the
+ * tokens it overlaps, are still in the ring). ring_only = 1 writes the rings
+ * and emits nothing (used after a bulk compression of the same tokens).
  */
 typedef struct {
   uint32_t struct_size;
@@ -307,6 +317,13 @@ cskv_status csa_index_score_topk_static(const cskv_index_args* args, void* strea
  *     RoPE at their key positions relative to the query; it is meaningful
  *     when V includes the RoPE channels (d_v = d_qk). lse is unchanged.
  *     A caller whose struct_size ends before these fields gets none.
+ *   chunk_desc [n_seqs, 3] int64 or NULL: prefill of several sequences in one
+ *     call (varlen). Sequence s's chunk rows are rows chunk_desc[s][0] ..
+ *     chunk_desc[s][0] + chunk_desc[s][2] - 1 of x_chunk and hold its
+ *     positions chunk_desc[s][1] .. + chunk_desc[s][2] - 1 (length 0: none);
+ *     chunk_len is then the number of rows of x_chunk and chunk_pos0 is not
+ *     used. Window rows outside a sequence's chunk come from its ring. A
+ *     descriptor outside x_chunk is reported (CSKV_ERR_OUT_OF_RANGE).
  * Workspace: cskv_attend_ws_bytes().
  */
 typedef struct {
@@ -330,6 +347,7 @@ typedef struct {
   int32_t* d_status;
   int32_t rope_dims;
   float rope_base;
+  const int64_t* chunk_desc;
 } cskv_attend_args;
 
 cskv_status cskv_attend_ws_bytes(const cskv_attend_args* args, size_t* bytes);

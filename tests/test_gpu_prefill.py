@@ -87,3 +87,64 @@ def test_prefill_chunk(ck, orc):
     assert model.check_status() == ck.OK
     for a, b in zip(before, [model.idx, model.o_csa, model.o_hca]):
         assert torch.equal(a, b)
+
+
+def test_varlen_prefill_several_sequences(ck, orc):
+    """Several sequences with their own cached and chunk lengths in one pass: the folds per sequence,
+    the indexer and both attentions over query blocks that span sequences (the window rows of each
+    from its own packed chunk through the chunk descriptor, or from its ring), and the rings after the
+    pass. Blocks of 512 rows cross sequence boundaries; 1024 + 640 + 384 rows in all."""
+    from compressed_sparse_kv_02_b200 import prefill, synth
+    cfg = synth.Config("prefill_varlen", 3, 6144 + 1024, 64, 128, 128, 4, 64, 256, seed=13)
+    cached, chunk = [6144, 1024, 2048], [1024, 640, 384]
+    model = prefill.VarlenPrefillModel(cfg, cached, chunk, q_block=512)
+    model.fill_synthetic()
+    model.step()
+    torch.cuda.synchronize()
+    assert model.check_status() == ck.OK
+    csa, hca = model.layers
+    inp = model.inputs
+    scale = 1.0 / math.sqrt(cfg.d_qk)
+    heads = np.array([0, 31, 63])
+    for b, (c0, T) in enumerate(zip(cached, chunk)):
+        r0 = model.row0[b]
+        # the chunk's entries, folded from its raw rows
+        for L, xs, zs, m in ((csa, "x", "z", 4), (hca, "x_h", "z_h", 128)):
+            got = L.read_entries(b, T // m, c0 // m)
+            x, z = inp[xs][r0:r0 + T].cpu(), inp[zs][r0:r0 + T].cpu()
+            ref = orc.store(orc.compress(stored_bf16(x), stored_bf16(z), m), orc.BF16)
+            assert_fold_close(orc.decode(stored_bf16(got["kv"])), orc.decode(ref), orc.decode(stored_bf16(x)), m,
+                              "seq %d entries m=%d" % (b, m))
+
+        def window(name, t):
+            rows = []
+            for p in range(max(0, t - 127), t + 1):
+                rows.append(inp[name][r0 + p - c0].cpu() if p >= c0 else
+                            inp["tail_" + name][b, p - (c0 - 128)].cpu())
+            return stored_bf16(torch.stack(rows))
+
+        for t in (c0, c0 + 1, c0 + 127, c0 + 128, c0 + T // 2 + 3, c0 + T - 1):
+            i = r0 + t - c0
+            nv = orc.visible_entries(t, 4, 128)
+            nv_h = orc.visible_entries(t, 128, 128)
+            ent = layer_entries(csa, b, nv)
+            sc = orc.index_scores(stored_bf16(inp["q_idx"][i]), inp["w"][i].double().cpu().numpy(), ent["idx"], nv)
+            idx = model.idx[i].cpu().numpy()
+            cnt = int(model.cnt[i])
+            check_topk(idx, cnt, sc, cfg.k)
+            keys = np.vstack([orc.decode(window("x", t)), orc.decode(ent["kv"].take_rows(idx[:cnt]))])
+            o, _ = orc.attend(stored_bf16(inp["q"][i][heads]), orc.f64(keys), cfg.d_v, scale)
+            assert_close(model.o_csa[i][heads].float().cpu().numpy(), o, ATOL_BF16, REL_BF16, "seq %d csa t=%d" % (b, t))
+            o, _ = orc.hca_query(t, 128, 128, stored_bf16(inp["q_h"][i][heads]), window("x_h", t),
+                                 layer_entries(hca, b, nv_h)["kv"], cfg.d_v, scale)
+            assert_close(model.o_hca[i][heads].float().cpu().numpy(), o, ATOL_BF16, REL_BF16, "seq %d hca t=%d" % (b, t))
+        for L, name in ((csa, "x"), (hca, "x_h")):
+            for p in (c0 + T - 128, c0 + T - 1):
+                assert torch.equal(L.ring_x[b][p % 128], inp[name][r0 + p - c0])
+    # the pass repeats on the same state
+    before = [model.idx.clone(), model.o_csa.clone(), model.o_hca.clone()]
+    model.step()
+    torch.cuda.synchronize()
+    assert model.check_status() == ck.OK
+    for a, b_ in zip(before, [model.idx, model.o_csa, model.o_hca]):
+        assert torch.equal(a, b_)

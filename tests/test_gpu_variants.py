@@ -120,3 +120,87 @@ def test_inverse_rope_latent_kernel(ck, orc):
 def test_inverse_rope_query_pair_kernel(ck, orc):
     """The query-pair kernel writes its bf16 output itself."""
     _many(ck, orc, "hca", 600, 2, 128 * 300, seed=63, rope_dims=64)
+
+
+# ----------------------------------------------------------------- block overlap in the fold
+def _assert_overlap_close(got, ref, x_raw, m, ov, what):
+    """One bf16 step plus the fp32 bound of an (m + ov)-term weighted sum of the stream's values."""
+    from gpu_helpers import bf16_ulp
+    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    tol = bf16_ulp(np.maximum(np.abs(got), np.abs(ref))) + 2.0 * (m + ov) * 2.0 ** -24 * np.abs(x_raw).max()
+    bad = np.abs(got - ref) > tol * 1.0000001
+    assert not bad.any(), "%s: %d beyond tolerance, e.g. got %r ref %r" % (what, int(bad.sum()), got[bad][:3], ref[bad][:3])
+
+
+@pytest.mark.parametrize("kind,m,ov,d", [("csa", 4, 2, 128), ("csa", 4, 4, 576), ("hca", 64, 64, 128)])
+def test_overlap_bulk_segments_and_append(ck, orc, kind, m, ov, d):
+    """The fold with block overlap (10100.com DeepSeek-V4 article, section 2.1) through three routes:
+    one bulk compression of the stream, two bulk segments with the second one's overlap tokens read from
+    the ring, and token-by-token decode appends. m = 64 with 64 overlap tokens takes the block-per-entry
+    bulk fold."""
+    from test_gpu_compress import _stream
+    B, n, n1, d_idx = 2, 768, 384, 64
+    is_csa = kind == "csa"
+    g = torch.Generator().manual_seed(70 + m + ov)
+    bias = (torch.randn(m + ov, d, generator=g) * 2).cuda()
+    bias_i = torch.randn(m + ov, d_idx, generator=g).cuda() if is_csa else None
+    layers = []
+    for _ in range(3):
+        L = make_layer(ck.LAYER_CSA if is_csa else ck.LAYER_HCA, m, d, d, B, n // m + 1,
+                       d_idx=d_idx if is_csa else 0, seed=71)
+        L.overlap = ov
+        L.pos_bias = bias
+        if is_csa:
+            L.pos_bias_idx = bias_i
+        layers.append(L)
+    La, Lb, Lc = layers
+    x, z = _stream(B, n, d, d, seed=72)
+    xi, zi = _stream(B, n, d_idx, d_idx, seed=73)
+    seq = torch.tensor([1, 0], dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def bulk(L, t0, t1):
+        sl = slice(t0, t1)
+        if is_csa:
+            ck.csa_compress_kv(L, seq, t0, x[:, sl].contiguous(), z[:, sl].contiguous(), xi[:, sl].contiguous(),
+                               zi[:, sl].contiguous(), status=status)
+        else:
+            ck.hca_compress_kv(L, seq, t0, x[:, sl].contiguous(), z[:, sl].contiguous(), status=status)
+
+    def append(L, t0, t1, ring_only=False):
+        sl = slice(t0, t1)
+        pos = torch.full((B,), t0, dtype=torch.int64, device="cuda")
+        ck.cskv_cache_append(L, seq, pos, x[:, sl].contiguous(), z[:, sl].contiguous(),
+                             xi[:, sl].contiguous() if is_csa else None, zi[:, sl].contiguous() if is_csa else None,
+                             ring_only=ring_only, status=status)
+
+    bulk(La, 0, n)
+    bulk(Lb, 0, n1)
+    append(Lb, n1 - 128, n1, ring_only=True)  # the state cache before the second segment
+    bulk(Lb, n1, n)
+    for t in range(n):
+        append(Lc, t, t + 1)
+    assert ck.cskv_get_status(status) == ck.OK
+    for b in range(B):
+        s = int(seq[b])
+        ref = orc.compress_overlap(stored_bf16(x[b]), stored_bf16(z[b]), m, ov, bias.cpu().double().numpy())
+        ref = orc.decode(orc.store(ref, orc.BF16))
+        xd = orc.decode(stored_bf16(x[b]))
+        if is_csa:
+            ref_i = orc.compress_overlap(stored_bf16(xi[b]), stored_bf16(zi[b]), m, ov, bias_i.cpu().double().numpy())
+            ref_i = orc.decode(orc.store(ref_i, orc.BF16))
+        for L, what in ((La, "one bulk"), (Lb, "two segments"), (Lc, "appends")):
+            e = layer_entries(L, s, n // m)
+            _assert_overlap_close(orc.decode(e["kv"]), ref, xd, m, ov, "%s kv seq %d" % (what, s))
+            if is_csa:
+                _assert_overlap_close(orc.decode(e["idx"]), ref_i, orc.decode(stored_bf16(xi[b])), m, ov,
+                                      "%s idx seq %d" % (what, s))
+
+
+def test_overlap_bound_is_checked(ck):
+    L = make_layer(ck.LAYER_CSA, 4, 128, 128, 1, 64, d_idx=64)
+    L.overlap = 125  # more than n_win - m: the borrowed tokens would have left the ring
+    x = torch.zeros(1, 4, 128, dtype=torch.bfloat16, device="cuda")
+    xi = torch.zeros(1, 4, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ck.CskvError):
+        ck.csa_compress_kv(L, torch.zeros(1, dtype=torch.int32, device="cuda"), 0, x, x, xi, xi)
