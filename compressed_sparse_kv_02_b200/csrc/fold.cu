@@ -351,6 +351,7 @@ constexpr int kSliceCh = 64;       // channels per CTA of the append kernel (who
 constexpr int kAppendMaxD = 1024;  // channels of the row buffer
 constexpr int kFoldPairs = 32;     // channel pairs of one fold pass (64 channels)
 constexpr int kFoldGroups = kAppendThreads / kFoldPairs;  // 16 token groups
+constexpr int kAppendBatch = 8;  // tokens per thread whose loads are in flight together (m' = 128: all of them)
 
 // Store channels [c_lo, c_hi) of one folded entry from the row buffer `sv`
 // (fp32, indexed by channel) into pool row `row` in the stream's storage type:
@@ -470,39 +471,55 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
       const int c = c0 + 2 * cp;
       const bool active = c < c_hi;
       float mx[2] = {-INFINITY, -INFINITY}, den[2] = {0.f, 0.f}, acc[2] = {0.f, 0.f};
-      for (int i = tg - p.ov; active && i < p.m; i += kFoldGroups) {
-        const int64_t q = j * p.m + i;
-        if (q < 0) continue;  // before the start of the stream
-        const uint16_t* xr;
-        const uint16_t* zr;
-        if (q >= pos) {
-          xr = S.x + ((int64_t)b * p.n_new + (q - pos)) * S.d;
-          zr = S.z + ((int64_t)b * p.n_new + (q - pos)) * S.gc;
-        } else {
-          const int64_t slot = q % p.n_win;
-          xr = S.ring_x + ((int64_t)seq * p.n_win + slot) * S.d;
-          zr = S.ring_z + ((int64_t)seq * p.n_win + slot) * S.gc;
-        }
-        const uint32_t xv = __ldg(reinterpret_cast<const uint32_t*>(xr + c));
-        float zl[2];
-        if (S.gc == 1) {
-          zl[0] = zl[1] = bf16_bits_to_f32(__ldg(zr));
-        } else {
-          const uint32_t zv = __ldg(reinterpret_cast<const uint32_t*>(zr + c));
-          zl[0] = __uint_as_float(zv << 16);
-          zl[1] = __uint_as_float(zv & 0xffff0000u);
-        }
-        const float xf[2] = {__uint_as_float(xv << 16), __uint_as_float(xv & 0xffff0000u)};
+      // kAppendBatch tokens per round: every load of the round is issued before the first
+      // weight is computed, so their latencies overlap instead of adding up
+      for (int i0 = tg - p.ov; active && i0 < p.m; i0 += kAppendBatch * kFoldGroups) {
+        uint32_t xv[kAppendBatch], zv[kAppendBatch];
+        float bv[kAppendBatch][2];
+        bool ok[kAppendBatch];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float bias = S.bias ? S.bias[(int64_t)(i + p.ov) * S.d + c + e] : 0.f;
-          const float l2 = (zl[e] + bias) * kLog2e;  // base-2 weights: 2^(l2 - max) = e^(z - max_z)
-          const float M = fmaxf(mx[e], l2);
-          const float corr = mx[e] == -INFINITY ? 0.f : exp2f(mx[e] - M);
-          const float pw = exp2f(l2 - M);
-          den[e] = den[e] * corr + pw;
-          acc[e] = acc[e] * corr + pw * xf[e];
-          mx[e] = M;
+        for (int u = 0; u < kAppendBatch; ++u) {
+          const int i = i0 + u * kFoldGroups;
+          const int64_t q = j * p.m + i;
+          ok[u] = i < p.m && q >= 0;  // q < 0: before the start of the stream
+          xv[u] = zv[u] = 0u;
+          bv[u][0] = bv[u][1] = 0.f;
+          if (!ok[u]) continue;
+          const uint16_t* xr;
+          const uint16_t* zr;
+          if (q >= pos) {
+            xr = S.x + ((int64_t)b * p.n_new + (q - pos)) * S.d;
+            zr = S.z + ((int64_t)b * p.n_new + (q - pos)) * S.gc;
+          } else {
+            const int64_t slot = q % p.n_win;
+            xr = S.ring_x + ((int64_t)seq * p.n_win + slot) * S.d;
+            zr = S.ring_z + ((int64_t)seq * p.n_win + slot) * S.gc;
+          }
+          xv[u] = __ldg(reinterpret_cast<const uint32_t*>(xr + c));
+          zv[u] = S.gc == 1 ? static_cast<uint32_t>(__ldg(zr)) << 16 : __ldg(reinterpret_cast<const uint32_t*>(zr + c));
+          if (S.bias) {
+            const float* br = S.bias + (int64_t)(i + p.ov) * S.d + c;
+            bv[u][0] = __ldg(br);
+            bv[u][1] = __ldg(br + 1);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kAppendBatch; ++u) {
+          if (!ok[u]) continue;
+          // a per-token gate (gc == 1) sits in the high half for both channels
+          const float zl[2] = {S.gc == 1 ? __uint_as_float(zv[u] & 0xffff0000u) : __uint_as_float(zv[u] << 16),
+                               __uint_as_float(zv[u] & 0xffff0000u)};
+          const float xf[2] = {__uint_as_float(xv[u] << 16), __uint_as_float(xv[u] & 0xffff0000u)};
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float l2 = (zl[e] + bv[u][e]) * kLog2e;  // base-2 weights: 2^(l2 - max) = e^(z - max_z)
+            const float M = fmaxf(mx[e], l2);
+            const float corr = mx[e] == -INFINITY ? 0.f : exp2f(mx[e] - M);
+            const float pw = exp2f(l2 - M);
+            den[e] = den[e] * corr + pw;
+            acc[e] = acc[e] * corr + pw * xf[e];
+            mx[e] = M;
+          }
         }
       }
       if (active) {

@@ -381,8 +381,10 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
       if (query_visible(p, b) < 0) report(p.status, CSKV_ERR_INVALID_ARG);
 
   const int64_t total = s_pref[p.n_q];
-  const int64_t u_begin = total * blockIdx.x / gridDim.x;
-  const int64_t n_units = total * (blockIdx.x + 1) / gridDim.x - u_begin;
+  // the units split over min(grid, total) CTAs, so that every CTA with work has at least one unit
+  const int64_t n_work = total < gridDim.x ? total : gridDim.x;
+  const int64_t u_begin = blockIdx.x < n_work ? total * blockIdx.x / n_work : total;
+  const int64_t n_units = blockIdx.x < n_work ? total * (blockIdx.x + 1) / n_work - u_begin : 0;
   auto locate = [&](int64_t u, int& b, int64_t& j0) {
     int lo = 0, hi = p.n_q - 1;  // last b with s_pref[b] <= u
     while (lo < hi) {

@@ -10,7 +10,8 @@
   with the oracle run on sampled queries and heads.
 * mixed: the quantised, mixed-length workload (FP8 KV with a scale per entry,
   FP4 indexer keys and queries, per-sequence lengths, layers CSA, HCA, CSA,
-  HCA) at a reduced batch and length, every query and both layer pairs.
+  HCA) at a reduced batch and length (every query), and at the benchmark's
+  full size (B = 64, lengths up to ~1M; sampled sequences), both layer pairs.
 """
 import math
 
@@ -174,24 +175,16 @@ def test_pro_fullsize_sampled(ck, orc):
     _fullsize(ck, orc, "pro", sample_b=[0, 7], sample_heads=[0, 1, 63, 64, 127])
 
 
-def test_mixed_fp8_fp4_two_pairs(ck, orc):
-    from compressed_sparse_kv_02_b200 import decode, synth
-    cfg = synth.Config("mixed_small", 4, 1 << 16, 128, 576, 512, 8, 128, 1024, seed=4, kv_dtype="fp8",
-                       idx_dtype="fp4")
-    lens = synth.mixed_lengths(cfg, lo=4096, hi=1 << 16)
-    lens[0] = 4096  # a sequence whose last token completes an HCA block (the append emits an entry)
-    model = decode.DecodeModel(cfg, ctx_lens=lens, n_pairs=2)
-    model.fill_synthetic()
-    model.step()
-    torch.cuda.synchronize()
-    assert model.check_status() == ck.OK
+def _mixed_checks(orc, model, cfg, lens, sample, heads):
+    """Selections (tie band, oracle scores on the stored FP4 keys) and both attentions (FP8 keys,
+    5e-2) of the sampled sequences, in both layer pairs."""
     scale = 1.0 / math.sqrt(cfg.d_qk)
-    heads = np.array([0, 5, 64, 127])
+    heads = np.array(heads)
     for li in range(2):
         csa, hca = model.layers[2 * li], model.layers[2 * li + 1]
         out, inp = model.out[li], model.inputs[li]
-        for b, n_b in enumerate(lens):
-            t = n_b - 1
+        for b in sample:
+            t = int(lens[b]) - 1
             nv = orc.visible_entries(t, 4, 128)
             nv_h = orc.visible_entries(t, 128, 128)
             ent = layer_entries(csa, b, nv)
@@ -209,3 +202,35 @@ def test_mixed_fp8_fp4_two_pairs(ck, orc):
                                  cfg.d_v, scale)
             assert_close(out["o_hca"][b][heads].float().cpu().numpy(), o, ATOL_LP, REL_LP,
                          "hca pair %d b=%d" % (li, b))
+
+
+def test_mixed_fp8_fp4_two_pairs(ck, orc):
+    from compressed_sparse_kv_02_b200 import decode, synth
+    cfg = synth.Config("mixed_small", 4, 1 << 16, 128, 576, 512, 8, 128, 1024, seed=4, kv_dtype="fp8",
+                       idx_dtype="fp4")
+    lens = synth.mixed_lengths(cfg, lo=4096, hi=1 << 16)
+    lens[0] = 4096  # a sequence whose last token completes an HCA block (the append emits an entry)
+    model = decode.DecodeModel(cfg, ctx_lens=lens, n_pairs=2)
+    model.fill_synthetic()
+    model.step()
+    torch.cuda.synchronize()
+    assert model.check_status() == ck.OK
+    _mixed_checks(orc, model, cfg, lens, range(len(lens)), [0, 5, 64, 127])
+
+
+def test_mixed_fullsize_sampled(ck, orc):
+    """The mixed workload at the benchmark's own size and launch configuration: B = 64 sequences with
+    log-uniform lengths up to ~1M (FP8 KV, FP4 indexer, layers CSA, HCA, CSA, HCA); the shortest and the
+    longest sequence and four others drawn at random, in both layer pairs."""
+    from compressed_sparse_kv_02_b200 import decode, synth
+    cfg = synth.CONFIGS["mixed"]
+    lens = synth.mixed_lengths(cfg)
+    model = decode.DecodeModel(cfg, ctx_lens=lens, n_pairs=2)
+    model.fill_synthetic()
+    model.step()
+    torch.cuda.synchronize()
+    assert model.check_status() == ck.OK
+    order = np.argsort(np.asarray(lens))
+    rng = np.random.default_rng(5)
+    others = rng.choice(order[1:-1], size=4, replace=False).tolist()
+    _mixed_checks(orc, model, cfg, lens, [int(order[0]), int(order[-1])] + others, [0, 37, 64, 127])

@@ -103,6 +103,54 @@ def test_ties_prefer_lower_index(ck, orc):
     assert out_idx.cpu().numpy()[0].tolist() == list(range(k))
 
 
+def test_heavy_ties_across_ctas(ck, orc):
+    # Threshold bins far larger than the selection's candidate list, split over many scanning
+    # CTAs: query 0's keys are three distinct rows (every score is one of three values; the
+    # top row 300 times, the second 25000 times, so 724 ties are taken at the second value),
+    # query 1's keys are all equal, and query 2 is plain random in the same call. Ties go to
+    # the lowest indices, so the expected selections are exact.
+    k = 1024
+    positions = [127 + 4 * 40000, 127 + 4 * 30000 + 1, 127 + 4 * 9000 + 2]
+    hi, di = 8, 128
+    B = len(positions)
+    n_e = max(positions) // 4 + 2
+    L = make_layer(ck.LAYER_CSA, 4, 128, 128, B, n_e, d_idx=di, seed=21)
+    g = torch.Generator().manual_seed(121)
+    q_idx = torch.randn(B, hi, di, generator=g).to(torch.bfloat16)
+    w = torch.rand(B, hi, generator=g)
+    rows = torch.randn(3, di, generator=g).to(torch.bfloat16)
+    qd, wd = q_idx[0].double(), w[0].double()
+    s3 = [(wd * torch.relu(qd @ rows[r].double())).sum().item() for r in range(3)]
+    order = sorted(range(3), key=lambda r: -s3[r])
+    assign = torch.full((n_e,), order[2], dtype=torch.long)
+    perm = torch.randperm(n_e, generator=g)
+    assign[perm[:25000]] = order[1]
+    assign[perm[25000:25300]] = order[0]
+    keys = [rows[assign], rows[0].expand(n_e, di).clone(), torch.randn(n_e, di, generator=g).to(torch.bfloat16)]
+    for b in range(B):
+        L.write_entries(b, 0, idx=keys[b].cuda())
+    q_idx, w = q_idx.cuda(), w.cuda()
+    seq = torch.arange(B, dtype=torch.int32, device="cuda")
+    pos = torch.tensor(positions, dtype=torch.int64, device="cuda")
+    out_idx = torch.full((B, k), -7, dtype=torch.int32, device="cuda")
+    out_cnt = torch.full((B,), -7, dtype=torch.int32, device="cuda")
+    out_sc = torch.zeros(B, k, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ck.csa_index_score_topk(L, seq, pos, max(positions), q_idx, w, k, out_idx, out_cnt, out_sc, status=status)
+    assert ck.cskv_get_status(status) == ck.OK
+    idx, cnt = out_idx.cpu().numpy(), out_cnt.cpu().numpy()
+    for b, t in enumerate(positions):
+        s = _oracle_scores(orc, L, b, t, q_idx, None, w, False)
+        assert int(cnt[b]) == k
+        if b < 2:
+            # distinct score values are far apart, equal ones identical: the top-k by (score desc,
+            # index asc), listed in ascending index order
+            want = np.sort(np.lexsort((np.arange(len(s)), -s))[:k])
+            assert idx[b].tolist() == want.tolist()
+        else:
+            check_topk(idx[b], k, s, k)
+
+
 def test_fp4_indexer(ck, orc):
     k = 128
     positions = [127 + 4 * 2000 + 1, 127 + 4 * 100, 127 + 4 * 5000]

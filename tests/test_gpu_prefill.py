@@ -1,8 +1,9 @@
-"""GPU parity of one prefill pass (PrefillModel) at reduced size.
+"""GPU parity of one prefill pass (PrefillModel), at reduced size and at the
+benchmark's full size.
 
 A sequence with 8192 cached tokens receives a chunk of 2048 new tokens
 (H = 64, d = 128, indexer 4 x 64, top-512), in two blocks of 1024 query
-positions. Checked against the oracle: the chunk's compressed entries (from
+positions; at full size 65536 new tokens on 65536 cached, in blocks of 4096. Checked against the oracle: the chunk's compressed entries (from
 the chunk's raw rows), the top-k and both attentions of sampled positions
 (window rows from the chunk or, before the chunk, from the restored ring),
 the rings after the pass, and that a second pass gives identical outputs.
@@ -27,18 +28,13 @@ def ck(cskv_built):
     return ck
 
 
-def test_prefill_chunk(ck, orc):
-    from compressed_sparse_kv_02_b200 import prefill, synth
-    cfg = synth.Config("prefill_small", 1, 8192 + 2048, 64, 128, 128, 4, 64, 512, seed=3)
-    c0, T = 8192, 2048
-    model = prefill.PrefillModel(cfg, cached=c0, chunk=T, q_block=1024)
-    model.fill_synthetic()
-    model.step()
-    torch.cuda.synchronize()
-    assert model.check_status() == ck.OK
+def _check_prefill(ck, orc, model, positions, heads_of):
+    """The chunk's compressed entries (from its raw rows), the top-k and both attentions at the given
+    positions (heads_of(t) -> head indices; window rows from the chunk or, before it, from the
+    restored ring), the rings after the pass, and that a second pass gives identical outputs."""
+    cfg, c0, T = model.cfg, model.cached, model.chunk
     csa, hca = model.layers
     inp = model.inputs
-    # the chunk's entries, from its raw rows
     for L, xs, zs, m in ((csa, "x", "z", 4), (hca, "x_h", "z_h", 128)):
         got = L.read_entries(0, T // m, c0 // m)
         x, z = inp[xs][0].cpu(), inp[zs][0].cpu()
@@ -60,21 +56,22 @@ def test_prefill_chunk(ck, orc):
         return stored_bf16(torch.stack(rows))
 
     scale = 1.0 / math.sqrt(cfg.d_qk)
-    heads = np.array([0, 17, 63])
-    for t in (c0, c0 + 1, c0 + 127, c0 + 128, c0 + 1023, c0 + 1024, c0 + T - 1):
+    ent_all = layer_entries(csa, 0, orc.visible_entries(c0 + T - 1, 4, 128))
+    hent_all = layer_entries(hca, 0, orc.visible_entries(c0 + T - 1, 128, 128))["kv"]
+    for t in positions:
         i = t - c0
+        heads = np.asarray(heads_of(t))
         nv = orc.visible_entries(t, 4, 128)
         nv_h = orc.visible_entries(t, 128, 128)
-        ent = layer_entries(csa, 0, nv)
-        sc = orc.index_scores(stored_bf16(inp["q_idx"][i]), inp["w"][i].double().cpu().numpy(), ent["idx"], nv)
+        sc = orc.index_scores(stored_bf16(inp["q_idx"][i]), inp["w"][i].double().cpu().numpy(), ent_all["idx"], nv)
         idx = model.idx[i].cpu().numpy()
         cnt = int(model.cnt[i])
         check_topk(idx, cnt, sc, cfg.k)
-        keys = np.vstack([orc.decode(window("x", t)), orc.decode(ent["kv"].take_rows(idx[:cnt]))])
+        keys = np.vstack([orc.decode(window("x", t)), orc.decode(ent_all["kv"].take_rows(idx[:cnt]))])
         o, _ = orc.attend(stored_bf16(inp["q"][i][heads]), orc.f64(keys), cfg.d_v, scale)
         assert_close(model.o_csa[i][heads].float().cpu().numpy(), o, ATOL_BF16, REL_BF16, "csa t=%d" % t)
         o, _ = orc.hca_query(t, 128, 128, stored_bf16(inp["q_h"][i][heads]), window("x_h", t),
-                             layer_entries(hca, 0, nv_h)["kv"], cfg.d_v, scale)
+                             hent_all.take_rows(np.arange(nv_h)), cfg.d_v, scale)
         assert_close(model.o_hca[i][heads].float().cpu().numpy(), o, ATOL_BF16, REL_BF16, "hca t=%d" % t)
     # the rings end with the chunk's last 128 rows (slot p % 128)
     for L, name in ((csa, "x"), (hca, "x_h")):
@@ -87,6 +84,40 @@ def test_prefill_chunk(ck, orc):
     assert model.check_status() == ck.OK
     for a, b in zip(before, [model.idx, model.o_csa, model.o_hca]):
         assert torch.equal(a, b)
+
+
+def test_prefill_chunk(ck, orc):
+    from compressed_sparse_kv_02_b200 import prefill, synth
+    cfg = synth.Config("prefill_small", 1, 8192 + 2048, 64, 128, 128, 4, 64, 512, seed=3)
+    c0, T = 8192, 2048
+    model = prefill.PrefillModel(cfg, cached=c0, chunk=T, q_block=1024)
+    model.fill_synthetic()
+    model.step()
+    torch.cuda.synchronize()
+    assert model.check_status() == ck.OK
+    _check_prefill(ck, orc, model, (c0, c0 + 1, c0 + 127, c0 + 128, c0 + 1023, c0 + 1024, c0 + T - 1),
+                   lambda t: [0, 17, 63])
+
+
+def test_prefill_fullsize_sampled(ck, orc):
+    """The prefill pass at the benchmark's own size and launch configuration: 65536 new tokens on 65536
+    cached, query blocks of 4096. Positions at block edges, the chunk's first and last positions and
+    twenty drawn at random; every head at five of them, three heads elsewhere."""
+    from compressed_sparse_kv_02_b200 import prefill, synth
+    cfg = synth.CONFIGS["prefill"]
+    c0, T = 65536, 65536
+    model = prefill.PrefillModel(cfg, cached=c0, chunk=T, q_block=4096)
+    model.fill_synthetic()
+    model.step()
+    torch.cuda.synchronize()
+    assert model.check_status() == ck.OK
+    edges = [c0 + 4096 * j + d for j in (1, 8, 15) for d in (-1, 0)]
+    rng = np.random.default_rng(11)
+    rand = sorted(int(x) for x in rng.integers(c0, c0 + T, size=20))
+    positions = [c0, c0 + 1, c0 + 127, c0 + 128] + edges + rand + [c0 + T - 1]
+    all_heads = {c0, c0 + 128, c0 + 4096, c0 + 8 * 4096 - 1, c0 + T - 1}
+    _check_prefill(ck, orc, model, positions,
+                   lambda t: list(range(cfg.heads)) if t in all_heads else [0, 17, 63])
 
 
 def test_varlen_prefill_several_sequences(ck, orc):
