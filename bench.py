@@ -21,7 +21,9 @@ events captured around it inside the graph. The default run then adds, under
 `secondary`, the metric's other figures from the same GPU: the prefill pass
 (65,536 new tokens on 65,536 cached; tokens/s against the sustained bf16
 tensor peak) and the mixed-length paged FP8 / FP4 decode (queries/s against
-HBM), each with its own roofline, e2e and clock record.
+HBM), each with its own roofline, e2e and clock record. `bf16_scores` reports,
+outside the timed region, the recall of the indexer's selection on bf16-rounded
+scores against its fp32 selection on the same inputs, and both op times.
 """
 from __future__ import annotations
 
@@ -37,6 +39,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 METRIC = "CSA/HCA decode queries/s at 1M ctx; HBM GB/s vs peak; prefill tok/s"
@@ -604,9 +607,48 @@ def run_ours(args, rank, world):
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": kernels_per_step * steps_timed,
     }
+    if rank == 0:
+        out["bf16_scores"] = bf16_score_report(model, cfg, stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(model, cfg, budget_s=args.cpu_budget)
     return out
+
+
+def bf16_score_report(model, cfg, stream, reps: int = 20) -> dict:
+    """The indexer's selection mode on bf16-rounded scores (DeepSeek-V4 report digest, section 7: index
+    scores in BF16) against the fp32 selection, on the first CSA layer of the step's own inputs (after the
+    timed region): the recall |S_bf16 & S_fp32| / |S_fp32| averaged over the queries, and the op time of
+    each mode (CUDA events on the launching stream, mean of `reps` calls)."""
+    import compressed_sparse_kv_02_b200 as ck
+    layer, inp = model.layers[0], model.inputs[0]
+    nq, k = cfg.batch, cfg.k
+    res = {}
+    for bf16 in (False, True):
+        idx = torch.empty(nq, k, dtype=torch.int32, device="cuda")
+        cnt = torch.empty(nq, dtype=torch.int32, device="cuda")
+        ws = torch.empty(ck.csa_index_ws_bytes(layer, nq, cfg.heads_idx, model.max_pos, k), dtype=torch.uint8,
+                         device="cuda")
+
+        def call():
+            ck.csa_index_score_topk(layer, model.seq, model.pos, model.max_pos, inp["q_idx"], inp["w"], k, idx, cnt,
+                                    q_idx_scale=inp.get("q_idx_scale"), workspace=ws, status=model.status,
+                                    stream=stream, score_bf16=bf16)
+        with torch.cuda.stream(stream):
+            call()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                call()
+            e1.record(stream)
+        stream.synchronize()
+        res[bf16] = (idx.cpu().numpy(), cnt.cpu().numpy(), e0.elapsed_time(e1) / reps)
+    (i32, c32, t32), (i16, c16, t16) = res[False], res[True]
+    rec = [len(set(i16[b, :c16[b]].tolist()) & set(i32[b, :c32[b]].tolist())) / max(1, int(c32[b]))
+           for b in range(nq)]
+    return {"recall_vs_fp32": round(float(np.mean(rec)), 5), "recall_min": round(float(np.min(rec)), 5),
+            "index_op_ms_fp32": round(t32, 5), "index_op_ms_bf16": round(t16, 5),
+            "note": "scores rounded to bf16 (RNE) before the selection; the scan reads the same keys, so the op "
+                    "time does not change"}
 
 
 # ----------------------------------------------------------------- the oracle on host cores
