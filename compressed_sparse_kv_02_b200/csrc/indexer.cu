@@ -899,12 +899,20 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
   __shared__ int s_peer[3 * kMaxCluster];
   constexpr int NW = kSelThreads / 32;
   __shared__ int s_wgt[NW], s_weq[NW];
+  // per warp: the slice positions of its keys at or above the threshold digit, in index order
+  // (built by the conversion pass when digit A is known first); the ordered output walks these
+  // short lists instead of the whole slice unless one of them overflowed
+  constexpr int kListCapW = 128;
+  __shared__ uint16_t s_list[NW][kListCapW];
+  __shared__ int s_wlen[NW];
+  __shared__ int s_over;
 
   for (int i = tid; i < kBinsA; i += kSelThreads) s_hA[i] = 0u;
   for (int i = tid; i < kBinsB; i += kSelThreads) s_hB[i] = 0u;
   for (int i = tid; i < kBinsC; i += kSelThreads) s_hC[i] = 0u;
   if (tid == 0) {
     s_ncand = 0;
+    s_over = 0;
     s_res[0] = s_res[1] = s_res[2] = 0u;
     mbar_init(&s_bar, 1);
     fence_barrier_init();
@@ -968,28 +976,95 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
       n4 = 0;
       len = 0;
     }
-    uint4* k4 = reinterpret_cast<uint4*>(s_keys);
-    for (int base = 0; base < n4; base += kSelThreads) {
-      const int i = base + tid;
-      uint4 kv = make_uint4(0u, 0u, 0u, 0u);
-      if (i < n4) {
-        const uint4 fv = k4[i];
-        kv = make_uint4(f2key(__uint_as_float(fv.x)), f2key(__uint_as_float(fv.y)), f2key(__uint_as_float(fv.z)),
-                        f2key(__uint_as_float(fv.w)));
-        k4[i] = kv;
+    if (gather_now) {
+      // Warp w scans its contiguous part [w*seg, (w+1)*seg) of the slice (seg a multiple of 128,
+      // four consecutive scores per lane per step) and keeps the positions of its keys at or above
+      // digit dA in order; the slice keeps the raw scores (keys are formed where they are read),
+      // the 0..3 scores past the bulk copy are copied in from global memory. The candidates of
+      // digit dA are then gathered from the lists.
+      const int seg = ((len + NW - 1) / NW + 127) / 128 * 128;
+      const int s_lo = wid * seg, s_hi = min(len, s_lo + seg);
+      int nl = 0;
+      for (int base = s_lo; base < s_hi; base += 128) {
+        const int i = base + 4 * lane;
+        uint32_t kk[4];
+        unsigned valid = 0u;
+        if (i + 3 < s_hi && i + 3 < 4 * n4) {
+          const uint4 fv = reinterpret_cast<const uint4*>(s_keys)[i >> 2];
+          kk[0] = f2key(__uint_as_float(fv.x));
+          kk[1] = f2key(__uint_as_float(fv.y));
+          kk[2] = f2key(__uint_as_float(fv.z));
+          kk[3] = f2key(__uint_as_float(fv.w));
+          valid = 15u;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = i + e;
+            kk[e] = 0u;
+            if (j < s_hi) {
+              const float f = j < 4 * n4 ? __uint_as_float(s_keys[j]) : sc[lo + j];
+              if (j >= 4 * n4) s_keys[j] = __float_as_uint(f);
+              kk[e] = f2key(f);
+              valid |= 1u << e;
+            }
+          }
+        }
+        int nq = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) nq += ((valid >> e) & 1u) && (kk[e] >> 21) >= dA ? 1 : 0;
+        if (__any_sync(kFull, nq > 0)) {
+          const int off = warp_exclusive_scan(nq, lane);
+          int at = nl + off;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (((valid >> e) & 1u) && (kk[e] >> 21) >= dA) {
+              if (at < kListCapW) s_list[wid][at] = static_cast<uint16_t>(i + e);
+              ++at;
+            }
+          }
+          nl += __shfl_sync(kFull, off + nq, 31);
+        }
       }
-      if (gather_now) {
-        gather(kv.x, i < n4 && (kv.x & maskA) == pre);
-        gather(kv.y, i < n4 && (kv.y & maskA) == pre);
-        gather(kv.z, i < n4 && (kv.z & maskA) == pre);
-        gather(kv.w, i < n4 && (kv.w & maskA) == pre);
+      if (lane == 0) {
+        s_wlen[wid] = nl;
+        if (nl > kListCapW) s_over = 1;
       }
-    }
-    for (int base = n4 << 2; base < len; base += kSelThreads) {  // the last 0..3 keys
-      const int i = base + tid;
-      const uint32_t key = i < len ? f2key(sc[lo + i]) : 0u;
-      if (i < len) s_keys[i] = key;
-      if (gather_now) gather(key, i < len && (key & maskA) == pre);
+      __syncthreads();
+      if (s_over == 0) {
+        for (int e0 = 0; e0 < nl; e0 += 32) {
+          const int e = e0 + lane;
+          const uint32_t key = e < nl ? f2key(__uint_as_float(s_keys[s_list[wid][e]])) : 0u;
+          gather(key, e < nl && (key & maskA) == pre);
+        }
+      }
+      __syncthreads();
+      // a list overflowed (a threshold bin of heavy ties): the slice is converted in place and
+      // gathered whole, and the passes below run over the slice
+      if (s_over) {
+        for (int j = tid; j < len; j += kSelThreads) {
+          const uint32_t key = f2key(__uint_as_float(s_keys[j]));
+          s_keys[j] = key;
+        }
+        for (int base = 0; base < len; base += kSelThreads) {
+          const int j = base + tid;
+          const uint32_t key = j < len ? s_keys[j] : 0u;
+          gather(key, j < len && (key & maskA) == pre);
+        }
+      }
+    } else {
+      uint4* k4 = reinterpret_cast<uint4*>(s_keys);
+      for (int base = 0; base < n4; base += kSelThreads) {
+        const int i = base + tid;
+        if (i < n4) {
+          const uint4 fv = k4[i];
+          k4[i] = make_uint4(f2key(__uint_as_float(fv.x)), f2key(__uint_as_float(fv.y)), f2key(__uint_as_float(fv.z)),
+                             f2key(__uint_as_float(fv.w)));
+        }
+      }
+      for (int base = n4 << 2; base < len; base += kSelThreads) {  // the last 0..3 keys
+        const int i = base + tid;
+        if (i < len) s_keys[i] = f2key(sc[lo + i]);
+      }
     }
   }
   __syncthreads();
@@ -1019,14 +1094,16 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
     // every CTA copies the cluster's candidates (nA keys in all) and finishes the select alone
     cluster.sync();
     __shared__ int s_pn[kMaxCluster + 1], s_pq[kMaxCluster + 1];  // prefix of keys / 16-byte pieces per peer
+    __shared__ int s_nr[kMaxCluster];
+    if (tid < CL) s_nr[tid] = min(*cluster.map_shared_rank(&s_ncand, tid), kCandCap);  // the peers' counts at once
+    __syncthreads();
     if (tid == 0) {
       int nk = 0, nq = 0;
       for (int r = 0; r < CL; ++r) {
         s_pn[r] = nk;
         s_pq[r] = nq;
-        const int n_r = min(*cluster.map_shared_rank(&s_ncand, r), kCandCap);
-        nk += n_r;
-        nq += (n_r + 3) >> 2;
+        nk += s_nr[r];
+        nq += (s_nr[r] + 3) >> 2;
       }
       s_pn[CL] = nk;
       s_pq[CL] = nq;
@@ -1100,15 +1177,26 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
       }
     }
   };
+  // every key >= T has a digit >= dA, so a complete list holds all of them
+  const bool listed = p.hist && nA <= kCandCap && s_over == 0;  // uniform across the CTA
+  const int nl = listed ? s_wlen[wid] : 0;
   int gt = 0, eq = 0;
-  for (int base = s_lo; base < s_hi; base += 128) {
-    uint32_t kk[4];
-    unsigned valid;
-    keys4(base + 4 * lane, kk, valid);
+  if (listed) {
+    for (int e = lane; e < nl; e += 32) {
+      const uint32_t key = f2key(__uint_as_float(s_keys[s_list[wid][e]]));  // raw scores on this path
+      gt += key > T;
+      eq += key == T;
+    }
+  } else {
+    for (int base = s_lo; base < s_hi; base += 128) {
+      uint32_t kk[4];
+      unsigned valid;
+      keys4(base + 4 * lane, kk, valid);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      gt += ((valid >> e) & 1u) && kk[e] > T;
-      eq += ((valid >> e) & 1u) && kk[e] == T;
+      for (int e = 0; e < 4; ++e) {
+        gt += ((valid >> e) & 1u) && kk[e] > T;
+        eq += ((valid >> e) & 1u) && kk[e] == T;
+      }
     }
   }
   gt = __reduce_add_sync(kFull, gt);
@@ -1165,7 +1253,25 @@ __global__ void __launch_bounds__(kSelThreads, 1) index_select_kernel(IndexParam
     w_eq_before += s_weq[w];
   }
   int run_eq = w_eq_before, run_sel = w_sel_before;
-  for (int base = s_lo; base < s_hi; base += 128) {
+  if (listed) {
+    for (int e0 = 0; e0 < nl; e0 += 32) {  // one list entry per lane, lanes in index order
+      const int e = e0 + lane;
+      const int pos = e < nl ? s_list[wid][e] : 0;
+      const uint32_t key = e < nl ? f2key(__uint_as_float(s_keys[pos])) : 0u;
+      const bool is_eq = e < nl && key == T;
+      const unsigned meq = __ballot_sync(kFull, is_eq);
+      const bool sel = (e < nl && key > T) || (is_eq && run_eq + __popc(meq & below) < take_eq);
+      const unsigned msel = __ballot_sync(kFull, sel);
+      const int at = run_sel + __popc(msel & below);
+      if (sel && at < k) {
+        oidx[at] = static_cast<int32_t>(lo + pos);
+        if (osc) osc[at] = key2f(key);
+      }
+      run_eq += __popc(meq);
+      run_sel += __popc(msel);
+    }
+  }
+  for (int base = s_lo; base < s_hi && !listed; base += 128) {
     const int i = base + 4 * lane;
     uint32_t kk[4];
     unsigned valid;
