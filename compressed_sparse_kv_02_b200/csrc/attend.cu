@@ -391,6 +391,8 @@ __global__ void __launch_bounds__(256) attend_merge_kernel(AttendParams p) {
 // The same merge over head-minor partial outputs ([query x split][d_v / 4][heads][4],
 // written by attend_tc_kernel): a CTA takes 128 consecutive heads x 2 groups of 4
 // channels, so every partial-output load is a warp's 512 contiguous bytes.
+constexpr int kMergeRegSplits = 12;  // splits merged from registers in one batch of loads
+
 __global__ void __launch_bounds__(256) attend_merge_t_kernel(AttendParams p) {
   grid_dependency_wait();  // the partial outputs come from the attention kernel ahead of this one
   grid_dependents_launch();
@@ -401,32 +403,60 @@ __global__ void __launch_bounds__(256) attend_merge_t_kernel(AttendParams p) {
   const int g4 = blockIdx.y * 2 + (threadIdx.x >> 7);  // group of 4 output channels
   if (h >= p.n_heads || g4 >= p.d_v / 4) return;
   const int64_t lbase = (int64_t)b * p.max_splits * p.n_heads + h;
-  float L = -INFINITY;
-  for (int s = 0; s < ns; ++s) L = fmaxf(L, p.part_lse[lbase + (int64_t)s * p.n_heads]);
+  const float4* po = reinterpret_cast<const float4*>(p.part_o);
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   float wsum = 0.f;
-  if (L != -INFINITY) {
-    const float4* po = reinterpret_cast<const float4*>(p.part_o);
-    for (int s0 = 0; s0 < ns; s0 += 8) {
-      float wg[8];
-      float4 o[8];
+  float L = -INFINITY;
+  if (ns <= kMergeRegSplits) {
+    // every split's log-sum-exp and partial output are loaded in one batch
+    float ls[kMergeRegSplits];
+    float4 o[kMergeRegSplits];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int s = s0 + j;
-        wg[j] = 0.f;
-        o[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (s < ns) {
-          wg[j] = expf(p.part_lse[lbase + (int64_t)s * p.n_heads] - L);
-          o[j] = po[(((int64_t)b * p.max_splits + s) * (p.d_v / 4) + g4) * p.n_heads + h];
-        }
+    for (int s = 0; s < kMergeRegSplits; ++s) {
+      ls[s] = -INFINITY;
+      o[s] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (s < ns) {
+        ls[s] = p.part_lse[lbase + (int64_t)s * p.n_heads];
+        o[s] = po[(((int64_t)b * p.max_splits + s) * (p.d_v / 4) + g4) * p.n_heads + h];
       }
+    }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        wsum += wg[j];
-        acc[0] += wg[j] * o[j].x;
-        acc[1] += wg[j] * o[j].y;
-        acc[2] += wg[j] * o[j].z;
-        acc[3] += wg[j] * o[j].w;
+    for (int s = 0; s < kMergeRegSplits; ++s) L = fmaxf(L, ls[s]);
+    if (L != -INFINITY) {
+#pragma unroll
+      for (int s = 0; s < kMergeRegSplits; ++s) {
+        const float wg = s < ns ? expf(ls[s] - L) : 0.f;
+        wsum += wg;
+        acc[0] += wg * o[s].x;
+        acc[1] += wg * o[s].y;
+        acc[2] += wg * o[s].z;
+        acc[3] += wg * o[s].w;
+      }
+    }
+  } else {
+    for (int s = 0; s < ns; ++s) L = fmaxf(L, p.part_lse[lbase + (int64_t)s * p.n_heads]);
+    if (L != -INFINITY) {
+      for (int s0 = 0; s0 < ns; s0 += 8) {
+        float wg[8];
+        float4 o[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int s = s0 + j;
+          wg[j] = 0.f;
+          o[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (s < ns) {
+            wg[j] = expf(p.part_lse[lbase + (int64_t)s * p.n_heads] - L);
+            o[j] = po[(((int64_t)b * p.max_splits + s) * (p.d_v / 4) + g4) * p.n_heads + h];
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          wsum += wg[j];
+          acc[0] += wg[j] * o[j].x;
+          acc[1] += wg[j] * o[j].y;
+          acc[2] += wg[j] * o[j].z;
+          acc[3] += wg[j] * o[j].w;
+        }
       }
     }
   }

@@ -197,7 +197,8 @@ __device__ __forceinline__ void issue_s(uint32_t d, uint32_t q, uint32_t k, uint
 template <bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ring,
-                     const __grid_constant__ CUtensorMap tm_kv, AttendParams p) {
+                     const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_kvg,
+                     AttendParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = sm + Smem::Q;
@@ -218,6 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + Smem::TMEM);
   volatile int* sAbort = reinterpret_cast<int*>(sm + Smem::FLAGS);
   volatile int* sLdOk = reinterpret_cast<int*>(sm + Smem::FLAGS) + 1;
+  volatile int* sPool = reinterpret_cast<int*>(sm + Smem::FLAGS) + 2;  // [2] per code warp: the tile is gatherable
   int* sPref = reinterpret_cast<int*>(sm + Smem::PREF);
   __shared__ int s_wsum[32];
 
@@ -242,6 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_ring);
     prefetch_tensormap(&tm_kv);
+    if (!FP8) prefetch_tensormap(&tm_kvg);
   }
   if (warp == 4) {
     tmem_alloc(sTmem, kTmemCols);
@@ -376,7 +379,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (lw < 2) {
           const unsigned bits = __ballot_sync(kFull, code != 0u);
-          if (ll == 0) sMask[st * 2 + lw] = bits;
+          // a bf16 tile whose rows are all pool rows (or none) is gathered by TMA
+          const bool pool = __all_sync(kFull, code == 0u || (code >> kRowBits) == 1u);
+          if (ll == 0) {
+            sMask[st * 2 + lw] = bits;
+            sPool[lw] = pool ? 1 : 0;
+          }
         }
         named_sync(3, kLoaders);
         uint8_t* dst = sK + st * kStageBytes;
@@ -387,6 +395,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(&kfull[st], kStageBytes);
             const CUtensorMap* map = mode == 0 ? &tm_ring : &tm_kv;
             for (int j = 0; j < kNb; ++j) tma_load_2d(dst + j * kBlkBytes, map, j * 64, row0, &kfull[st]);
+          }
+          if (it + 1 < ntiles) {
+            ncode = code_of(it + 1, nsc);
+            int rr0;
+            if (tile_src(it + 1, rr0) < 0) prefetch(ncode);
+          }
+        } else if (!fp8 && sPool[0] && sPool[1]) {
+          // the tile's rows by TMA gather, four rows of one 64-channel block per copy; a key without
+          // a row reads row -1, outside the map: zeros, as the copies below would write
+          if (lt == 0) mbar_arrive_expect_tx(&kfull[st], kStageBytes);
+          named_sync(3, kLoaders);  // the stage's byte count is set before any of its copies lands
+          for (int q = lt; q < kNb * (kNk / 4); q += kLoaders) {
+            const int j = q / (kNk / 4), r4 = (q % (kNk / 4)) * 4;
+            int y[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t cd = sCode[st * kNk + r4 + e];
+              y[e] = (cd >> kRowBits) == 1u ? static_cast<int>(cd & kRowMask) : -1;
+            }
+            tma_gather4(dst + j * kBlkBytes + r4 * 128, &tm_kvg, j * 64, y[0], y[1], y[2], y[3], &kfull[st]);
           }
           if (it + 1 < ntiles) {
             ncode = code_of(it + 1, nsc);
@@ -676,7 +704,7 @@ void attend_tc_plan(AttendParams& p, int n_sm) {
 }
 
 cudaError_t launch_attend_tc(AttendParams& p, int n_sm, cudaStream_t st) {
-  CUtensorMap tm_q, tm_ring, tm_kv;
+  CUtensorMap tm_q, tm_ring, tm_kv, tm_kvg;
   const uint64_t kv_rows = static_cast<uint64_t>(p.n_pages) * p.page_size;
   const uint64_t ring_rows = static_cast<uint64_t>(p.n_seqs_layer) * p.n_win;
   if (kv_rows > kRowMask || ring_rows > kRowMask || static_cast<uint64_t>(p.chunk_len) > kRowMask)
@@ -685,7 +713,10 @@ cudaError_t launch_attend_tc(AttendParams& p, int n_sm, cudaStream_t st) {
       !encode_rows(&tm_ring, p.ring_x, ring_rows, kNk) ||
       // an FP8 pool is never read by TMA (its tiles are widened by the loaders)
       !encode_rows(&tm_kv, p.kv_dtype == CSKV_FP8_E4M3 ? static_cast<const void*>(p.ring_x) : p.kv_pool,
-                   p.kv_dtype == CSKV_FP8_E4M3 ? ring_rows : kv_rows, kNk))
+                   p.kv_dtype == CSKV_FP8_E4M3 ? ring_rows : kv_rows, kNk) ||
+      // one-row boxes of the bf16 pool for the gathered tiles (the selection's rows)
+      !encode_rows(&tm_kvg, p.kv_dtype == CSKV_FP8_E4M3 ? static_cast<const void*>(p.ring_x) : p.kv_pool,
+                   p.kv_dtype == CSKV_FP8_E4M3 ? ring_rows : kv_rows, 1))
     return cudaErrorNotSupported;
   const size_t smem = Smem::bytes(p.n_q);
   const bool fp8 = p.kv_dtype == CSKV_FP8_E4M3;
@@ -697,7 +728,7 @@ cudaError_t launch_attend_tc(AttendParams& p, int n_sm, cudaStream_t st) {
   const int grid = static_cast<int>(items < n_sm ? items : n_sm);
   p.part_t = 1;
   e = launch_pdl(kern, dim3(static_cast<unsigned>(grid < 1 ? 1 : grid)), dim3(kThreads), smem, st, tm_q, tm_ring,
-                 tm_kv, p);
+                 tm_kv, tm_kvg, p);
   if (e != cudaSuccess) return e;
   return launch_attend_merge(p, st);
 }

@@ -24,6 +24,7 @@
 // chosen indices are written in ascending order (equal scores prefer the
 // lower index).
 #include <cooperative_groups.h>
+#include <string.h>
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -318,21 +319,24 @@ constexpr int kTmaThreads = 32 * (1 + kTmaConsumerWarps);
 constexpr int kUnitKeys = 64;
 constexpr int kTmaRingBytes = 128 * 1024;
 
-template <int NCH>
+template <int NCH, bool FP4 = false>
 struct TmaScanShape {
-  static constexpr int ROWB = NCH * 64;                     // bytes per key row
-  static constexpr int STAGE_BYTES = kUnitKeys * ROWB;      // one 64-key unit
-  static constexpr int NSTAGE = kTmaRingBytes / STAGE_BYTES;  // even
+  // bf16: rows of NCH * 64 bytes (2D TMA, 128-byte swizzle); FP4: the unit's codes (d_I / 2 bytes
+  // per row) then its e4m3 scales (d_I / 16 bytes per row), each one contiguous block of the pool
+  static constexpr int ROWB = FP4 ? NCH * 16 : NCH * 64;    // code bytes per key row
+  static constexpr int SCALEB = FP4 ? NCH * 2 : 0;          // scale bytes per key row
+  static constexpr int STAGE_BYTES = kUnitKeys * (ROWB + SCALEB);  // one 64-key unit
+  static constexpr int NSTAGE = kTmaRingBytes / STAGE_BYTES;  // a multiple of the consumer groups
   static size_t smem_bytes(int n_q) {
     return 1024 + (size_t)kTmaRingBytes + 2 * NSTAGE * sizeof(uint64_t) + NSTAGE * sizeof(int) +
            sizeof(int) * (size_t)(n_q + 1);
   }
 };
 
-template <int NCH, int NTH>
+template <int NCH, int NTH, bool FP4>
 __global__ void __launch_bounds__(kTmaThreads, 1)
     index_scan_tma_kernel(const __grid_constant__ CUtensorMap tmap, IndexParams p) {
-  using Sh = TmaScanShape<NCH>;
+  using Sh = TmaScanShape<NCH, FP4>;
   constexpr int NSTAGE = Sh::NSTAGE;
   constexpr int NGROUP = kTmaConsumerWarps / 4;
   static_assert(NSTAGE % NGROUP == 0, "each consumer group owns a fixed set of stages");
@@ -405,7 +409,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     // ------------------------------------------------------------ producer
     // The warp resolves the pool rows of 32 units at a time (one page-table
     // load per lane, in parallel); lane 0 then issues their loads in order.
-    if (lane == 0) prefetch_tensormap(&tmap);
+    if (lane == 0 && !FP4) prefetch_tensormap(&tmap);
     int64_t issued = 0;
     bool ok = true;
     for (int64_t i0 = 0; i0 < n_units && ok; i0 += 32) {
@@ -434,10 +438,17 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
             if (r0 >= 0) {
               s_valid[s] = 1;
               mbar_arrive_expect_tx(&full[s], Sh::STAGE_BYTES);
+              uint8_t* dst = tiles + (size_t)s * Sh::STAGE_BYTES;
+              if constexpr (FP4) {  // 64 consecutive pool rows: their codes, then their scales
+                bulk_load(dst, static_cast<const uint8_t*>(p.idx_pool) + (size_t)r0 * Sh::ROWB, kUnitKeys * Sh::ROWB,
+                          &full[s]);
+                bulk_load(dst + kUnitKeys * Sh::ROWB, p.idx_scale + (size_t)r0 * Sh::SCALEB,
+                          kUnitKeys * Sh::SCALEB, &full[s]);
+              } else {
 #pragma unroll
-              for (int box = 0; box < Sh::ROWB / 128; ++box)
-                tma_load_2d(tiles + (size_t)s * Sh::STAGE_BYTES + box * (kUnitKeys * 128), &tmap, box * 64, r0,
-                            &full[s]);
+                for (int box = 0; box < Sh::ROWB / 128; ++box)
+                  tma_load_2d(dst + box * (kUnitKeys * 128), &tmap, box * 64, r0, &full[s]);
+              }
             } else {
               report(p.status, CSKV_ERR_OUT_OF_RANGE);
               s_valid[s] = 0;
@@ -478,10 +489,21 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
 #pragma unroll
       for (int nt = 0; nt < NTH; ++nt) {
         const int n = 8 * nt + g;
-        const uint16_t* qr = static_cast<const uint16_t*>(p.q_idx) + ((int64_t)b * p.n_heads_idx + n) * p.d_idx;
+        if constexpr (FP4) {  // the thread's channels c*d/4 .. (c+1)*d/4 - 1, as the keys' (fp16, exact)
+          const uint8_t* qr = static_cast<const uint8_t*>(p.q_idx) + ((int64_t)b * p.n_heads_idx + n) * (p.d_idx / 2) +
+                              c * (NCH * 4);
+          const uint8_t* qs = p.q_idx_scale + ((int64_t)b * p.n_heads_idx + n) * (p.d_idx / 16) + c * (NCH / 2);
 #pragma unroll
-        for (int jj = 0; jj < NCH; ++jj)
-          qf[nt][jj] = n < p.n_heads_idx ? ldg16(qr + (c + 4 * jj) * 8) : make_uint4(0u, 0u, 0u, 0u);
+          for (int jj = 0; jj < NCH; ++jj)
+            qf[nt][jj] = n < p.n_heads_idx
+                             ? fp4x8_to_half8(__ldg(reinterpret_cast<const uint32_t*>(qr) + jj), __ldg(qs + jj / 2))
+                             : make_uint4(0u, 0u, 0u, 0u);
+        } else {
+          const uint16_t* qr = static_cast<const uint16_t*>(p.q_idx) + ((int64_t)b * p.n_heads_idx + n) * p.d_idx;
+#pragma unroll
+          for (int jj = 0; jj < NCH; ++jj)
+            qf[nt][jj] = n < p.n_heads_idx ? ldg16(qr + (c + 4 * jj) * 8) : make_uint4(0u, 0u, 0u, 0u);
+        }
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int h = 8 * nt + 2 * c + e;
@@ -502,18 +524,50 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
         for (int h = 0; h < 2; ++h)
 #pragma unroll
           for (int nt = 0; nt < NTH; ++nt) acc[h][nt][0] = acc[h][nt][1] = acc[h][nt][2] = acc[h][nt][3] = 0.f;
+        if constexpr (FP4) {
+          // rows r0 and r0 + 8: the thread's NCH * 4 code bytes (channels c*d/4 ..) and NCH / 2 scales
+          const uint8_t* ca = tb + r0 * Sh::ROWB + c * (NCH * 4);
+          const uint8_t* cb = ca + 8 * Sh::ROWB;
+          const uint8_t* sa = tb + kUnitKeys * Sh::ROWB + r0 * Sh::SCALEB + c * (NCH / 2);
+          const uint8_t* sb = sa + 8 * Sh::SCALEB;
+          uint32_t wa[NCH], wb[NCH];
+          if constexpr (NCH == 4) {
+            const uint4 va = lds16(ca), vb = lds16(cb);
+            wa[0] = va.x; wa[1] = va.y; wa[2] = va.z; wa[3] = va.w;
+            wb[0] = vb.x; wb[1] = vb.y; wb[2] = vb.z; wb[3] = vb.w;
+          } else {
 #pragma unroll
-        for (int jj = 0; jj < NCH; ++jj) {
-          const int q = c + 4 * jj;
-          const int off = (q >> 3) * (kUnitKeys * 128) + (((q & 7) ^ pg) << 4);
-          const uint4 ka = lds16(tb + off + r0 * 128);
-          const uint4 kb = lds16(tb + off + (r0 + 8) * 128);
+            for (int jj = 0; jj < NCH; ++jj) {
+              wa[jj] = reinterpret_cast<const uint32_t*>(ca)[jj];
+              wb[jj] = reinterpret_cast<const uint32_t*>(cb)[jj];
+            }
+          }
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t a[4] = {u4_at(ka, 2 * h), u4_at(kb, 2 * h), u4_at(ka, 2 * h + 1), u4_at(kb, 2 * h + 1)};
+          for (int jj = 0; jj < NCH; ++jj) {
+            const uint4 ka = fp4x8_to_half8(wa[jj], sa[jj / 2]);
+            const uint4 kb = fp4x8_to_half8(wb[jj], sb[jj / 2]);
 #pragma unroll
-            for (int nt = 0; nt < NTH; ++nt)
-              mma_bf16(acc[h][nt], a, u4_at(qf[nt][jj], 2 * h), u4_at(qf[nt][jj], 2 * h + 1));
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t a[4] = {u4_at(ka, 2 * h), u4_at(kb, 2 * h), u4_at(ka, 2 * h + 1), u4_at(kb, 2 * h + 1)};
+#pragma unroll
+              for (int nt = 0; nt < NTH; ++nt)
+                mma_f16(acc[h][nt], a, u4_at(qf[nt][jj], 2 * h), u4_at(qf[nt][jj], 2 * h + 1));
+            }
+          }
+        } else {
+#pragma unroll
+          for (int jj = 0; jj < NCH; ++jj) {
+            const int q = c + 4 * jj;
+            const int off = (q >> 3) * (kUnitKeys * 128) + (((q & 7) ^ pg) << 4);
+            const uint4 ka = lds16(tb + off + r0 * 128);
+            const uint4 kb = lds16(tb + off + (r0 + 8) * 128);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t a[4] = {u4_at(ka, 2 * h), u4_at(kb, 2 * h), u4_at(ka, 2 * h + 1), u4_at(kb, 2 * h + 1)};
+#pragma unroll
+              for (int nt = 0; nt < NTH; ++nt)
+                mma_bf16(acc[h][nt], a, u4_at(qf[nt][jj], 2 * h), u4_at(qf[nt][jj], 2 * h + 1));
+            }
           }
         }
         s0 = 0.f;
@@ -1354,21 +1408,24 @@ cudaError_t launch_scan(IndexParams& p, int n_sm, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int NCH, int NTH>
+template <int NCH, int NTH, bool FP4>
 cudaError_t launch_scan_tma(IndexParams& p, int n_sm, cudaStream_t st) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return cudaErrorNotSupported;
   CUtensorMap map;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.d_idx), static_cast<cuuint64_t>(p.n_pages) * p.page_size};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.d_idx) * 2};
-  const cuuint32_t box[2] = {64, kUnitKeys};
-  const cuuint32_t estr[2] = {1, 1};
-  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p.idx_pool), dims, strides, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  auto kern = index_scan_tma_kernel<NCH, NTH>;
-  const size_t smem = TmaScanShape<NCH>::smem_bytes(p.n_q);
+  memset(&map, 0, sizeof(map));
+  if (!FP4) {  // FP4 units are two plain bulk copies; bf16 rows go through a swizzled 2D map
+    auto enc = tensor_map_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.d_idx), static_cast<cuuint64_t>(p.n_pages) * p.page_size};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.d_idx) * 2};
+    const cuuint32_t box[2] = {64, kUnitKeys};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p.idx_pool), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  auto kern = index_scan_tma_kernel<NCH, NTH, FP4>;
+  const size_t smem = TmaScanShape<NCH, FP4>::smem_bytes(p.n_q);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int64_t units_max = (visible_entries(p.max_pos, p.m, p.n_win) + kUnitKeys - 1) / kUnitKeys;
@@ -1658,11 +1715,12 @@ cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st) {
   cudaError_t e = cudaSuccess;
   const bool fp4 = p.idx_dtype == CSKV_FP4_E2M1;
   const int nth = (p.n_heads_idx + 7) / 8;
-  const bool tma_ok = !fp4 && p.page_size % kUnitKeys == 0 && (p.d_idx == 64 || p.d_idx == 128) && nth <= 2 &&
+  const bool tma_ok = p.page_size % kUnitKeys == 0 && (p.d_idx == 64 || p.d_idx == 128) && nth <= 2 &&
                       (reinterpret_cast<uintptr_t>(p.idx_pool) & 15u) == 0 &&
+                      (!fp4 || (reinterpret_cast<uintptr_t>(p.idx_scale) & 15u) == 0) &&
                       (int64_t)p.n_pages * p.page_size < (int64_t(1) << 31);
   // many queries in one call (a prefill chunk): the grouped scan reads each key once per group
-  const bool grouped = tma_ok && p.n_q >= kGroupScanMinQueries && (p.n_heads_idx == 4 || p.n_heads_idx == 8);
+  const bool grouped = tma_ok && !fp4 && p.n_q >= kGroupScanMinQueries && (p.n_heads_idx == 4 || p.n_heads_idx == 8);
   if (nv_max > 0 && grouped) {
     if (scan_tc_supported(p)) e = launch_scan_tc(p, n_sm, st);
     else if (p.d_idx == 64 && p.n_heads_idx == 4) e = launch_scan_group<2, 4>(p, n_sm, st);
@@ -1674,10 +1732,17 @@ cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st) {
     p.hist = reinterpret_cast<uint32_t*>(p.scores + (size_t)p.n_q * p.vis_stride);
     e = cudaMemsetAsync(p.hist, 0, sizeof(uint32_t) * kHistBins * (size_t)p.n_q, st);
     if (e != cudaSuccess) return e;
-    if (p.d_idx == 64 && nth == 1) e = launch_scan_tma<2, 1>(p, n_sm, st);
-    else if (p.d_idx == 64 && nth == 2) e = launch_scan_tma<2, 2>(p, n_sm, st);
-    else if (p.d_idx == 128 && nth == 1) e = launch_scan_tma<4, 1>(p, n_sm, st);
-    else e = launch_scan_tma<4, 2>(p, n_sm, st);
+    if (fp4) {
+      if (p.d_idx == 64 && nth == 1) e = launch_scan_tma<2, 1, true>(p, n_sm, st);
+      else if (p.d_idx == 64 && nth == 2) e = launch_scan_tma<2, 2, true>(p, n_sm, st);
+      else if (p.d_idx == 128 && nth == 1) e = launch_scan_tma<4, 1, true>(p, n_sm, st);
+      else e = launch_scan_tma<4, 2, true>(p, n_sm, st);
+    } else {
+      if (p.d_idx == 64 && nth == 1) e = launch_scan_tma<2, 1, false>(p, n_sm, st);
+      else if (p.d_idx == 64 && nth == 2) e = launch_scan_tma<2, 2, false>(p, n_sm, st);
+      else if (p.d_idx == 128 && nth == 1) e = launch_scan_tma<4, 1, false>(p, n_sm, st);
+      else e = launch_scan_tma<4, 2, false>(p, n_sm, st);
+    }
     if (e != cudaSuccess) return e;
   } else if (nv_max > 0) {
     if (!fp4 && p.d_idx == 64 && nth == 1) e = launch_scan<2, 1, 2, false>(p, n_sm, st);
@@ -1696,8 +1761,7 @@ cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st) {
   // selection: a cluster of CL CTAs per query, each holding a slice of scores
   int cl_min = static_cast<int>((nv_max + kSliceCap - 1) / kSliceCap);
   if (cl_min < 1) cl_min = 1;
-  if (cl_min > kMaxCluster) return cudaErrorNotSupported;
-  if (p.n_q == 0) return cudaSuccess;
+  if (cl_min > kMaxCluster) return launch_select_stream(p, st);  // slices beyond a 16-CTA cluster
   int cl0 = n_sm / p.n_q;
   if (cl0 > kMaxCluster) cl0 = kMaxCluster;
   if (cl0 < cl_min) cl0 = cl_min;
@@ -1733,19 +1797,20 @@ cudaError_t launch_index(IndexParams& p, void* ws, int n_sm, cudaStream_t st) {
   };
   // The largest cluster, down from cl0, whose n_q clusters are all resident at
   // once (a second wave would double the time); clusters above 8 CTAs must fit
-  // in one GPC, which not every GPC can host. If none fits in one wave, the
-  // largest portable size.
+  // in one GPC, which not every GPC can host.
   int chosen = -1;
   for (int cl = cl0; cl >= cl_min && chosen < 0; --cl) {
     shape(cl);
     const int fit = max_active_clusters(cl, cfg.dynamicSmemBytes, &cfg);
     if (fit >= p.n_q) chosen = cl;
   }
+  // no cluster size fits all queries in one wave (many long queries): the clusters run in waves
+  // (one streaming CTA per query would stream the longest queries' scores too slowly)
   if (chosen < 0) {
     chosen = cl0 < 8 ? cl0 : (cl_min > 8 ? cl_min : 8);
     if (chosen > 8) {
       shape(chosen);
-      if (max_active_clusters(chosen, cfg.dynamicSmemBytes, &cfg) < 1) return cudaErrorNotSupported;
+      if (max_active_clusters(chosen, cfg.dynamicSmemBytes, &cfg) < 1) return launch_select_stream(p, st);
     }
   }
   shape(chosen);
