@@ -188,7 +188,11 @@ def workload_text(cfg, nq, model):
 # the digest of the kernel sources it was captured from; once those sources change
 # the figure no longer describes the build and `traffic` is reported as null.
 INDEX_OP_SOURCES = ("compressed_sparse_kv_02_b200/csrc/indexer.cu", "compressed_sparse_kv_02_b200/csrc/cskv_device.cuh")
-INDEX_OP_DRAM = {}  # workload -> (source digest, DRAM bytes per query)
+INDEX_OP_DRAM = {  # workload -> (digest of INDEX_OP_SOURCES at the capture, DRAM bytes per query)
+    # ncu dram__bytes_read.sum + dram__bytes_write.sum of the scan and the select of one indexer call
+    # of the Pro 1M workload at batch 2 (134.31 + 3.74 + 2.20 MB), per query
+    "pro": ("929dd11793dc7cb3", 70125568),
+}
 
 
 def sources_digest(paths=INDEX_OP_SOURCES):
