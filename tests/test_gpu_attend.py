@@ -154,16 +154,18 @@ def test_prefill_chunk_window(ck, orc):
         assert_close(out[i].float().cpu().numpy(), o, ATOL_BF16, REL_BF16, "chunk row %d" % i)
 
 
-def test_invalid_selection_is_reported(ck, orc):
-    B, d, H, m, k = 1, 128, 16, 4, 8
+@pytest.mark.parametrize("d,dv,H", [(128, 128, 16), (576, 512, 128)])  # the generic and the tensor-memory kernel
+def test_invalid_selection_is_reported(ck, orc, d, dv, H):
+    # (with 576 / 512 the selected rows are gathered by TMA; the bad index's row reads as zeros and is masked)
+    B, m, k = 1, 4, 8
     t = 127 + 4 * 20
-    L = make_layer(ck.LAYER_CSA, m, d, d, B, 40, d_idx=64, seed=16)
+    L = make_layer(ck.LAYER_CSA, m, d, dv, B, 40, d_idx=64, seed=16)
     g = torch.Generator().manual_seed(16)
     _fill(ck, L, B, 40, g, sharp=False)
     sel = torch.tensor([[0, 3, 25, -1, -1, -1, -1, -1]], dtype=torch.int32, device="cuda")  # 25 is not visible
     cnt = torch.tensor([3], dtype=torch.int32, device="cuda")
     q = torch.randn(B, H, d, generator=g).to(torch.bfloat16).cuda()
-    out = torch.zeros(B, H, d, dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros(B, H, dv, dtype=torch.bfloat16, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     ck.csa_attend(L, torch.zeros(1, dtype=torch.int32, device="cuda"), torch.tensor([t], device="cuda"), t, q, sel,
                   cnt, out, status=status)
@@ -172,7 +174,7 @@ def test_invalid_selection_is_reported(ck, orc):
     win = ring_window(L, 0, t)
     ent = layer_entries(L, 0, 20)["kv"]
     keys = np.vstack([orc.decode(win), orc.decode(ent)[[0, 3]]])
-    o, _ = orc.attend(stored_bf16(q[0]), orc.f64(keys), d, 1.0 / math.sqrt(d))
+    o, _ = orc.attend(stored_bf16(q[0]), orc.f64(keys), dv, 1.0 / math.sqrt(d))
     assert_close(out[0].float().cpu().numpy(), o, ATOL_BF16, REL_BF16, "masked")
 
 
