@@ -351,12 +351,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         else
           prefetch_l2(code_row(p, c), kDqk * 2);
       };
+      // the next tile's source (its page-table lookup included) is found before its stage frees
       float nsc = 0.f;
       uint32_t ncode = ntiles > 0 ? code_of(0, nsc) : 0u;
-      {
-        int rr0;
-        if (ntiles > 0 && tile_src(0, rr0) < 0) prefetch(ncode);
-      }
+      int nrow0 = 0;
+      int nmode = ntiles > 0 ? tile_src(0, nrow0) : -1;
+      if (ntiles > 0 && nmode < 0) prefetch(ncode);
       for (int it = 0; it < ntiles; ++it) {
         const uint32_t gt = g + it;
         const int st = gt & 1;
@@ -388,8 +388,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         named_sync(3, kLoaders);
         uint8_t* dst = sK + st * kStageBytes;
-        int row0 = 0;
-        const int mode = tile_src(it, row0);
+        const int row0 = nrow0;
+        const int mode = nmode;
         if (mode >= 0) {
           if (lt == 0) {
             mbar_arrive_expect_tx(&kfull[st], kStageBytes);
@@ -398,8 +398,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (it + 1 < ntiles) {
             ncode = code_of(it + 1, nsc);
-            int rr0;
-            if (tile_src(it + 1, rr0) < 0) prefetch(ncode);
+            nmode = tile_src(it + 1, nrow0);
+            if (nmode < 0) prefetch(ncode);
           }
         } else if (!fp8 && sPool[0] && sPool[1]) {
           // the tile's rows by TMA gather, four rows of one 64-channel block per copy; a key without
@@ -418,8 +418,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (it + 1 < ntiles) {
             ncode = code_of(it + 1, nsc);
-            int rr0;
-            if (tile_src(it + 1, rr0) < 0) prefetch(ncode);
+            nmode = tile_src(it + 1, nrow0);
+            if (nmode < 0) prefetch(ncode);
           }
         } else {
           // consecutive threads take consecutive 16-byte chunks of a row (coalesced): chunk c of key
@@ -462,8 +462,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           cp_async_commit();
           if (it + 1 < ntiles) {  // the next tile's rows are looked up while this tile's copies fly
             ncode = code_of(it + 1, nsc);
-            int rr0;
-            if (tile_src(it + 1, rr0) < 0) prefetch(ncode);
+            nmode = tile_src(it + 1, nrow0);
+            if (nmode < 0) prefetch(ncode);
           }
           cp_async_wait<0>();
           fence_proxy_async_smem();
