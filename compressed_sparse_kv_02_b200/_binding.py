@@ -67,7 +67,7 @@ class AppendArgs(ctypes.Structure):
     _fields_ = [
         ("struct_size", ctypes.c_uint32), ("layer", ctypes.POINTER(LayerStruct)), ("n_seq", _I32),
         ("n_new", _I32), ("seq_ids", _P), ("pos", _P), ("x", _P), ("z", _P), ("xi", _P), ("zi", _P),
-        ("ring_only", _I32), ("d_status", _P),
+        ("ring_only", _I32), ("d_status", _P), ("emit_only", _I32),
     ]
 
 
@@ -335,8 +335,9 @@ def hca_compress_kv(layer: Layer, seq_ids, tok0: int, x, z, status=None, stream=
 
 
 def cskv_cache_append(layer: Layer, seq_ids, pos, x, z, xi=None, zi=None, ring_only=False, status=None,
-                      stream=None):
-    """Append n_new tokens per sequence to the state-cache rings; fold completed blocks into the cache."""
+                      stream=None, emit_only=False):
+    """Append n_new tokens per sequence to the state-cache rings; fold completed blocks into the cache
+    (ring_only: the rings only; emit_only: the completed blocks only, the rings holding the tokens already)."""
     n_seq, n_new = x.shape[0], x.shape[1]
     _need(seq_ids, "seq_ids", torch.int32, (n_seq,))
     _need(pos, "pos", torch.int64, (n_seq,))
@@ -347,7 +348,7 @@ def cskv_cache_append(layer: Layer, seq_ids, pos, x, z, xi=None, zi=None, ring_o
         _need(zi, "zi", torch.bfloat16, (n_seq, n_new, layer.gate_cols_idx))
     _need(status, "status", torch.int32, optional=True)
     a = AppendArgs(ctypes.sizeof(AppendArgs), ctypes.pointer(layer.struct), n_seq, n_new, _ptr(seq_ids), _ptr(pos),
-                   _ptr(x), _ptr(z), _ptr(xi), _ptr(zi), int(bool(ring_only)), _ptr(status))
+                   _ptr(x), _ptr(z), _ptr(xi), _ptr(zi), int(bool(ring_only)), _ptr(status), int(bool(emit_only)))
     _check(lib().cskv_cache_append(ctypes.byref(a), _stream(stream)), "cskv_cache_append")
 
 

@@ -243,6 +243,12 @@ cskv_status attend_impl(const cskv_attend_args* a, void* ws, size_t ws_bytes, vo
   return from_cuda(cskv::launch_attend(p, ws, n_sm, static_cast<cudaStream_t>(stream)));
 }
 
+// struct_size of the append args before emit_only was added (such callers get 0)
+constexpr size_t kAppendArgsV1 = offsetof(cskv_append_args, d_status) + sizeof(int32_t*);
+int32_t append_emit_only(const cskv_append_args* a) {
+  return a->struct_size >= offsetof(cskv_append_args, emit_only) + sizeof(int32_t) ? a->emit_only : 0;
+}
+
 }  // namespace
 
 extern "C" {
@@ -276,7 +282,9 @@ cskv_status hca_compress_kv(const cskv_compress_args* args, void* stream) {
 }
 
 cskv_status cskv_cache_append(const cskv_append_args* a, void* stream) {
-  if (!a || a->struct_size < sizeof(cskv_append_args)) return CSKV_ERR_INVALID_ARG;
+  if (!a || a->struct_size < kAppendArgsV1) return CSKV_ERR_INVALID_ARG;
+  const int32_t emit_only = append_emit_only(a);
+  if (emit_only && a->ring_only) return CSKV_ERR_INVALID_ARG;
   const cskv_layer* L = a->layer;
   cskv_status s = check_layer_shape(L);
   if (s) return s;
@@ -297,6 +305,7 @@ cskv_status cskv_cache_append(const cskv_append_args* a, void* stream) {
   p.pos = a->pos;
   p.n_new = a->n_new;
   p.ring_only = a->ring_only;
+  p.emit_only = emit_only;
   p.status = a->d_status;
   return from_cuda(cskv::launch_append(p, static_cast<cudaStream_t>(stream)));
 }

@@ -65,7 +65,8 @@ struct FoldParams {
   // append: rows [n_seq, n_new, ...] starting at pos[b]
   const int64_t* pos;
   int n_new;
-  int ring_only;
+  int ring_only;  // the rings only
+  int emit_only;  // the completed blocks only (the rings already hold the tokens)
   int32_t* status;
 };
 

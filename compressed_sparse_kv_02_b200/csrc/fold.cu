@@ -414,9 +414,10 @@ __device__ void store_row(const FoldStream& S, int64_t row, const float* sv, int
 
 // Grid (sequence, 64-channel slice, stream); an FP8 stream is handled whole by
 // slice 0 (its scale is the row's amax). Each CTA copies its channels of the
-// new rows into the rings, then folds its channels of every block the new
-// tokens complete (old rows from the ring, new rows from the input; the slots
-// written and the slots read never coincide because n_new + m - 1 <= n_win).
+// new rows into the rings (not with emit_only), then folds its channels of
+// every block the new tokens complete (not with ring_only; old rows from the
+// ring, new rows from the input; the slots written and the slots read never
+// coincide because n_new + m - 1 <= n_win).
 // All 512 threads fold: thread (token group g, channel pair) runs the online
 // softmax of the gate over tokens g, g + 16, ... of the block for its two
 // channels, and one thread per channel merges the 16 groups' states from
@@ -441,7 +442,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(FoldParams p) {
   const int c_hi = whole ? S.d : min(S.d, c_lo + kSliceCh);
   if (c_lo >= S.d || (whole && slice != 0)) return;
   const int64_t pos = p.pos[b];
-  {  // ring rows of the new tokens (this CTA's channels; gate logits: a per-token logit goes with c_lo == 0)
+  if (!p.emit_only) {  // ring rows of the new tokens (this CTA's channels; gate logits: a per-token logit goes with c_lo == 0)
     const int cx = (c_hi - c_lo) / 8;
     for (int k = t; k < p.n_new * cx; k += kAppendThreads) {
       const int i = k / cx, ch = k % cx;

@@ -6,9 +6,19 @@ Per layer pair and step, for a batch of sequences whose newest token sits at
 position t_b:
   CSA: cskv_cache_append -> csa_index_score_topk -> csa_attend
   HCA: cskv_cache_append -> hca_attend
-The argument blocks are marshalled once (`DecodeModel.prepare`) so that a step
-is five foreign calls per layer pair; the whole step can also be captured in
-a CUDA graph (every call is stream-ordered and allocates nothing).
+The entry a step completes covers positions inside the step's own window, so
+no query of the step reads it (the visibility rule: an entry is visible once
+it lies wholly before the window). Its compression therefore runs off the
+critical path, on a second stream:
+  CSA: the whole append runs beside the indexer; csa_attend, which reads the
+       ring's new row, waits for it;
+  HCA: the ring rows are written first (ring_only), the compression
+       (emit_only) runs beside hca_attend;
+and the step ends when both streams have finished (the next append of a layer
+overwrites ring rows that the compression reads). The argument blocks are
+marshalled once (`DecodeModel.prepare`); the whole step can also be captured
+in a CUDA graph (every call is stream-ordered and allocates nothing, and the
+second stream forks from and joins the first through events).
 """
 from __future__ import annotations
 
@@ -22,11 +32,15 @@ from . import _binding as B
 from . import synth
 
 
-class _Call:
-    __slots__ = ("fn", "args", "ws", "ws_bytes", "where")
+FORK = "fork"  # the side stream waits for everything issued on the main stream so far
+JOIN = "join"  # the main stream waits for everything issued on the side stream so far
 
-    def __init__(self, fn, args, ws=None, where=""):
-        self.fn, self.args, self.where = fn, args, where
+
+class _Call:
+    __slots__ = ("fn", "args", "ws", "ws_bytes", "where", "side")
+
+    def __init__(self, fn, args, ws=None, where="", side=False):
+        self.fn, self.args, self.where, self.side = fn, args, where, side
         self.ws = None if ws is None else ctypes.c_void_p(ws.data_ptr())
         self.ws_bytes = 0 if ws is None else ws.numel()
 
@@ -92,6 +106,8 @@ class DecodeModel:
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.inputs = None
         self._calls = None
+        self._ops = None
+        self._side = torch.cuda.Stream(device=device) if torch.device(device).type == "cuda" else None
 
     @property
     def n_pairs(self) -> int:
@@ -180,11 +196,15 @@ class DecodeModel:
         torch.cuda.synchronize()
 
     def prepare(self, inputs: Optional[dict] = None):
-        """Marshal every call of a step once; `inputs` (device tensors) defaults to self.inputs."""
+        """Marshal every call of a step once; `inputs` (device tensors) defaults to self.inputs.
+
+        Returns the step's ops for `run`: the calls in issue order (a call's `side` says which stream
+        it goes to) with FORK / JOIN markers between them."""
         inp = self.inputs if inputs is None else inputs
         L = B.lib()
         cfg = self.cfg
         calls = []
+        ops = []
         sm = 1.0 / math.sqrt(cfg.d_qk)
         self._keep = []
         for li in range(self.n_pairs):
@@ -195,35 +215,66 @@ class DecodeModel:
                 self._keep.append(s)
                 lp = ctypes.pointer(s)
                 is_csa = kind == "csa"
-                a = B.AppendArgs(ctypes.sizeof(B.AppendArgs), lp, cfg.batch, 1, B._ptr(self.seq), B._ptr(self.pos),
-                                 B._ptr(x[kind + "_x"]), B._ptr(x[kind + "_z"]),
-                                 B._ptr(x["csa_xi"]) if is_csa else None, B._ptr(x["csa_zi"]) if is_csa else None,
-                                 0, B._ptr(self.status))
-                calls.append(_Call(L.cskv_cache_append, a, where="cskv_cache_append"))
+                def append_args(ring_only, emit_only):
+                    return B.AppendArgs(ctypes.sizeof(B.AppendArgs), lp, cfg.batch, 1, B._ptr(self.seq),
+                                        B._ptr(self.pos), B._ptr(x[kind + "_x"]), B._ptr(x[kind + "_z"]),
+                                        B._ptr(x["csa_xi"]) if is_csa else None,
+                                        B._ptr(x["csa_zi"]) if is_csa else None,
+                                        ring_only, B._ptr(self.status), emit_only)
+
+                n0 = len(calls)
                 if is_csa:
                     ia = B._index_args(layer, self.seq, self.pos, self.max_pos, x["q_idx"], x["w"], cfg.k, o["idx"],
                                        o["cnt"], None, x.get("q_idx_scale"), self.status)
-                    calls.append(_Call(L.csa_index_score_topk, ia, self.ws_index, "csa_index_score_topk"))
                     aa = B._attend_args(layer, self.seq, self.pos, self.max_pos, x["q_csa"], o["idx"], o["cnt"],
                                         cfg.k, sm, o["o_csa"], o["lse_csa"], None, 0, self.status)
-                    calls.append(_Call(L.csa_attend, aa, self.ws_csa, "csa_attend"))
+                    calls += [_Call(L.cskv_cache_append, append_args(0, 0), where="cskv_cache_append", side=True),
+                              _Call(L.csa_index_score_topk, ia, self.ws_index, "csa_index_score_topk"),
+                              _Call(L.csa_attend, aa, self.ws_csa, "csa_attend")]
+                    ops += [FORK, calls[n0], calls[n0 + 1], JOIN, calls[n0 + 2]]
                 else:
                     aa = B._attend_args(layer, self.seq, self.pos, self.max_pos, x["q_hca"], None, None, 0, sm,
                                         o["o_hca"], o["lse_hca"], None, 0, self.status)
-                    calls.append(_Call(L.hca_attend, aa, self.ws_hca, "hca_attend"))
-                for c in calls[-3 if is_csa else -2:]:
-                    if hasattr(c.args, "layer"):
-                        self._keep.append(c.args)
+                    calls += [_Call(L.cskv_cache_append, append_args(1, 0), where="cskv_cache_append_ring"),
+                              _Call(L.cskv_cache_append, append_args(0, 1), where="cskv_cache_append_emit", side=True),
+                              _Call(L.hca_attend, aa, self.ws_hca, "hca_attend")]
+                    ops += [calls[n0], FORK, calls[n0 + 1], calls[n0 + 2]]
+                for c in calls[n0:]:
+                    self._keep.append(c.args)
+        ops.append(JOIN)
         self._calls = calls
-        return calls
+        self._ops = ops
+        return ops
+
+    def run(self, ops, stream=None, before=None, after=None):
+        """Issue `ops` (from `prepare`) on `stream` (default: torch's current stream) and the side stream;
+        before / after (optional) are called as f(i, call, stream) around the i-th call."""
+        main = torch.cuda.current_stream() if stream is None else stream
+        side = self._side
+        i = 0
+        for op in ops:
+            if op is FORK:
+                e = torch.cuda.Event()
+                e.record(main)
+                side.wait_event(e)
+            elif op is JOIN:
+                e = torch.cuda.Event()
+                e.record(side)
+                main.wait_event(e)
+            else:
+                s = side if op.side else main
+                if before is not None:
+                    before(i, op, s)
+                op(B._stream(s))
+                if after is not None:
+                    after(i, op, s)
+                i += 1
 
     def step(self, stream=None):
         """Run one decode step (all layer pairs) on `stream` (default: torch's current stream)."""
-        if self._calls is None:
+        if self._ops is None:
             self.prepare()
-        st = B._stream(stream)
-        for c in self._calls:
-            c(st)
+        self.run(self._ops, stream)
 
     def check_status(self) -> int:
         return B.cskv_get_status(self.status)

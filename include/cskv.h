@@ -200,6 +200,15 @@ cskv_status hca_compress_kv(const cskv_compress_args* args, void* stream);
  * Requires n_new + m - 1 + overlap <= n_win (every completed block, and the
  * tokens it overlaps, are still in the ring). ring_only = 1 writes the rings
  * and emits nothing (used after a bulk compression of the same tokens).
+ * emit_only = 1 (a field added after d_status; callers whose struct_size ends
+ * before it get 0) writes no ring row and only compresses the blocks these
+ * tokens complete: for a caller that has already written the same tokens with
+ * ring_only = 1, stream-ordered before this call, and that moves the
+ * compression off its critical path (an entry completed at position t covers
+ * positions inside t's window, so no query up to t reads it). Until this call
+ * has completed, the ring rows of the blocks it compresses must not be
+ * overwritten (the layer's next append) and the entries it writes not read.
+ * ring_only and emit_only together are an invalid argument.
  */
 typedef struct {
   uint32_t struct_size;
@@ -214,6 +223,7 @@ typedef struct {
   const void* zi;
   int32_t ring_only;
   int32_t* d_status;
+  int32_t emit_only;
 } cskv_append_args;
 
 cskv_status cskv_cache_append(const cskv_append_args* args, void* stream);

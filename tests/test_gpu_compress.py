@@ -185,6 +185,53 @@ def test_multi_token_append_and_ring_only(ck, orc):
     assert torch.equal(L1.ring_x, L2.ring_x) and torch.equal(L1.ring_zi, L2.ring_zi)
 
 
+@pytest.mark.parametrize("kind,m", [("csa", 4), ("hca", 128)])
+def test_append_ring_then_emit_equals_append(ck, kind, m):
+    """The split append of a decode step (ring_only, then emit_only with the same tokens, as the decode
+    step issues it to take the compression off its critical path) writes the same ring rows and the same
+    entries, bit for bit, as one append; emit_only writes no ring row; both flags at once are refused."""
+    B, d, d_idx = 2, 128, 64
+    n = 2 * 128 + 8
+    is_csa = kind == "csa"
+    mk = lambda: make_layer(ck.LAYER_CSA if is_csa else ck.LAYER_HCA, m, d, d, B, n // m + 2,
+                            d_idx=d_idx if is_csa else 0, seed=6)
+    La, Lb = mk(), mk()
+    x, z = _stream(B, n + 1, d, d, seed=20)
+    xi, zi = _stream(B, n + 1, d_idx, d_idx, seed=21)
+    seq = torch.tensor([1, 0], dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def tok(t):
+        sl = slice(t, t + 1)
+        return (x[:, sl].contiguous(), z[:, sl].contiguous(), xi[:, sl].contiguous() if is_csa else None,
+                zi[:, sl].contiguous() if is_csa else None)
+
+    for t in range(n):
+        pos = torch.full((B,), t, dtype=torch.int64, device="cuda")
+        ck.cskv_cache_append(La, seq, pos, *tok(t), status=status)
+        ck.cskv_cache_append(Lb, seq, pos, *tok(t), ring_only=True, status=status)
+        ck.cskv_cache_append(Lb, seq, pos, *tok(t), emit_only=True, status=status)
+    assert ck.cskv_get_status(status) == ck.OK
+    rings = ("ring_x", "ring_z") + (("ring_xi", "ring_zi") if is_csa else ())
+    for r in rings:
+        assert torch.equal(getattr(La, r), getattr(Lb, r)), r
+    for b in range(B):
+        ea, eb = layer_entries(La, int(seq[b]), n // m), layer_entries(Lb, int(seq[b]), n // m)
+        assert np.array_equal(ea["kv"].data, eb["kv"].data)
+        if is_csa:
+            assert np.array_equal(ea["idx"].data, eb["idx"].data)
+    before = {r: getattr(Lb, r).clone() for r in rings}
+    ck.cskv_cache_append(Lb, seq, torch.full((B,), n, dtype=torch.int64, device="cuda"), *tok(n), emit_only=True,
+                         status=status)
+    assert ck.cskv_get_status(status) == ck.OK
+    for r in rings:
+        assert torch.equal(getattr(Lb, r), before[r]), r
+    with pytest.raises(ck.CskvError) as e:
+        ck.cskv_cache_append(Lb, seq, torch.full((B,), n, dtype=torch.int64, device="cuda"), *tok(n),
+                             ring_only=True, emit_only=True)
+    assert e.value.code == ck.ERR_INVALID_ARG
+
+
 def test_append_rejects_too_many_tokens(ck):
     L = make_layer(ck.LAYER_CSA, 4, 128, 128, 1, 64, d_idx=64)
     x = torch.zeros(1, 126, 128, dtype=torch.bfloat16, device="cuda")
