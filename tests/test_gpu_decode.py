@@ -12,6 +12,8 @@
   FP4 indexer keys and queries, per-sequence lengths, layers CSA, HCA, CSA,
   HCA) at a reduced batch and length (every query), and at the benchmark's
   full size (B = 64, lengths up to ~1M; sampled sequences), both layer pairs.
+* a step captured in a CUDA graph (compression on the second stream) writes
+  what the eager step writes, bit for bit.
 """
 import math
 
@@ -216,6 +218,64 @@ def test_mixed_fp8_fp4_two_pairs(ck, orc):
     torch.cuda.synchronize()
     assert model.check_status() == ck.OK
     _mixed_checks(orc, model, cfg, lens, range(len(lens)), [0, 5, 64, 127])
+
+
+def test_graph_replayed_step_matches_eager(ck):
+    """A decode step captured in a CUDA graph (the form the benchmark times: the compression of the
+    completed entries on a second stream, forked and joined through events) writes what the eager step
+    writes: both layer pairs' outputs, the new ring rows and the entries the appends emit, bit for bit.
+    The outputs, the new rows and the emitted entries are cleared before the replay, so each must come
+    from it; a sequence whose last token completes both a CSA and an HCA block makes both appends emit."""
+    from compressed_sparse_kv_02_b200 import decode, synth
+    cfg = synth.Config("mixed_small", 4, 1 << 16, 128, 576, 512, 8, 128, 1024, seed=4, kv_dtype="fp8",
+                       idx_dtype="fp4")
+    lens = synth.mixed_lengths(cfg, lo=4096, hi=1 << 16)
+    lens[0] = 4096
+    model = decode.DecodeModel(cfg, ctx_lens=lens, n_pairs=2)
+    model.fill_synthetic()
+    model.step()
+    torch.cuda.synchronize()
+    assert model.check_status() == ck.OK
+    t = lens[0] - 1
+    rings = ("ring_x", "ring_z", "ring_xi", "ring_zi")
+
+    def snapshot():
+        snap = {}
+        for li, d in model.out.items():
+            for k_, v in d.items():
+                snap["out%d.%s" % (li, k_)] = v.clone()
+        for i, L in enumerate(model.layers):
+            for r in rings:
+                if getattr(L, r) is not None:
+                    snap["L%d.%s" % (i, r)] = getattr(L, r)[0][t % cfg.n_win].clone()
+            j = (t + 1) // L.m - 1
+            for k_, v in L.read_entries(0, 1, j0=j).items():
+                snap["L%d.%s" % (i, k_)] = v.clone()
+        return snap
+
+    eager = snapshot()
+    stream = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        model.step(stream)
+    for d in model.out.values():
+        for v in d.values():
+            v.zero_()
+    for L in model.layers:
+        for r in rings:
+            if getattr(L, r) is not None:
+                getattr(L, r)[0][t % cfg.n_win].zero_()
+        j = (t + 1) // L.m - 1
+        e = L.read_entries(0, 1, j0=j)
+        L.write_entries(0, j, **{k_: torch.zeros_like(v) for k_, v in e.items()})
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert model.check_status() == ck.OK
+    replayed = snapshot()
+    for k_, v in eager.items():
+        assert torch.equal(v, replayed[k_]), k_
 
 
 def test_mixed_fullsize_sampled(ck, orc):
