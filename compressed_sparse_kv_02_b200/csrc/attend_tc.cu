@@ -421,6 +421,70 @@ __global__ void __launch_bounds__(kThreads, 1)
             nmode = tile_src(it + 1, nrow0);
             if (nmode < 0) prefetch(ncode);
           }
+        } else if (fp8 && sPool[0] && sPool[1]) {
+          // FP8 pool rows: the tile's E4M3 codes (half a bf16 tile) are copied into the stage's upper
+          // half by cp.async, block-major (block j's 64 codes of every key at stg + 4096 j), so the
+          // next tile's row lookups overlap the copies; then they are widened exactly to bf16 in
+          // place, in passes whose writes cover only staged blocks that earlier passes have read:
+          // blocks 0-3 (below the staged codes), 4-5, 6, 7, then 8, whose own codes it overwrites
+          // (read first, then a barrier). A key without a row gets zeros.
+          constexpr int kStg = kStageBytes / 2;            // 36864
+          constexpr int kCodeBlk = kNk * 64;               // 4096: one staged block of codes
+          static_assert(kStg + kNb * kCodeBlk == kStageBytes && 4 * kBlkBytes <= kStg, "staging");
+          uint8_t* stg = dst + kStg;
+          const uint8_t* pool = static_cast<const uint8_t*>(p.kv_pool);
+          for (int q = lt; q < kNk * kNb * 4; q += kLoaders) {  // (key, block, 16-byte piece)
+            const int kr = q / (kNb * 4), j = (q / 4) % kNb, c4 = q % 4;
+            const uint32_t cd = sCode[st * kNk + kr];
+            if (cd)
+              cp_async16(stg + j * kCodeBlk + kr * 64 + c4 * 16,
+                         pool + (size_t)(cd & kRowMask) * kDqk + j * 64 + c4 * 16, 16);
+          }
+          cp_async_commit();
+          if (it + 1 < ntiles) {  // the next tile's rows are looked up while the codes fly
+            ncode = code_of(it + 1, nsc);
+            nmode = tile_src(it + 1, nrow0);
+            if (nmode < 0) prefetch(ncode);
+          }
+          cp_async_wait<0>();
+          // the 8 codes of bf16 chunk (key kr, block j, piece pc), and their widened store
+          auto codes_at = [&](int kr, int j, int pc) -> uint2 {
+            return sCode[st * kNk + kr] ? *reinterpret_cast<const uint2*>(stg + j * kCodeBlk + kr * 64 + pc * 8)
+                                        : make_uint2(0u, 0u);
+          };
+          auto put = [&](int kr, int j, int pc, uint2 c8) {
+            *reinterpret_cast<uint4*>(dst + j * kBlkBytes + kr * 128 + ((pc ^ (kr & 7)) << 4)) = e4m3x8_to_bf16x8(c8);
+          };
+          auto widen = [&](int j0, int j1) {  // blocks j0 .. j1 - 1
+            for (int id = lt; id < kNk * (j1 - j0) * 8; id += kLoaders) {
+              const int kr = id / ((j1 - j0) * 8), j = j0 + (id / 8) % (j1 - j0), pc = id % 8;
+              put(kr, j, pc, codes_at(kr, j, pc));
+            }
+          };
+          named_sync(3, kLoaders);  // every staged code is visible to every loader
+          widen(0, 4);
+          named_sync(3, kLoaders);
+          widen(4, 6);  // overwrites staged blocks 0-2
+          named_sync(3, kLoaders);
+          widen(6, 7);  // 3-4
+          named_sync(3, kLoaders);
+          widen(7, 8);  // 5-6
+          constexpr int kLastPer = (kNk * 8 + kLoaders - 1) / kLoaders;  // 6
+          uint2 last[kLastPer];
+#pragma unroll
+          for (int k2 = 0; k2 < kLastPer; ++k2) {
+            const int id = lt + k2 * kLoaders;
+            last[k2] = id < kNk * 8 ? codes_at(id / 8, kNb - 1, id % 8) : make_uint2(0u, 0u);
+          }
+          named_sync(3, kLoaders);  // block 8 overwrites staged blocks 7-8, read by now
+#pragma unroll
+          for (int k2 = 0; k2 < kLastPer; ++k2) {
+            const int id = lt + k2 * kLoaders;
+            if (id < kNk * 8) put(id / 8, kNb - 1, id % 8, last[k2]);
+          }
+          fence_proxy_async_smem();
+          named_sync(3, kLoaders);
+          if (lt == 0) mbar_arrive(&kfull[st]);
         } else {
           // consecutive threads take consecutive 16-byte chunks of a row (coalesced): chunk c of key
           // kr is 16-byte piece c & 7 of channel block c >> 3; FP8 entries are read as 8 codes and
