@@ -31,10 +31,13 @@
 //   - one warp issues only S, so the next tile's S runs while this tile's
 //     exponentials are taken; softmax thread 0 issues the tile's P V once every
 //     row has stored its P (a named barrier that also decides aborts uniformly);
-//   - loaders look up each tile's source rows just before its copy: TMA when a
+//   - loaders look up each tile's source rows one tile ahead, while the tile
+//     before it is copied (its page-table reads included): TMA when a
 //     tile's rows are contiguous (window rows of the ring, HCA entries of one
-//     page), cp.async through the looked-up rows otherwise (the CSA selection),
-//     FP8 entries widened exactly to bf16.
+//     page), TMA gather of single rows for a bf16 tile of pool rows (the CSA
+//     selection), the codes of an FP8 tile of pool rows staged by cp.async and
+//     widened exactly to bf16 in place, cp.async through the looked-up rows
+//     otherwise.
 // O is rescaled only when a row's running max rises by more than 2^8 (the
 // probabilities stay below 256 in bf16), so most tiles skip it. Window keys are
 // taken in ring-slot order (the softmax does not depend on the order of its
